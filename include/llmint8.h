@@ -1,0 +1,181 @@
+/*
+ * llmint8 — the LLM.int8() mixed-precision linear layer Y = X . W^T on B200
+ * (sm_100a), as a plain C ABI.
+ *
+ * Source of the method: the page "Hugging Face 将 LLM.int8() 8-bit 量化集成进
+ * transformers 与 accelerate" (a translation of the Hugging Face blog post "A
+ * Gentle Introduction to 8-bit Matrix Multiplication for transformers at
+ * scale"). Sections cited below:
+ *   [Q]  "模型量化简介" (Introduction to model quantization): absmax
+ *        quantization (scale 127 / absmax, round, int8 range [-127, 127]) and
+ *        vector-wise quantization dequantized by the outer product of the row
+ *        and column absmax vectors.
+ *   [S]  "LLM.int8() 的简要总结" (A gentle summary of LLM.int8()): the three
+ *        steps - outlier columns of the hidden states to fp16, the rest to an
+ *        int8 matmul, dequantize and add.
+ *   [M]  "MatMul 内部" (Inside the MatMul): threshold "magnitude 6 or greater",
+ *        hidden states quantized per row, weights per output row.
+ *   [U]  "用法" (Usage): the int8 weight CB and its row statistics SCB, and the
+ *        recovery CB * SCB / 127 of fp16 weights for the outlier matmul.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked (device) are CUDA device pointers the CALLER allocated
+ *     and owns. The library never allocates or frees memory, and keeps no
+ *     state besides cached device properties and function pointers.
+ *   - All device pointers must be 16-byte aligned; matrices are dense and
+ *     row-major with the last dimension contiguous. K (cols) must be a
+ *     multiple of 16 and at most LLMINT8_MAX_K (so int32 sums of int8
+ *     products cannot overflow: 133143 * 127^2 < 2^31).
+ *   - Work is queued on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream) and returns without waiting, except where stated.
+ *   - Argument errors are returned before anything is queued. A failed launch
+ *     returns LLMINT8_ERR_CUDA. Kernels never trap: a bounded wait that runs
+ *     out sets a bit in the workspace status word (llmint8_read_status).
+ *   - fp16 inputs must be finite; NaN or Inf inputs are outside the contract.
+ *   - M (rows) == 0 or N == 0 is a no-op that returns LLMINT8_OK.
+ */
+#ifndef LLMINT8_H
+#define LLMINT8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LLMINT8_API __attribute__((visibility("default")))
+#else
+#define LLMINT8_API
+#endif
+
+typedef struct CUstream_st *llmint8_stream_t; /* same type as cudaStream_t */
+
+typedef enum llmint8_status {
+    LLMINT8_OK = 0,
+    LLMINT8_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad flag */
+    LLMINT8_ERR_ALIGNMENT = 2,         /* a pointer is not 16-byte aligned */
+    LLMINT8_ERR_UNSUPPORTED_SHAPE = 3, /* K % 16 != 0, K > LLMINT8_MAX_K, sizes past 2^31 */
+    LLMINT8_ERR_WORKSPACE = 4,         /* workspace smaller than the *_workspace_size() answer */
+    LLMINT8_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    LLMINT8_ERR_DEVICE = 6             /* a kernel reported a failure in the status word */
+} llmint8_status;
+
+#define LLMINT8_MAX_K 133143
+/* Device status word bits (llmint8_read_status). */
+#define LLMINT8_DEV_TIMEOUT_PRODUCER 0x1u
+#define LLMINT8_DEV_TIMEOUT_MMA 0x2u
+#define LLMINT8_DEV_TIMEOUT_EPILOGUE 0x4u
+
+/* Human-readable name of a status code. Never NULL. */
+LLMINT8_API const char *llmint8_status_string(int status);
+
+/* Bytes of workspace needed by llmint8_quantize_rowwise for `rows` x `cols`. */
+LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t rows, int64_t cols);
+
+/* Bytes of workspace needed by llmint8_matmul_mixed for X [M x K], W [N x K]. */
+LLMINT8_API size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* Zero a workspace (a cudaMemsetAsync). A workspace must be zeroed once before
+ * its first use; every call leaves it ready for the next one. */
+LLMINT8_API llmint8_status llmint8_workspace_init(void *workspace, size_t ws_bytes, llmint8_stream_t stream);
+
+/* Synchronously read (and, if clear != 0, reset) the device status word of a
+ * workspace after the stream has finished. *out == 0 means no kernel reported
+ * a failure. Waits for the whole device (cudaDeviceSynchronize). */
+LLMINT8_API llmint8_status llmint8_read_status(void *workspace, size_t ws_bytes, int clear, uint32_t *out);
+
+/*
+ * Row-wise absmax quantization with outlier-column decomposition ([Q], [M]).
+ *
+ *   X_f16        (device) fp16 [rows x cols], read only.
+ *   threshold    t. If t > 0, column c is an outlier when some row holds
+ *                |x| >= t; the outlier columns are OR-ed into outlier_bitmap,
+ *                row_absmax[i] = max |x[i,c]| over the NON-outlier columns c,
+ *                and codes of outlier columns are 0. If t <= 0 (or +inf) there
+ *                is no decomposition: row_absmax is over the whole row.
+ *   codes        (device) int8 [rows x cols] out: round-half-even(x * s) with
+ *                s = 127 / row_absmax[i] computed in fp32 (0 for a zero row).
+ *   row_absmax   (device) fp32 [rows] out (the "SCB" statistics of [U]).
+ *   outlier_bitmap (device) uint32 [ceil(cols/32)] out, bit (c & 31) of word
+ *                c >> 5 set for outlier column c. Required when t > 0; may be
+ *                NULL when t <= 0 (if given, it is cleared). It is written, not
+ *                accumulated: the call clears it first.
+ *   workspace    (device) at least llmint8_quantize_workspace_size(rows, cols)
+ *                bytes, zeroed once before first use.
+ * Weight preparation (offline, [U]) is this call with t <= 0 on W [N x K]:
+ * it yields CB = codes and SCB = row_absmax.
+ */
+LLMINT8_API llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t cols,
+                                        float threshold, int8_t *codes, float *row_absmax,
+                                        uint32_t *outlier_bitmap, void *workspace,
+                                        size_t ws_bytes, llmint8_stream_t stream);
+
+/*
+ * The outlier column set as ascending column indices ([S] step 1).
+ *   outlier_bitmap (device) uint32 [ceil(cols/32)] in (as written above).
+ *   col_idx      (device) int32 [cols] out: the first *count entries are the
+ *                set columns in ascending order; the rest is left untouched.
+ *   d_count      (device) int32 [1] out: |O|, written on the device (no sync).
+ *   h_count      (host, may be NULL) if given, the call waits for the stream
+ *                and copies |O| here.
+ */
+LLMINT8_API llmint8_status llmint8_find_outlier_cols(const uint32_t *outlier_bitmap, int64_t cols,
+                                         int32_t *col_idx, int32_t *d_count, int32_t *h_count,
+                                         llmint8_stream_t stream);
+
+/* Optional outputs of llmint8_matmul_mixed for parity checks. Every pointer is
+ * a device pointer or NULL (not written). */
+typedef struct llmint8_debug {
+    int8_t *codes;      /* [M x K] CX: X's int8 codes after decomposition */
+    float *row_absmax;  /* [M]     SX: X's row absmax over non-outlier columns */
+    int32_t *col_idx;   /* [K]     ascending outlier columns (first |O| valid) */
+    int32_t *count;     /* [1]     |O| */
+    int32_t *acc;       /* [M x N] int32 accumulators of the int8 part (runs the
+                           int8 GEMM a second time with a raw int32 epilogue) */
+} llmint8_debug;
+
+/*
+ * The LLM.int8() linear: Y = X . W^T with mixed-precision decomposition
+ * ([S], [M], [U]):
+ *   O      = outlier columns of X at threshold t (none if t <= 0),
+ *   CX, SX = row-wise int8 codes / absmax of X over the columns not in O,
+ *   acc    = CX . CB^T exactly in int32 (columns in O contribute 0),
+ *   Y[i,j] = fp16( acc[i,j] * SX[i] * SCB[j] / 127^2
+ *                  + sum_{c in O} X[i,c] * Wt[j,c] ),   evaluated in fp32,
+ * where Wt[j,c] = W_f16[j,c] if W_f16 is given ("has fp16 weights"), else
+ * CB[j,c] * SCB[j] / 127 in fp32 (the recovery of [U], per output row).
+ *
+ *   X_f16      (device) fp16 [M x K]
+ *   CB         (device) int8 [N x K], SCB (device) fp32 [N]: W's codes and row
+ *              absmax, from llmint8_quantize_rowwise(W, t <= 0).
+ *   W_f16      (device, may be NULL) fp16 [N x K]
+ *   Y_f16      (device) fp16 [M x N] out
+ *   workspace  (device) >= llmint8_workspace_size(M, N, K) bytes, zeroed once.
+ *   dbg        (host struct of device pointers, may be NULL)
+ * M <= 32 runs the decode kernel (W streamed once, tokens on the MMA N side);
+ * larger M runs the persistent prefill GEMM.
+ */
+LLMINT8_API llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
+                                    const float *SCB, const void *W_f16, int64_t N,
+                                    float threshold, void *Y_f16, void *workspace,
+                                    size_t ws_bytes, const llmint8_debug *dbg,
+                                    llmint8_stream_t stream);
+
+/*
+ * Plain int8 GEMM with int32 output: acc[i,j] = sum_k A[i,k] * B[j,k]
+ * (the int8 product of vector-wise quantization, [Q]).
+ *   A (device) int8 [M x K], B (device) int8 [N x K], acc (device) int32 [M x N].
+ *   workspace: >= llmint8_workspace_size(M, N, K) bytes, zeroed once (only
+ *   its status word is used).
+ */
+LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B, int64_t N,
+                                    int64_t K, int32_t *acc, void *workspace, size_t ws_bytes,
+                                    llmint8_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLMINT8_H */

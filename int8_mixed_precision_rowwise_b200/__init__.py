@@ -1,0 +1,234 @@
+"""Python binding of ``libllmint8.so``, the B200 LLM.int8() linear layer.
+
+The functions below carry the C entry points' names (without the
+``llmint8_`` prefix) and only marshal arguments: torch supplies device
+memory and the current CUDA stream, every step of the computation runs in
+the library's CUDA kernels. There is no CPU path: if the library is missing
+or no CUDA device is present, calls fail loudly.
+
+Method: the LLM.int8() mixed-precision decomposition described on the page
+"Hugging Face 将 LLM.int8() 8-bit 量化集成进 transformers 与 accelerate"
+(sections "模型量化简介", "LLM.int8() 的简要总结", "MatMul 内部", "用法").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "LIB_PATH", "LLMInt8Error", "status_string", "quantize_workspace_size", "workspace_size",
+    "workspace_init", "read_status", "quantize_rowwise", "find_outlier_cols", "matmul_mixed",
+    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
+DEFAULT_THRESHOLD = 6.0
+
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(7)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m int8_mixed_precision_rowwise_b200.build` "
+        "(nvcc, sm_100a). There is no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_ST = ctypes.c_int
+
+
+class _Debug(ctypes.Structure):
+    _fields_ = [("codes", _P), ("row_absmax", _P), ("col_idx", _P), ("count", _P), ("acc", _P)]
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_status_string = _sig("llmint8_status_string", ctypes.c_char_p, [ctypes.c_int])
+_quantize_workspace_size = _sig("llmint8_quantize_workspace_size", ctypes.c_size_t, [_I64, _I64])
+_workspace_size = _sig("llmint8_workspace_size", ctypes.c_size_t, [_I64, _I64, _I64])
+_workspace_init = _sig("llmint8_workspace_init", _ST, [_P, ctypes.c_size_t, _P])
+_read_status = _sig("llmint8_read_status", _ST, [_P, ctypes.c_size_t, ctypes.c_int,
+                                                  ctypes.POINTER(ctypes.c_uint32)])
+_quantize_rowwise = _sig("llmint8_quantize_rowwise", _ST,
+                         [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P])
+_find_outlier_cols = _sig("llmint8_find_outlier_cols", _ST, [_P, _I64, _P, _P, _P, _P])
+_matmul_mixed = _sig("llmint8_matmul_mixed", _ST,
+                     [_P, _I64, _I64, _P, _P, _P, _I64, ctypes.c_float, _P, _P, ctypes.c_size_t,
+                      ctypes.POINTER(_Debug), _P])
+_gemm_s8s8s32 = _sig("llmint8_gemm_s8s8s32", _ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P])
+
+EXPORTED = ("llmint8_status_string", "llmint8_quantize_workspace_size", "llmint8_workspace_size",
+            "llmint8_workspace_init", "llmint8_read_status", "llmint8_quantize_rowwise",
+            "llmint8_find_outlier_cols", "llmint8_matmul_mixed", "llmint8_gemm_s8s8s32")
+
+
+class LLMInt8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def status_string(status: int) -> str:
+    return _status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise LLMInt8Error(status, where)
+
+
+def quantize_workspace_size(rows: int, cols: int) -> int:
+    return int(_quantize_workspace_size(rows, cols))
+
+
+def workspace_size(M: int, N: int, K: int) -> int:
+    return int(_workspace_size(M, N, K))
+
+
+# --------------------------------------------------------------------- torch glue
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(device):
+    torch = _torch()
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(t, name, dtype=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+_workspaces: dict = {}
+
+
+def get_workspace(nbytes: int, device):
+    """A zeroed, cached workspace of at least nbytes on `device` (grown on demand)."""
+    torch = _torch()
+    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def workspace_init(ws) -> None:
+    _check(_workspace_init(ws.data_ptr(), ws.numel(), _stream_ptr(ws.device)), "llmint8_workspace_init")
+
+
+def read_status(ws, clear: bool = True) -> int:
+    out = ctypes.c_uint32(0)
+    _check(_read_status(ws.data_ptr(), ws.numel(), int(clear), ctypes.byref(out)), "llmint8_read_status")
+    return int(out.value)
+
+
+def quantize_rowwise(X, threshold: float = 0.0, codes=None, row_absmax=None, outlier_bitmap=None,
+                     workspace=None):
+    """(codes int8, row_absmax fp32, outlier_bitmap int32 words or None) of fp16 X [rows x cols]."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    rows, cols = X.shape
+    dev = X.device
+    if codes is None:
+        codes = torch.empty((rows, cols), dtype=torch.int8, device=dev)
+    if row_absmax is None:
+        row_absmax = torch.empty(rows, dtype=torch.float32, device=dev)
+    if outlier_bitmap is None and threshold > 0:
+        outlier_bitmap = torch.empty((cols + 31) // 32, dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else get_workspace(quantize_workspace_size(rows, cols), dev)
+    _check(_quantize_rowwise(X.data_ptr(), rows, cols, float(threshold), codes.data_ptr(),
+                             row_absmax.data_ptr(), _ptr(outlier_bitmap), ws.data_ptr(), ws.numel(),
+                             _stream_ptr(dev)), "llmint8_quantize_rowwise")
+    return codes, row_absmax, outlier_bitmap
+
+
+def find_outlier_cols(outlier_bitmap, cols: int, col_idx=None, d_count=None, sync_count: bool = True):
+    """(col_idx int32 [cols], d_count int32 [1], host count or None)."""
+    torch = _torch()
+    dev = outlier_bitmap.device
+    if col_idx is None:
+        col_idx = torch.empty(cols, dtype=torch.int32, device=dev)
+    if d_count is None:
+        d_count = torch.empty(1, dtype=torch.int32, device=dev)
+    h = ctypes.c_int32(-1)
+    _check(_find_outlier_cols(outlier_bitmap.data_ptr(), cols, col_idx.data_ptr(), d_count.data_ptr(),
+                              ctypes.byref(h) if sync_count else None, _stream_ptr(dev)),
+           "llmint8_find_outlier_cols")
+    return col_idx, d_count, (int(h.value) if sync_count else None)
+
+
+def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y=None, workspace=None,
+                 debug: dict | None = None):
+    """Y fp16 [M x N] = LLM.int8()(X fp16 [M x K], W given as CB int8 [N x K] + SCB fp32 [N]).
+
+    ``debug`` may map any of codes/row_absmax/col_idx/count/acc to CUDA tensors
+    the call fills (parity checks)."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    _need_cuda(CB, "CB", torch.int8)
+    _need_cuda(SCB, "SCB", torch.float32)
+    if W_f16 is not None:
+        _need_cuda(W_f16, "W_f16", torch.float16)
+    M, K = X.shape
+    N = CB.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    ws = workspace if workspace is not None else get_workspace(workspace_size(M, N, K), dev)
+    dbg = None
+    if debug:
+        dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")))
+    _check(_matmul_mixed(X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N, float(threshold),
+                         Y.data_ptr(), ws.data_ptr(), ws.numel(), ctypes.byref(dbg) if dbg else None,
+                         _stream_ptr(dev)), "llmint8_matmul_mixed")
+    return Y
+
+
+def gemm_s8s8s32(A, B, acc=None, workspace=None):
+    """int32 [M x N] = A int8 [M x K] . B int8 [N x K]^T."""
+    torch = _torch()
+    _need_cuda(A, "A", torch.int8)
+    _need_cuda(B, "B", torch.int8)
+    M, K = A.shape
+    N = B.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=A.device)
+    ws = workspace if workspace is not None else get_workspace(workspace_size(M, N, K), A.device)
+    _check(_gemm_s8s8s32(A.data_ptr(), M, B.data_ptr(), N, K, acc.data_ptr(), ws.data_ptr(), ws.numel(),
+                         _stream_ptr(A.device)), "llmint8_gemm_s8s8s32")
+    return acc
+
+
+class Int8MixedLinear:
+    """An LLM.int8() linear layer without bias: holds CB/SCB (and optionally the
+    fp16 weight for the outlier columns) and applies matmul_mixed."""
+
+    def __init__(self, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD):
+        self.CB, self.SCB, self.W_f16, self.threshold = CB, SCB, W_f16, threshold
+
+    @classmethod
+    def from_fp16(cls, W, threshold: float = DEFAULT_THRESHOLD, keep_fp16_weights: bool = True):
+        """Quantize W fp16 [N x K] per output row (offline weight preparation)."""
+        CB, SCB, _ = quantize_rowwise(W, 0.0)
+        return cls(CB, SCB, W if keep_fp16_weights else None, threshold)
+
+    def __call__(self, X, Y=None):
+        return matmul_mixed(X, self.CB, self.SCB, self.W_f16, self.threshold, Y=Y)

@@ -1,0 +1,306 @@
+// C-ABI front end: argument checks, workspace layout and launch order for the
+// LLM.int8() linear. Argument errors return before anything is queued.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "llmint8.h"
+#include "internal.h"
+
+namespace llmint8 {
+
+cudaError_t device_info(DeviceInfo *out)
+{
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && have[dev]) {
+        *out = cache[dev];
+        return cudaSuccess;
+    }
+    DeviceInfo d{};
+    d.device = dev;
+    if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+        cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < 64) {
+        cache[dev] = d;
+        have[dev] = true;
+    }
+    *out = d;
+    return cudaSuccess;
+}
+
+} // namespace llmint8
+
+using namespace llmint8;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Thresholds that switch the decomposition off: t <= 0, +inf, NaN.
+float effective_threshold(float t)
+{
+    if (!(t > 0.f) || std::isinf(t))
+        return 0.f;
+    return t;
+}
+
+llmint8_status check_k(int64_t K)
+{
+    if (K <= 0 || K % 16 != 0 || K > LLMINT8_MAX_K)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    return LLMINT8_OK;
+}
+
+llmint8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
+
+} // namespace
+
+extern "C" {
+
+const char *llmint8_status_string(int status)
+{
+    switch (status) {
+    case LLMINT8_OK: return "LLMINT8_OK";
+    case LLMINT8_ERR_INVALID_ARG: return "LLMINT8_ERR_INVALID_ARG: null pointer, negative size or bad flag";
+    case LLMINT8_ERR_ALIGNMENT: return "LLMINT8_ERR_ALIGNMENT: device pointers must be 16-byte aligned";
+    case LLMINT8_ERR_UNSUPPORTED_SHAPE:
+        return "LLMINT8_ERR_UNSUPPORTED_SHAPE: K must be a positive multiple of 16 and at most 133143, sizes "
+               "below 2^31";
+    case LLMINT8_ERR_WORKSPACE: return "LLMINT8_ERR_WORKSPACE: workspace too small";
+    case LLMINT8_ERR_CUDA: return "LLMINT8_ERR_CUDA: a CUDA call or kernel launch failed";
+    case LLMINT8_ERR_DEVICE: return "LLMINT8_ERR_DEVICE: a kernel reported a failure in the status word";
+    default: return "LLMINT8_ERR_UNKNOWN";
+    }
+}
+
+size_t llmint8_quantize_workspace_size(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0)
+        return 0;
+    return carve(nullptr, rows, cols, false, nullptr);
+}
+
+size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    (void)N;
+    if (M < 0 || N < 0 || K < 0)
+        return 0;
+    return carve(nullptr, M, K, true, nullptr);
+}
+
+llmint8_status llmint8_workspace_init(void *workspace, size_t ws_bytes, llmint8_stream_t stream)
+{
+    if (!workspace || ws_bytes < 256)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(workspace))
+        return LLMINT8_ERR_ALIGNMENT;
+    return cuda_status(cudaMemsetAsync(workspace, 0, ws_bytes, stream));
+}
+
+llmint8_status llmint8_read_status(void *workspace, size_t ws_bytes, int clear, uint32_t *out)
+{
+    if (!workspace || !out || ws_bytes < 256)
+        return LLMINT8_ERR_INVALID_ARG;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(out, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear)
+        e = cudaMemset(workspace, 0, sizeof(uint32_t));
+    return cuda_status(e);
+}
+
+llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t cols, float threshold,
+                                        int8_t *codes, float *row_absmax, uint32_t *outlier_bitmap,
+                                        void *workspace, size_t ws_bytes, llmint8_stream_t stream)
+{
+    if (rows < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k(cols);
+    if (st != LLMINT8_OK)
+        return st;
+    if (rows > INT32_MAX || rows * cols > (int64_t)1 << 40)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    const float t = effective_threshold(threshold);
+    if (!X_f16 || !codes || !row_absmax || !workspace || (t > 0.f && !outlier_bitmap))
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X_f16) || !aligned16(codes) || !aligned16(row_absmax) || !aligned16(workspace) ||
+        (outlier_bitmap && !aligned16(outlier_bitmap)))
+        return LLMINT8_ERR_ALIGNMENT;
+    Workspace ws;
+    const size_t need = carve(static_cast<char *>(workspace), rows, cols, false, &ws);
+    if (ws_bytes < need)
+        return LLMINT8_ERR_WORKSPACE;
+    if (rows == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    const size_t nwords = (size_t)((cols + 31) / 32);
+    if (outlier_bitmap) {
+        if ((e = cudaMemsetAsync(outlier_bitmap, 0, nwords * 4, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    }
+    e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.argmax, ws.col_idx,
+                        ws.count, dev, stream);
+    return cuda_status(e);
+}
+
+llmint8_status llmint8_find_outlier_cols(const uint32_t *outlier_bitmap, int64_t cols, int32_t *col_idx,
+                                         int32_t *d_count, int32_t *h_count, llmint8_stream_t stream)
+{
+    if (cols <= 0 || cols > INT32_MAX - 32)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (!outlier_bitmap || !col_idx || !d_count)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(outlier_bitmap) || !aligned16(col_idx) || (reinterpret_cast<uintptr_t>(d_count) & 3u))
+        return LLMINT8_ERR_ALIGNMENT;
+    if ((cols + 31) / 32 * 4 > 200 * 1024)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    cudaError_t e = launch_compact(outlier_bitmap, cols, col_idx, d_count, stream);
+    if (e != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if (h_count) {
+        if ((e = cudaMemcpyAsync(h_count, d_count, sizeof(int32_t), cudaMemcpyDeviceToHost, stream)) !=
+            cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if ((e = cudaStreamSynchronize(stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    }
+    return LLMINT8_OK;
+}
+
+llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
+                                    const float *SCB, const void *W_f16, int64_t N, float threshold,
+                                    void *Y_f16, void *workspace, size_t ws_bytes, const llmint8_debug *dbg,
+                                    llmint8_stream_t stream)
+{
+    if (M < 0 || N < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k(K);
+    if (st != LLMINT8_OK)
+        return st;
+    if (M > INT32_MAX || N > INT32_MAX || M * K > (int64_t)1 << 40 || N * K > (int64_t)1 << 40)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (!X_f16 || !CB || !SCB || !Y_f16 || !workspace)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X_f16) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y_f16) || !aligned16(workspace) ||
+        (W_f16 && !aligned16(W_f16)))
+        return LLMINT8_ERR_ALIGNMENT;
+    if (dbg) {
+        if ((dbg->codes && !aligned16(dbg->codes)) || (dbg->row_absmax && !aligned16(dbg->row_absmax)) ||
+            (dbg->col_idx && !aligned16(dbg->col_idx)) || (dbg->acc && !aligned16(dbg->acc)) ||
+            (dbg->count && (reinterpret_cast<uintptr_t>(dbg->count) & 3u)))
+            return LLMINT8_ERR_ALIGNMENT;
+    }
+    Workspace ws;
+    const size_t need = carve(static_cast<char *>(workspace), M, K, true, &ws);
+    if (ws_bytes < need)
+        return LLMINT8_ERR_WORKSPACE;
+    if (M == 0 || N == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    const float t = effective_threshold(threshold);
+
+    // Clear |O| and the bitmap (one memset: they sit next to each other).
+    char *clear_from = reinterpret_cast<char *>(ws.count);
+    const size_t clear_bytes = (reinterpret_cast<char *>(ws.bitmap) - clear_from) + (size_t)((K + 31) / 32) * 4;
+    if ((e = cudaMemsetAsync(clear_from, 0, clear_bytes, stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if ((e = launch_quantize(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws.argmax, ws.col_idx, ws.count, dev,
+                             stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+
+    GemmArgs g{};
+    g.A = ws.cx;
+    g.B = CB;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.sx = ws.sx;
+    g.sb = SCB;
+    g.X16 = X_f16;
+    g.W16 = W_f16;
+    g.col_idx = ws.col_idx;
+    g.count = ws.count;
+    g.status = ws.status;
+    g.epi = Epilogue::MixedFp16;
+    g.Y = Y_f16;
+    if ((e = launch_gemm(g, dev, stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+
+    if (dbg) {
+        if (dbg->acc) {
+            GemmArgs r = g;
+            r.epi = Epilogue::RawInt32;
+            r.Y = dbg->acc;
+            if ((e = launch_gemm(r, dev, stream)) != cudaSuccess)
+                return LLMINT8_ERR_CUDA;
+        }
+        if (dbg->codes && (e = cudaMemcpyAsync(dbg->codes, ws.cx, (size_t)M * K, cudaMemcpyDeviceToDevice,
+                                               stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if (dbg->row_absmax && (e = cudaMemcpyAsync(dbg->row_absmax, ws.sx, (size_t)M * 4,
+                                                    cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if (dbg->col_idx && (e = cudaMemcpyAsync(dbg->col_idx, ws.col_idx, (size_t)K * 4,
+                                                 cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if (dbg->count && (e = cudaMemcpyAsync(dbg->count, ws.count, 4, cudaMemcpyDeviceToDevice, stream)) !=
+                              cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    }
+    return LLMINT8_OK;
+}
+
+llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B, int64_t N, int64_t K,
+                                    int32_t *acc, void *workspace, size_t ws_bytes, llmint8_stream_t stream)
+{
+    if (M < 0 || N < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k(K);
+    if (st != LLMINT8_OK)
+        return st;
+    if (M > INT32_MAX || N > INT32_MAX)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (!A || !B || !acc || !workspace)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(acc) || !aligned16(workspace))
+        return LLMINT8_ERR_ALIGNMENT;
+    Workspace ws;
+    const size_t need = carve(static_cast<char *>(workspace), M, K, true, &ws);
+    if (ws_bytes < need)
+        return LLMINT8_ERR_WORKSPACE;
+    if (M == 0 || N == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    GemmArgs g{};
+    g.A = A;
+    g.B = B;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.epi = Epilogue::RawInt32;
+    g.Y = acc;
+    g.status = ws.status;
+    return cuda_status(launch_gemm(g, dev, stream));
+}
+
+} // extern "C"

@@ -1,0 +1,558 @@
+// int8 x int8 -> int32 GEMM on the 5th-generation tensor cores (tcgen05,
+// kind::i8) with the LLM.int8() epilogue fused in.
+//
+// The int8 product of the non-outlier part is the vector-wise quantized
+// matmul of page "Hugging Face 将 LLM.int8() 8-bit 量化集成进 transformers 与
+// accelerate", section "模型量化简介" (Introduction to model quantization):
+// rows of X and output rows of W are quantized separately and the int32
+// result is dequantized by the outer product of their absmax vectors. The
+// epilogue adds the fp16 outlier product of section "LLM.int8() 的简要总结"
+// (step 2: outlier columns in fp16; step 3: dequantize and add).
+//
+// Structure (one CTA per SM, 192 threads, persistent over output tiles):
+//   warp 0      TMA producer: 128x128-byte K-major int8 tiles of both
+//               operands into a STAGES-deep shared-memory ring (128B swizzle).
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma kind::i8
+//               (M=128, N=BN, K=32 per instruction) into one of two TMEM
+//               int32 accumulators and commits stage releases / tile done.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator, dequant
+//               acc * SX[i] * SB[j] / 127^2, plus sum over outlier columns
+//               c of X[i,c] * Wt[j,c] in fp32 FMAs, fp16 store. The outlier
+//               operands for the next tile are staged while the tensor cores
+//               run its main loop.
+// SWAP=true is the decode form (few tokens): W takes the MMA M side (128
+// output features per tile) and the tokens the N side (BN = 16 or 32).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include "llmint8.h"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace llmint8 {
+
+namespace {
+
+constexpr int BM = 128;       // MMA M: rows of the A operand per tile
+constexpr int BK = 128;       // K bytes per pipeline stage (one 128-byte swizzle row)
+constexpr int UK = 32;        // K per tcgen05.mma kind::i8
+constexpr int OC = 32;        // outlier columns staged per chunk in the epilogue
+constexpr int NTHREADS = 192; // 6 warps
+constexpr float kInv127Sq = 1.0f / 16129.0f;
+
+struct KParams {
+    int rows_a, rows_b, K;     // operand rows (A on the MMA M side), K in bytes
+    int num_m_blk, num_n_blk, num_kb;
+    int M, N;                  // problem sizes: tokens, output features
+    const float *sx, *sb;
+    const __half *X16, *W16;
+    const int8_t *CB;
+    const int32_t *col_idx, *count;
+    void *Y;
+    uint32_t *status;
+};
+
+template <int BN, int STAGES>
+struct Smem {
+    static constexpr int A_BYTES = BM * BK;
+    static constexpr int B_BYTES = BN * BK;
+    static constexpr int A_OFF = 0;
+    static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
+    static constexpr int SIDE_OFF = B_OFF + STAGES * B_BYTES;          // float [OC][BN]
+    static constexpr int SCALE_OFF = SIDE_OFF + OC * BN * 4;           // float [BN]
+    static constexpr int BAR_OFF = SCALE_OFF + BN * 4;                 // uint64 barriers
+    static constexpr int NBARS = 2 * STAGES + 5;                       // full, empty, tfull[2], tempty[2], drain
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;               // tmem base, abort flag
+    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int ALLOC = BYTES + 1024;                         // slack for 1024-byte alignment
+    static constexpr uint32_t TMEM_COLS = (2 * BN) <= 32 ? 32 : (2 * BN) <= 64 ? 64 : (2 * BN) <= 128 ? 128
+                                         : (2 * BN) <= 256 ? 256 : 512;
+    static_assert(ALLOC <= 232448, "shared memory over the 227 KB per-CTA limit");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+};
+
+__device__ __forceinline__ float wtilde(const KParams &p, int j, int c)
+{
+    // W's outlier column value: the fp16 weight if given, else CB * SCB / 127
+    // per output row (page section "用法", Usage), in fp32.
+    if (p.W16)
+        return __half2float(p.W16[(int64_t)j * p.K + c]);
+    return __fdiv_rn(__fmul_rn((float)p.CB[(int64_t)j * p.K + c], p.sb[j]), 127.0f);
+}
+
+__device__ __forceinline__ void report(const KParams &p, volatile int *s_abort, uint32_t bit)
+{
+    atomicOr(p.status, bit);
+    *s_abort = 1;
+}
+
+template <int BN, int STAGES, bool SWAP, bool RAW>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_gemm_i8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const KParams p)
+{
+    using L = Smem<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *s_side = reinterpret_cast<float *>(smem + L::SIDE_OFF);
+    float *s_scale = reinterpret_cast<float *>(smem + L::SCALE_OFF);
+    const uint32_t bar0 = sbase + L::BAR_OFF;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 4); // one arrival per epilogue warp
+        }
+        mbar_init(drain_bar, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(s_tmem), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int num_tiles = p.num_m_blk * p.num_n_blk;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, armed = 0, armed_phase = 0;
+            constexpr uint32_t TX = (uint32_t)(L::A_BYTES + L::B_BYTES);
+            for (int tile = blockIdx.x; tile < num_tiles && !*s_abort; tile += gridDim.x) {
+                const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_PRODUCER);
+                        break;
+                    }
+                    if (*s_abort)
+                        break;
+                    mbar_arrive_expect_tx(full_bar(stage), TX);
+                    tma_load_2d(sbase + L::A_OFF + stage * L::A_BYTES, &tmA, full_bar(stage), kb * BK, mb * BM);
+                    tma_load_2d(sbase + L::B_OFF + stage * L::B_BYTES, &tmB, full_bar(stage), kb * BK, nb * BN);
+                    armed |= 1u << stage;
+                    armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*s_abort) {
+                // Let every copy this thread started land before the CTA exits.
+                for (int s = 0; s < STAGES; ++s)
+                    if ((armed >> s) & 1u)
+                        mbar_wait(full_bar(s), (armed_phase >> s) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t tph[2] = {0u, 0u};
+            constexpr uint32_t IDESC = idesc_i8(BM, BN);
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*s_abort; tile += gridDim.x, ++local) {
+                const int b = local & 1;
+                if (!mbar_wait(tempty_bar(b), tph[b] ^ 1u)) {
+                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
+                    break;
+                }
+                tph[b] ^= 1u;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+                bool ok = true;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase)) {
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = sbase + L::A_OFF + stage * L::A_BYTES;
+                    const uint32_t b0 = sbase + L::B_OFF + stage * L::B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UK; ++k)
+                        mma_i8(d_tmem, smem_desc_k128(a0 + k * UK), smem_desc_k128(b0 + k * UK), IDESC,
+                               (kb | k) != 0 ? 1u : 0u);
+                    mma_commit(empty_bar(stage)); // stage free once these MMAs have read it
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit(tfull_bar(b)); // accumulator b complete
+            }
+            // Wait for every MMA this thread issued before TMEM is released.
+            mma_commit(drain_bar);
+            if (!mbar_wait(drain_bar, 0u))
+                report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter this warp may read
+        const int et = threadIdx.x - 64;        // 0..127
+        const int r_in_tile = q * 32 + lane;    // accumulator row (A-side row in the tile)
+        const int cnt = RAW ? 0 : min(*p.count, p.K);
+        const bool fast = cnt <= OC;
+        uint32_t tph[2] = {0u, 0u};
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int b = local & 1;
+            const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
+            const int arow = mb * BM + r_in_tile;   // A-operand row of this thread
+            const int brow0 = nb * BN;               // first B-operand row of the tile
+            float own_scale = 0.f;
+            float own_side[OC];
+#pragma unroll
+            for (int k = 0; k < OC; ++k)
+                own_side[k] = 0.f;
+            if (!RAW) {
+                // Stage the outlier operands and scales while the MMAs run.
+                named_barrier_sync(1, 128);
+                for (int idx = et; idx < BN; idx += 128) {
+                    const int r = brow0 + idx;
+                    s_scale[idx] = SWAP ? (r < p.M ? p.sx[r] : 0.f) : (r < p.N ? p.sb[r] : 0.f);
+                }
+                if (fast) {
+                    for (int idx = et; idx < cnt * BN; idx += 128) {
+                        const int k = idx / BN, c = idx - k * BN;
+                        const int r = brow0 + c;
+                        const int col = p.col_idx[k];
+                        float v = 0.f;
+                        if (SWAP) {
+                            if (r < p.M)
+                                v = __half2float(p.X16[(int64_t)r * p.K + col]);
+                        } else {
+                            if (r < p.N)
+                                v = wtilde(p, r, col);
+                        }
+                        s_side[idx] = v;
+                    }
+                }
+                if (SWAP) {
+                    if (arow < p.N) {
+                        own_scale = p.sb[arow];
+                        if (fast) {
+#pragma unroll
+                            for (int k = 0; k < OC; ++k)
+                                if (k < cnt)
+                                    own_side[k] = wtilde(p, arow, p.col_idx[k]);
+                        }
+                    }
+                } else {
+                    if (arow < p.M) {
+                        own_scale = p.sx[arow];
+                        if (fast) {
+#pragma unroll
+                            for (int k = 0; k < OC; ++k)
+                                if (k < cnt)
+                                    own_side[k] = __half2float(p.X16[(int64_t)arow * p.K + p.col_idx[k]]);
+                        }
+                    }
+                }
+                named_barrier_sync(1, 128);
+            }
+
+            // All 128 epilogue threads leave together if any of them gave up,
+            // so no thread is left waiting at a named barrier.
+            const bool got = mbar_wait(tfull_bar(b), tph[b]);
+            if (named_barrier_or(1, 128, !got)) {
+                if (!got)
+                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                break;
+            }
+            tph[b] ^= 1u;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+
+            if constexpr (!SWAP) {
+                const int i = arow;
+#pragma unroll 1
+                for (int g = 0; g < BN / 32; ++g) {
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(tbase + g * 32, acc);
+                    tmem_wait_ld();
+                    const int j0 = brow0 + g * 32;
+                    if constexpr (RAW) {
+                        int32_t *Yr = reinterpret_cast<int32_t *>(p.Y) + (int64_t)i * p.N;
+                        if (i < p.M) {
+                            if (j0 + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+                                for (int c = 0; c < 32; c += 4)
+                                    *reinterpret_cast<uint4 *>(Yr + j0 + c) =
+                                        make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                            } else {
+                                for (int c = 0; c < 32; ++c)
+                                    if (j0 + c < p.N)
+                                        Yr[j0 + c] = (int32_t)acc[c];
+                            }
+                        }
+                        continue;
+                    }
+                    float y[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
+                    if (fast) {
+#pragma unroll
+                        for (int k = 0; k < OC; ++k) {
+                            if (k < cnt) {
+                                const float xv = own_side[k];
+                                const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                                for (int c4 = 0; c4 < 8; ++c4) {
+                                    const float4 w = wrow[c4];
+                                    y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                    y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                    y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                    y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                                }
+                            }
+                        }
+                    } else {
+                        // More outlier columns than one staged chunk holds.
+                        for (int ch = 0; ch < cnt; ch += OC) {
+                            const int nk = min(OC, cnt - ch);
+                            named_barrier_sync(1, 128);
+                            for (int idx = et; idx < nk * 32; idx += 128) {
+                                const int k = idx >> 5, c = idx & 31;
+                                const int j = j0 + c;
+                                s_side[idx] = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
+                            }
+                            named_barrier_sync(1, 128);
+                            for (int k = 0; k < nk; ++k) {
+                                const float xv =
+                                    i < p.M ? __half2float(p.X16[(int64_t)i * p.K + p.col_idx[ch + k]]) : 0.f;
+#pragma unroll
+                                for (int c = 0; c < 32; ++c)
+                                    y[c] = fmaf(xv, s_side[k * 32 + c], y[c]);
+                            }
+                        }
+                    }
+                    if (i < p.M) {
+                        __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
+                        if (j0 + 32 <= p.N && (p.N & 7) == 0) {
+#pragma unroll
+                            for (int c = 0; c < 32; c += 8) {
+                                uint4 pk;
+                                __half2 *h = reinterpret_cast<__half2 *>(&pk);
+                                h[0] = __floats2half2_rn(y[c + 0], y[c + 1]);
+                                h[1] = __floats2half2_rn(y[c + 2], y[c + 3]);
+                                h[2] = __floats2half2_rn(y[c + 4], y[c + 5]);
+                                h[3] = __floats2half2_rn(y[c + 6], y[c + 7]);
+                                *reinterpret_cast<uint4 *>(Yr + j0 + c) = pk;
+                            }
+                        } else {
+                            for (int c = 0; c < 32; ++c)
+                                if (j0 + c < p.N)
+                                    Yr[j0 + c] = __float2half_rn(y[c]);
+                        }
+                    }
+                }
+            } else {
+                // Decode form: this thread owns output feature j = arow; the
+                // accumulator columns are tokens brow0 .. brow0 + BN - 1.
+                const int j = arow;
+                uint32_t acc[BN];
+                if constexpr (BN == 32) {
+                    tmem_ld_32x32b_x32(tbase, acc);
+                } else {
+                    tmem_ld_32x32b_x16(tbase, acc);
+                }
+                tmem_wait_ld();
+                if constexpr (RAW) {
+                    if (j < p.N) {
+                        int32_t *Yc = reinterpret_cast<int32_t *>(p.Y) + j;
+#pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if (brow0 + c < p.M)
+                                Yc[(int64_t)(brow0 + c) * p.N] = (int32_t)acc[c];
+                    }
+                } else {
+                    float y[BN];
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
+                    if (fast) {
+#pragma unroll
+                        for (int k = 0; k < OC; ++k) {
+                            if (k < cnt) {
+                                const float wv = own_side[k];
+#pragma unroll
+                                for (int c = 0; c < BN; ++c)
+                                    y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                            }
+                        }
+                    } else {
+                        for (int ch = 0; ch < cnt; ch += OC) {
+                            const int nk = min(OC, cnt - ch);
+                            named_barrier_sync(1, 128);
+                            for (int idx = et; idx < nk * BN; idx += 128) {
+                                const int k = idx / BN, c = idx - k * BN;
+                                const int r = brow0 + c;
+                                s_side[idx] =
+                                    r < p.M ? __half2float(p.X16[(int64_t)r * p.K + p.col_idx[ch + k]]) : 0.f;
+                            }
+                            named_barrier_sync(1, 128);
+                            for (int k = 0; k < nk; ++k) {
+                                const float wv = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
+#pragma unroll
+                                for (int c = 0; c < BN; ++c)
+                                    y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                            }
+                        }
+                    }
+                    if (j < p.N) {
+                        __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
+#pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if (brow0 + c < p.M)
+                                Yc[(int64_t)(brow0 + c) * p.N] = __float2half_rn(y[c]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(tempty_bar(b));
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major int8 [rows x K] as a 2-D tensor map with a 128-byte x box_rows box.
+bool make_map_i8(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, bool SWAP, bool RAW>
+cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+{
+    using L = Smem<BN, STAGES>;
+    auto kern = k_gemm_i8<BN, STAGES, SWAP, RAW>;
+    static std::atomic<uint64_t> configured{0};
+    const uint64_t bit = 1ull << (dev.device & 63);
+    if (!(configured.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+        if (e != cudaSuccess)
+            return e;
+        configured.fetch_or(bit);
+    }
+    // A operand rides the MMA M side (128 rows per tile).
+    const int8_t *Aop = SWAP ? a.B : a.A;
+    const int8_t *Bop = SWAP ? a.A : a.B;
+    const int64_t rows_a = SWAP ? a.N : a.M;
+    const int64_t rows_b = SWAP ? a.M : a.N;
+    CUtensorMap ta, tb;
+    if (!make_map_i8(&ta, Aop, rows_a, a.K, BM) || !make_map_i8(&tb, Bop, rows_b, a.K, BN))
+        return cudaErrorInvalidValue;
+    KParams p;
+    p.rows_a = (int)rows_a;
+    p.rows_b = (int)rows_b;
+    p.K = (int)a.K;
+    p.num_m_blk = (int)((rows_a + BM - 1) / BM);
+    p.num_n_blk = (int)((rows_b + BN - 1) / BN);
+    p.num_kb = (int)((a.K + BK - 1) / BK);
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.sx = a.sx;
+    p.sb = a.sb;
+    p.X16 = reinterpret_cast<const __half *>(a.X16);
+    p.W16 = reinterpret_cast<const __half *>(a.W16);
+    p.CB = a.B;
+    p.col_idx = a.col_idx;
+    p.count = a.count;
+    p.Y = a.Y;
+    p.status = a.status;
+    const int tiles = p.num_m_blk * p.num_n_blk;
+    const int grid = std::min(tiles, dev.num_sms);
+    kern<<<grid, NTHREADS, L::ALLOC, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+} // namespace
+
+cudaError_t launch_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (a.M <= 0 || a.N <= 0)
+        return cudaSuccess;
+    const bool raw = a.epi == Epilogue::RawInt32;
+    if (a.M <= 16)
+        return raw ? run<16, 8, true, true>(a, dev, stream) : run<16, 8, true, false>(a, dev, stream);
+    if (a.M <= 32)
+        return raw ? run<32, 8, true, true>(a, dev, stream) : run<32, 8, true, false>(a, dev, stream);
+    return raw ? run<256, 4, false, true>(a, dev, stream) : run<256, 4, false, false>(a, dev, stream);
+}
+
+} // namespace llmint8

@@ -44,20 +44,17 @@
 int64_t oracle_outlier_cols(const float *X, int64_t rows, int64_t cols, float t,
                             uint8_t *is_outlier)
 {
-    int64_t count = 0;
-    for (int64_t c = 0; c < cols; ++c) {
-        uint8_t hit = 0;
-        if (t > 0.0f) {
-            for (int64_t i = 0; i < rows; ++i) {
-                if (fabsf(X[i * cols + c]) >= t) {
-                    hit = 1;
-                    break;
-                }
-            }
-        }
-        is_outlier[c] = hit;
-        count += hit;
+    for (int64_t c = 0; c < cols; ++c)
+        is_outlier[c] = 0;
+    if (t > 0.0f) {
+        for (int64_t i = 0; i < rows; ++i)
+            for (int64_t c = 0; c < cols; ++c)
+                if (fabsf(X[i * cols + c]) >= t)
+                    is_outlier[c] = 1;
     }
+    int64_t count = 0;
+    for (int64_t c = 0; c < cols; ++c)
+        count += is_outlier[c];
     return count;
 }
 

@@ -1,0 +1,123 @@
+"""Host-side checks of the C-ABI library: it loads without a GPU, exports
+every entry point the header declares, sizes its workspace, and rejects bad
+arguments before queuing any GPU work. Fake (never dereferenced) pointer
+values stand in for device memory; every call here returns before any CUDA
+call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "llmint8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from int8_mixed_precision_rowwise_b200 import build as b
+    b.build()
+    import int8_mixed_precision_rowwise_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LLMINT8_API\s+[\w\s\*]+?\b(llmint8_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for need in ("llmint8_quantize_rowwise", "llmint8_find_outlier_cols", "llmint8_matmul_mixed"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    cdll = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(cdll, name), name
+    assert set(lib.EXPORTED) == set(declared_functions())
+
+
+def test_status_strings(lib):
+    assert lib.status_string(0) == "LLMINT8_OK"
+    for s in range(1, 7):
+        assert lib.status_string(s).startswith("LLMINT8_ERR_")
+    assert lib.status_string(99) == "LLMINT8_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    M, N, K = 2048, 16384, 4096
+    need = lib.workspace_size(M, N, K)
+    # at least CX + SX + argmax + col_idx + bitmap
+    assert need >= M * K + 4 * M + 4 * M + 4 * K + K // 8
+    assert need % 256 == 0
+    assert lib.workspace_size(M, N, K) == lib.workspace_size(M, 1, K)  # W is not staged
+    assert lib.quantize_workspace_size(M, K) < need
+    assert lib.workspace_size(-1, N, K) == 0
+
+
+A = 0x10000  # aligned fake device address
+P = ctypes.c_void_p
+
+
+def _mm(lib, X=A, M=64, K=128, CB=A, SCB=A, W=None, N=64, t=6.0, Y=A, ws=A, wsb=None):
+    wsb = lib.workspace_size(M, N, K) if wsb is None else wsb
+    return lib._matmul_mixed(X, M, K, CB, SCB, W, N, t, Y, ws, wsb, None, None)
+
+
+def test_matmul_argument_errors(lib):
+    assert _mm(lib, K=100) == lib.ERR_UNSUPPORTED_SHAPE     # K % 16
+    assert _mm(lib, K=0) == lib.ERR_UNSUPPORTED_SHAPE
+    assert _mm(lib, K=133152) == lib.ERR_UNSUPPORTED_SHAPE  # > LLMINT8_MAX_K
+    assert _mm(lib, M=-1) == lib.ERR_INVALID_ARG
+    assert _mm(lib, X=None) == lib.ERR_INVALID_ARG
+    assert _mm(lib, CB=None) == lib.ERR_INVALID_ARG
+    assert _mm(lib, SCB=None) == lib.ERR_INVALID_ARG
+    assert _mm(lib, Y=None) == lib.ERR_INVALID_ARG
+    assert _mm(lib, ws=None) == lib.ERR_INVALID_ARG
+    assert _mm(lib, X=A + 8) == lib.ERR_ALIGNMENT
+    assert _mm(lib, W=A + 2) == lib.ERR_ALIGNMENT
+    assert _mm(lib, Y=A + 4) == lib.ERR_ALIGNMENT
+    assert _mm(lib, wsb=1024) == lib.ERR_WORKSPACE
+    assert _mm(lib, M=0) == lib.OK   # empty: no-op, nothing queued
+    assert _mm(lib, N=0) == lib.OK
+
+
+def test_quantize_argument_errors(lib):
+    q = lib._quantize_rowwise
+    ws = lib.quantize_workspace_size(32, 64)
+    assert q(A, 32, 60, 6.0, A, A, A, A, ws, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert q(A, 32, 64, 6.0, A, A, None, A, ws, None) == lib.ERR_INVALID_ARG     # bitmap needed when t > 0
+    assert q(A, 32, 64, 6.0, A, A + 1, A, A, ws, None) == lib.ERR_ALIGNMENT
+    assert q(A, 32, 64, 6.0, A, A, A, A, 16, None) == lib.ERR_WORKSPACE
+    assert q(A, 0, 64, 6.0, A, A, A, A, ws, None) == lib.OK
+    assert q(A, 0, 64, 0.0, A, A, None, A, ws, None) == lib.OK                   # no bitmap when t <= 0
+
+
+def test_find_outlier_cols_argument_errors(lib):
+    f = lib._find_outlier_cols
+    assert f(None, 64, A, A, None, None) == lib.ERR_INVALID_ARG
+    assert f(A, 0, A, A, None, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert f(A + 4, 64, A, A, None, None) == lib.ERR_ALIGNMENT
+
+
+def test_gemm_argument_errors(lib):
+    g = lib._gemm_s8s8s32
+    ws = lib.workspace_size(64, 64, 128)
+    assert g(A, 64, A, 64, 120, A, A, ws, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert g(A, 64, None, 64, 128, A, A, ws, None) == lib.ERR_INVALID_ARG
+    assert g(A, 64, A, 64, 128, A + 8, A, ws, None) == lib.ERR_ALIGNMENT
+    assert g(A, 64, A, 64, 128, A, A, 8, None) == lib.ERR_WORKSPACE
+    assert g(A, 0, A, 64, 128, A, A, ws, None) == lib.OK
+
+
+def test_no_cpu_fallback(lib):
+    """Tensors on the CPU are refused: the library has no host compute path."""
+    import torch
+    X = torch.zeros((4, 16), dtype=torch.float16)
+    with pytest.raises(TypeError):
+        lib.quantize_rowwise(X, 6.0)
+    with pytest.raises(TypeError):
+        lib.matmul_mixed(X, torch.zeros((4, 16), dtype=torch.int8), torch.zeros(4))

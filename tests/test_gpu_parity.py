@@ -1,0 +1,362 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle.
+
+Bar (the pages' definition, see the oracle): int8 codes, row absmax (as fp32
+bits), the outlier column set and the int32 accumulators are bit-exact; the
+fp16 output satisfies |y - y_ref| <= 1e-2 + 2e-3 |y_ref| elementwise, with
+y_ref the oracle's fp64 value.
+
+Sizes here span several 128x256 output tiles with ragged edges in M, N and
+K, so the oracle finishes in seconds; the full-size workloads are compared on
+sampled rows and columns the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from synthetic import Linear, make_activations, make_random, make_weight
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 1e-2, 2e-3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import int8_mixed_precision_rowwise_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def dev(lib):
+    return torch.device("cuda", 0)
+
+
+def to_dev(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def bitmap_to_mask(words: np.ndarray, cols: int) -> np.ndarray:
+    bits = np.unpackbits(words.astype("<u4").view(np.uint8), bitorder="little")
+    return bits[:cols].astype(np.uint8)
+
+
+def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, what=""):
+    y = y_gpu.astype(np.float64)
+    err = np.abs(y - y_ref)
+    tol = ATOL + RTOL * np.abs(y_ref)
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst err "
+                           f"{err.max():.4g} at {np.unravel_index(np.argmax(err - tol), err.shape)}")
+
+
+def gpu_mixed(lib, dev, X16, W16, t, give_w16=True, with_debug=True):
+    X = to_dev(X16, dev)
+    W = to_dev(W16, dev)
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    M, K = X16.shape
+    N = W16.shape[0]
+    dbg = None
+    if with_debug:
+        dbg = dict(codes=torch.empty((M, K), dtype=torch.int8, device=dev),
+                   row_absmax=torch.empty(M, dtype=torch.float32, device=dev),
+                   col_idx=torch.full((K,), -1, dtype=torch.int32, device=dev),
+                   count=torch.empty(1, dtype=torch.int32, device=dev),
+                   acc=torch.empty((M, N), dtype=torch.int32, device=dev))
+    Y = lib.matmul_mixed(X, CB, SCB, W if give_w16 else None, t, debug=dbg)
+    torch.cuda.synchronize()
+    out = dict(Y=Y.cpu().numpy(), CB=CB.cpu().numpy(), SB=SCB.cpu().numpy())
+    if dbg:
+        n = int(dbg["count"].item())
+        out.update(CX=dbg["codes"].cpu().numpy(), SX=dbg["row_absmax"].cpu().numpy(),
+                   O=dbg["col_idx"][:n].cpu().numpy().astype(np.int64), acc=dbg["acc"].cpu().numpy())
+    return out
+
+
+def check_full(lib, dev, oracle_mod, X16, W16, t, give_w16=True):
+    g = gpu_mixed(lib, dev, X16, W16, t, give_w16)
+    r = oracle_mod.matmul_mixed(X16, t, W=W16, use_fp16_weight_cols=give_w16)
+    assert np.array_equal(g["CB"], r["CB"]), "weight codes"
+    assert np.array_equal(g["SB"].view(np.uint32), r["SB"].view(np.uint32)), "weight absmax bits"
+    assert np.array_equal(g["O"], r["O"]), f"outlier columns {g['O']} vs {r['O']}"
+    assert np.array_equal(g["SX"].view(np.uint32), r["SX"].view(np.uint32)), "row absmax bits"
+    assert np.array_equal(g["CX"], r["CX"]), "activation codes"
+    assert np.array_equal(g["acc"], r["acc"]), "int32 accumulators"
+    assert_y_close(g["Y"], r["Y"], "Y")
+    return g, r
+
+
+# ------------------------------------------------------------------ quantizer
+
+@pytest.mark.parametrize("M,K,nout,scale", [(8, 64, 2, 20.0), (300, 1024, 5, 40.0), (513, 4096, 8, 40.0),
+                                            (64, 14336, 6, 60.0), (9, 57344, 29, 60.0), (3, 16, 1, 60.0)])
+def test_quantize_rowwise_matches_oracle(lib, dev, oracle_mod, M, K, nout, scale):
+    X16, _ = make_activations(Linear("q", M, 0, K, nout, scale), seed=M + K)
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
+    mask = oracle_mod.outlier_mask(X16, 6.0)
+    c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_quantizer_workload_full(lib, dev, oracle_mod):
+    """The 4096 x 4096 quantizer workload (8 columns x40), compared in full."""
+    lin = synthetic.QUANT_4096.linears[0]
+    X16, cols = make_activations(lin, seed=0)
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
+    mask = oracle_mod.outlier_mask(X16, 6.0)
+    assert set(cols.tolist()) <= set(np.flatnonzero(mask).tolist())
+    c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), lin.K), mask)
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_quantize_threshold_off_is_plain_absmax(lib, dev, oracle_mod):
+    W16 = make_random((777, 1024), seed=7, scale=0.02)
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(W16, dev), 0.0)
+    c_ref, a_ref = oracle_mod.quantize_rowwise(W16, None)
+    assert bm is None
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_quantize_worked_example(lib, dev):
+    """The pages' absmax example (padded to 16 columns with zeros)."""
+    x = np.zeros((1, 16), dtype=np.float16)
+    x[0, :8] = [1.2, -0.5, -4.3, 1.2, -3.1, 0.8, 2.4, 5.4]
+    codes, absmax, _ = lib.quantize_rowwise(to_dev(x, dev), 0.0)
+    assert codes.cpu().numpy()[0, :8].tolist() == [28, -12, -101, 28, -73, 19, 56, 127]
+
+
+def test_quantize_edge_rows(lib, dev, oracle_mod):
+    """Zero rows, rows made only of outliers, exact-threshold values, .5 ties,
+    and rows whose maximum sits in a column that is an outlier only because
+    of another row (the fix-up path)."""
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((200, 256)).astype(np.float32)
+    X[3] = 0.0
+    X[4] = 7.0
+    X[5, 10] = 6.0                       # exactly the threshold: outlier column 10
+    X[6] = 0.0
+    X[6, :3] = [127.0, 2.5, 3.5]         # ties: s = 1
+    X[:, 40] *= 0.1
+    X[7, 40] = 50.0                      # column 40 outlier because of row 7 ...
+    X[8:100, 40] = 5.5                   # ... and the maximum of rows 8..99 sits there
+    X[150:, 77] = 5.9                    # column 77 never reaches 6: it stays in the int8 part
+    X16 = X.astype(np.float16)
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
+    mask = oracle_mod.outlier_mask(X16, 6.0)
+    c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+    assert mask[10] and mask[40] and not mask[77]
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 256), mask)
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_find_outlier_cols(lib, dev):
+    K = 14336
+    rng = np.random.default_rng(9)
+    for n in (0, 1, 29, 700):
+        cols = np.sort(rng.choice(K, n, replace=False))
+        mask = np.zeros(K, dtype=np.uint8)
+        mask[cols] = 1
+        words = np.packbits(mask, bitorder="little").view("<u4").astype(np.int32)
+        col_idx, d_count, h = lib.find_outlier_cols(to_dev(words, dev), K)
+        assert h == n and int(d_count.item()) == n
+        assert np.array_equal(col_idx[:n].cpu().numpy(), cols)
+
+
+# ------------------------------------------------------------------ int8 GEMM
+
+@pytest.mark.parametrize("M,N,K", [(1, 300, 512), (8, 200, 256), (17, 129, 1040), (32, 136, 768),
+                                   (33, 257, 1024), (300, 520, 1040), (128, 256, 128), (257, 513, 80),
+                                   (64, 64, 16)])
+def test_gemm_s8s8s32_exact(lib, dev, oracle_mod, M, N, K):
+    rng = np.random.default_rng(M * 7 + N)
+    A = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+    B = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+    acc = lib.gemm_s8s8s32(to_dev(A, dev), to_dev(B, dev))
+    assert np.array_equal(acc.cpu().numpy(), oracle_mod.int8_matmul(A, B))
+
+
+def test_gemm_int32_margin(lib, dev):
+    """K = 57344 with every code at +-127: the sums reach 924,901,376 exactly."""
+    K = 57344
+    A = np.full((40, K), 127, dtype=np.int8)
+    A[1::2] = -127
+    B = np.full((24, K), 127, dtype=np.int8)
+    B[::3] = -127
+    acc = lib.gemm_s8s8s32(to_dev(A, dev), to_dev(B, dev)).cpu().numpy()
+    ref = (np.where(np.arange(40) % 2, -1, 1)[:, None] * np.where(np.arange(24) % 3 == 0, -1, 1)[None, :]
+           * K * 127 * 127)
+    assert np.array_equal(acc.astype(np.int64), ref)
+
+
+def test_gemm_matches_torch_int_mm(lib, dev):
+    """An independent library check of the int32 product at a tile-spanning size."""
+    rng = np.random.default_rng(1)
+    A = torch.from_numpy(rng.integers(-127, 128, size=(512, 2048), dtype=np.int8)).to(dev)
+    B = torch.from_numpy(rng.integers(-127, 128, size=(768, 2048), dtype=np.int8)).to(dev)
+    acc = lib.gemm_s8s8s32(A, B)
+    ref = torch._int_mm(A, B.t().contiguous())
+    assert torch.equal(acc, ref)
+
+
+# ------------------------------------------------------------------ full linear
+
+def test_tiny_workload(lib, dev, oracle_mod):
+    lin = synthetic.TINY.linears[0]
+    X16, W16, _ = synthetic.make_problem(lin, seed=0)
+    g, r = check_full(lib, dev, oracle_mod, X16, W16, 6.0)
+    assert g["O"].tolist() == [5, 37]
+
+
+@pytest.mark.parametrize("M,N,K,nout,give_w16", [
+    (333, 777, 1024, 5, True), (333, 777, 1024, 5, False), (129, 300, 2048, 40, True),
+    (1, 640, 1024, 6, False), (8, 640, 1024, 6, True), (16, 200, 512, 3, False), (17, 640, 1024, 6, True),
+    (32, 640, 1024, 6, False), (256, 512, 256, 0, True), (200, 384, 80, 2, True)])
+def test_matmul_mixed_matches_oracle(lib, dev, oracle_mod, M, N, K, nout, give_w16):
+    lin = Linear("t", M, N, K, nout, 60.0)
+    X16, cols = make_activations(lin, seed=M + N)
+    W16 = make_weight(lin, seed=K)
+    g, r = check_full(lib, dev, oracle_mod, X16, W16, 6.0, give_w16)
+    assert set(cols.tolist()) <= set(r["O"].tolist())
+
+
+def test_threshold_off_and_no_outliers(lib, dev, oracle_mod):
+    X16 = make_random((150, 512), seed=3)
+    W16 = make_random((300, 512), seed=4, scale=0.02)
+    check_full(lib, dev, oracle_mod, X16, W16, 0.0)
+    g, _ = check_full(lib, dev, oracle_mod, X16, W16, 6.0)     # N(0,1): nothing reaches 6
+    assert g["O"].size == 0
+
+
+@pytest.mark.parametrize("M", [48, 7])
+def test_all_columns_outliers(lib, dev, oracle_mod, M):
+    """A tiny threshold sends every column to the fp16 side (more outlier
+    columns than the epilogue stages at once)."""
+    X16 = make_random((M, 96), seed=11)
+    W16 = make_random((136, 96), seed=12, scale=0.02)
+    g, r = check_full(lib, dev, oracle_mod, X16, W16, 1e-3)
+    assert g["O"].size == 96 and not g["CX"].any()
+
+
+def test_repeat_calls_identical(lib, dev):
+    lin = Linear("t", 300, 600, 1024, 4, 60.0)
+    X16, _ = make_activations(lin, seed=1)
+    W16 = make_weight(lin, seed=1)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    layer = lib.Int8MixedLinear.from_fp16(W)
+    y1 = layer(X).clone()
+    y2 = layer(X)
+    assert torch.equal(y1, y2)
+
+
+def test_cuda_graph_capture(lib, dev):
+    lin = Linear("t", 256, 512, 1024, 4, 60.0)
+    X16, _ = make_activations(lin, seed=2)
+    W16 = make_weight(lin, seed=2)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    layer = lib.Int8MixedLinear.from_fp16(W)
+    ref = layer(X).clone()
+    Y = torch.empty_like(ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer(X, Y=Y)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer(X, Y=Y)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y, ref)
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+
+def sampled_check(lib, dev, oracle_mod, X, W, t, give_w16, rows, cols):
+    """Run the layer on device tensors X [M x K] and W [N x K]; compare the
+    outlier set and SX in full, CX / acc / Y on the sampled rows x columns,
+    and CB / SB on the sampled weight rows, against the oracle on host copies."""
+    M, K = X.shape
+    N = W.shape[0]
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    dbg = dict(codes=torch.empty((M, K), dtype=torch.int8, device=dev),
+               row_absmax=torch.empty(M, dtype=torch.float32, device=dev),
+               col_idx=torch.empty(K, dtype=torch.int32, device=dev),
+               count=torch.empty(1, dtype=torch.int32, device=dev),
+               acc=torch.empty((M, N), dtype=torch.int32, device=dev))
+    Y = lib.matmul_mixed(X, CB, SCB, W if give_w16 else None, t, debug=dbg)
+    torch.cuda.synchronize()
+    Xh = X.cpu().numpy()
+    O = oracle_mod.outlier_cols(Xh, t)
+    n = int(dbg["count"].item())
+    assert np.array_equal(dbg["col_idx"][:n].cpu().numpy(), O)
+    cx_ref, sx_ref = oracle_mod.quantize_rowwise(Xh[rows], O)
+    assert np.array_equal(dbg["row_absmax"].cpu().numpy()[rows].view(np.uint32), sx_ref.view(np.uint32))
+    assert np.array_equal(dbg["codes"][rows].cpu().numpy(), cx_ref)
+    Wh = W[cols].cpu().numpy()
+    cb_ref, sb_ref = oracle_mod.quantize_weight(Wh)
+    assert np.array_equal(CB[cols].cpu().numpy(), cb_ref)
+    assert np.array_equal(SCB[cols].cpu().numpy().view(np.uint32), sb_ref.view(np.uint32))
+    acc_ref = oracle_mod.int8_matmul(cx_ref, cb_ref)
+    acc = dbg["acc"][rows][:, cols].cpu().numpy()
+    assert np.array_equal(acc, acc_ref)
+    wt = oracle_mod.outlier_weight(O, len(cols), K, W=Wh if give_w16 else None, CB=cb_ref, SB=sb_ref)
+    y_ref = oracle_mod.mixed_output(acc_ref, sx_ref, sb_ref, Xh[rows], O, wt)
+    assert_y_close(Y[rows][:, cols].cpu().numpy(), y_ref, "Y sampled")
+    return O
+
+
+def _samples(M, N, seed, nrows=8, ncols=96):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, min(nrows, M), replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, min(ncols, N), replace=False)]))
+    return rows, cols
+
+
+def test_prefill_workload_sampled(lib, dev, oracle_mod):
+    """Prefill, 7B-class: X [2048 x 4096] with 4 columns x60, W [16384 x 4096]."""
+    lin = synthetic.PREFILL_7B.linears[0]
+    X16, cols = make_activations(lin, seed=0)
+    W16 = make_weight(lin, seed=0)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    rows, jcols = _samples(lin.M, lin.N, 3)
+    O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols)
+    assert set(cols.tolist()) <= set(O.tolist())
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_decode_workload_sampled(lib, dev, oracle_mod, M):
+    """Decode at BLOOM width: X [M x 14336], W int8-prequantized [14336 x 14336]
+    (outlier columns of W recovered as CB * SCB / 127)."""
+    lin = synthetic.decode_bloom(M).linears[0]
+    X, W, cols = synthetic.torch_device_problem(lin, seed=M, device=dev)
+    rows, jcols = _samples(lin.M, lin.N, M, ncols=160)
+    O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, False, rows, jcols)
+    assert set(cols.tolist()) <= set(O.tolist())
+
+
+@pytest.mark.parametrize("name", ["qkv", "attn_out", "fc1", "fc2"])
+def test_bloom_block_linear_sampled(lib, dev, oracle_mod, name):
+    lin = {l.name: l for l in synthetic.BLOOM_BLOCK_2048.linears}[name]
+    seed = {"qkv": 11, "attn_out": 12, "fc1": 13, "fc2": 14}[name]
+    X, W, cols = synthetic.torch_device_problem(lin, seed=seed, device=dev)
+    rows, jcols = _samples(lin.M, lin.N, 7, nrows=6, ncols=64)
+    O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols)
+    assert set(cols.tolist()) <= set(O.tolist())
+    del X, W
+    torch.cuda.empty_cache()
+
+
+def test_status_word_clean(lib, dev):
+    """No kernel reported a timed-out wait during this module."""
+    from int8_mixed_precision_rowwise_b200 import _workspaces
+    for ws in _workspaces.values():
+        assert lib.read_status(ws, clear=False) == 0
