@@ -1,0 +1,437 @@
+"""Benchmark of the LLM.int8() mixed-precision linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+
+One step = the four BLOOM-176B block linears (QKV 43008x14336, attn-out
+14336x14336, fc1 57344x14336, fc2 14336x57344) at 2048 tokens, each a full
+llmint8_matmul_mixed call: fused quantizer + outlier detection, fix-up and
+compaction, and the tcgen05 int8 GEMM with the fused dequant + fp16 outlier
+epilogue. Inputs are seeded synthetic data with the workload's outlier columns
+(~0.05% of hidden columns x60), threshold 6.0, weights random N(0, 0.02)
+quantized once per output row before timing (offline weight preparation).
+
+Metric: int8-mixed linear TOPS = sum of 2*M*N*K over the four linears per
+step / step time. Every linear's int8 weight (205-822 MB) is larger than L2,
+so no explicit flush is needed between iterations.
+
+--impl reference times the CPU oracle (plain single-threaded C, the
+definition the GPU path is checked against) on a bounded sample of the same
+workload: all 2048 tokens against a slice of each weight's output rows.
+
+Multi-GPU: the layer has no exchange step on this path; `--gpus N` (under
+torchrun) runs one independent replica per GPU and reports the aggregate.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+WORKLOAD = synthetic.BLOOM_BLOCK_2048
+METRIC = "int8-mixed linear TOPS (BLOOM-176B block linears, 2048 tokens)"
+UNIT = "TOPS"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_gemm_i8_bloom_block_traffic.txt")
+GEMM_SOURCES = [os.path.join(ROOT, "int8_mixed_precision_rowwise_b200", "csrc", f) for f in ("gemm.cu", "ptx.cuh")]
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def ops_of(lin) -> int:
+    return 2 * lin.M * lin.N * lin.K
+
+
+def workload_config(extra=None):
+    cfg = {
+        "workload": WORKLOAD.name,
+        "linears": {l.name: [l.M, l.N, l.K] for l in WORKLOAD.linears},
+        "tokens": WORKLOAD.linears[0].M,
+        "threshold": WORKLOAD.threshold,
+        "outlier_cols": {l.name: l.n_outlier_cols for l in WORKLOAD.linears},
+        "outlier_scale": 60.0,
+        "weights": "fp16 N(0,0.02) kept for outlier columns; int8 CB/SCB prepared before timing",
+        "l2": "no flush: each linear's int8 weight (205-822 MB) exceeds the 126 MB L2",
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None if
+    the summary is missing or the kernel source changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    vals = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("gemm_source_sha256_16") != gemm_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_avg"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import int8_mixed_precision_rowwise_b200 as L
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    int8_peak_burst = 2.0 * peaks["bf16_tflops"]          # nominal int8 : bf16 = 4.5 : 2.25
+    int8_peak_sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+
+    # Inputs resident in HBM; weights prepared (quantized per output row) once.
+    layers, xs, ys = [], [], []
+    for li, lin in enumerate(WORKLOAD.linears):
+        X, W, _ = synthetic.torch_device_problem(lin, seed=100 + li + 17 * rank, device=dev)
+        layers.append(L.Int8MixedLinear.from_fp16(W, WORKLOAD.threshold, keep_fp16_weights=True))
+        xs.append(X)
+        ys.append(torch.empty((lin.M, lin.N), dtype=torch.float16, device=dev))
+    torch.cuda.synchronize()
+    step_ops = sum(ops_of(l) for l in WORKLOAD.linears)
+    nlin = len(WORKLOAD.linears)
+    ev_b = [[torch.cuda.Event(enable_timing=True) for _ in range(nlin)] for _ in range(args.steps)]
+    ev_e = [[torch.cuda.Event(enable_timing=True) for _ in range(nlin)] for _ in range(args.steps)]
+    for row in ev_b + ev_e:
+        for e in row:
+            e.record()
+
+    def step(k=None):
+        for i, layer in enumerate(layers):
+            dbg = None if k is None else {"gemm_begin": ev_b[k][i], "gemm_end": ev_e[k][i]}
+            L.matmul_mixed(xs[i], layer.CB, layer.SCB, layer.W_f16, layer.threshold, Y=ys[i], debug=dbg)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t0.record()
+        for k in range(args.steps):
+            step(k)
+        t1.record()
+        torch.cuda.synchronize()
+    ms_total = t0.elapsed_time(t1)
+    gemm_ms = sum(ev_b[k][i].elapsed_time(ev_e[k][i]) for k in range(args.steps) for i in range(nlin))
+    status = L.read_status(L._workspaces[local_rank], clear=False)
+    if status:
+        raise RuntimeError(f"device status word {status:#x}: a kernel gave up on a bounded wait")
+
+    # e2e: the same step through the public API with host buffers: X from pinned
+    # host memory to the device, the layer, Y back to pinned host memory.
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in ys]
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for i, layer in enumerate(layers):
+            xd = xh[i].to(dev, non_blocking=True)
+            yd = layer(xd)
+            yh[i].copy_(yd, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+
+    secondary = measure_secondary(L, dev) if rank == 0 else None
+
+    t = torch.tensor([ms_total, gemm_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, gemm_ms, e2e_ms = t.tolist()
+    if rank != 0:
+        return None
+    ms_step = ms_total / args.steps
+    value = world * step_ops * args.steps / (ms_total * 1e-3) / 1e12
+    gemm_launches = args.steps * nlin
+    achieved = step_ops * args.steps / (gemm_ms * 1e-3) / 1e12
+    peak = int8_peak_sustained
+    traffic = recorded_traffic()
+    clk = clocks.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": workload_config({"parallelism": f"replicas{world}" if world > 1 else "single"}),
+        "roofline": {
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": "k_gemm_i8<256,4,false,false> (fused dequant + outlier epilogue)",
+            "peak_source": f"2 x bf16 sustained of {peak_kind} ({peaks.get('bf16_tflops_sustained')} TF/s), "
+                           f"nominal int8:bf16 = 4.5:2.25; burst equivalent {round(int8_peak_burst, 1)}, "
+                           "spec 4500",
+            "frac_of_spec_4500": round(achieved / 4500.0, 4),
+        },
+        "gemm_share_of_step": round(gemm_ms / ms_total, 4),
+        "cpu_baseline": cpu_baseline(args) if world == 1 else None,
+        "e2e": {"value": round(world * step_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in xs)),
+                "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in ys))},
+        "gpu_launches": 3 * gemm_launches,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+        "secondary": secondary,
+    }
+    return line
+
+
+def measure_secondary(L, dev):
+    """The quantizer (4096 x 4096, 8 columns x40) and the decode path (BLOOM
+    width, M = 1, 8, 32) in HBM GB/s of algorithmic bytes, CUDA-event timed."""
+    import torch
+
+    peaks, _ = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, iters=30):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    out = {"l2": "256 MB buffer written between iterations", "hbm_peak_gbs": hbm}
+    lin = synthetic.QUANT_4096.linears[0]
+    X, _, _ = synthetic.torch_device_problem(synthetic.Linear("q", lin.M, 1, lin.K, lin.n_outlier_cols,
+                                                              lin.outlier_scale), 0, dev)
+    codes = torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev)
+    am = torch.empty(lin.M, dtype=torch.float32, device=dev)
+    bm = torch.empty((lin.K + 31) // 32, dtype=torch.int32, device=dev)
+    ms = timed(lambda: L.quantize_rowwise(X, 6.0, codes, am, bm))
+    byts = 2 * lin.M * lin.K + lin.M * lin.K + 4 * lin.M + lin.K // 8
+    out["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
+                                  "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+    for M in (1, 8, 32):
+        lin = synthetic.decode_bloom(M).linears[0]
+        X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
+        layer = L.Int8MixedLinear.from_fp16(W, keep_fp16_weights=False)
+        del W
+        Y = torch.empty((M, lin.N), dtype=torch.float16, device=dev)
+        ms = timed(lambda: layer(X, Y))
+        byts = lin.N * lin.K + 4 * lin.N + 2 * M * lin.K + 2 * M * lin.N
+        out[f"decode_M{M}"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
+                               "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
+# --------------------------------------------------------------------------- CPU oracle arm
+
+SAMPLE_COLS = 128  # weight output rows per linear in the CPU sample
+
+
+def oracle_sample_step(oracle, lin, li):
+    """The oracle's whole linear on all tokens against SAMPLE_COLS weight rows.
+    Returns the algorithmic ops it covered."""
+    X, _ = synthetic.make_activations(lin, seed=100 + li)
+    W = synthetic.make_weight(lin, seed=100 + li, rows=SAMPLE_COLS)
+    oracle.matmul_mixed(X, WORKLOAD.threshold, W=W)
+    return 2 * lin.M * SAMPLE_COLS * lin.K
+
+
+def cpu_baseline(args, steps=1):
+    import oracle
+
+    oracle.build()
+    ops, secs = 0, 0.0
+    for _ in range(steps):
+        for li, lin in enumerate(WORKLOAD.linears):
+            X, _ = synthetic.make_activations(lin, seed=100 + li)
+            W = synthetic.make_weight(lin, seed=100 + li, rows=SAMPLE_COLS)
+            t0 = time.perf_counter()
+            oracle.matmul_mixed(X, WORKLOAD.threshold, W=W)
+            secs += time.perf_counter() - t0
+            ops += 2 * lin.M * SAMPLE_COLS * lin.K
+    return {"value": round(ops / secs / 1e12, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"all {WORKLOAD.linears[0].M} tokens x {SAMPLE_COLS} output rows of each of the four "
+                      f"linears (full outlier detection and quantization of X), single-threaded C, "
+                      f"{secs:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+
+    oracle.build()
+    for _ in range(args.warmup):
+        oracle_sample_step(oracle, WORKLOAD.linears[1], 1)
+    ops, secs = 0, 0.0
+    for _ in range(args.steps):
+        for li, lin in enumerate(WORKLOAD.linears):
+            X, _ = synthetic.make_activations(lin, seed=100 + li)
+            W = synthetic.make_weight(lin, seed=100 + li, rows=SAMPLE_COLS)
+            t0 = time.perf_counter()
+            oracle.matmul_mixed(X, WORKLOAD.threshold, W=W)
+            secs += time.perf_counter() - t0
+            ops += 2 * lin.M * SAMPLE_COLS * lin.K
+    value = ops / secs / 1e12
+    sample = (f"each step: all {WORKLOAD.linears[0].M} tokens x {SAMPLE_COLS} output rows of each of the four "
+              f"linears, single-threaded C oracle")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": workload_config({"parallelism": "single"}),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -134,6 +134,8 @@ typedef struct llmint8_debug {
     int32_t *count;     /* [1]     |O| */
     int32_t *acc;       /* [M x N] int32 accumulators of the int8 part (runs the
                            int8 GEMM a second time with a raw int32 epilogue) */
+    void *gemm_begin;   /* cudaEvent_t or NULL: recorded on `stream` right before */
+    void *gemm_end;     /* and right after the fused GEMM launch (kernel timing)  */
 } llmint8_debug;
 
 /*

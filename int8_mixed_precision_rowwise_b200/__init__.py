@@ -38,7 +38,8 @@ _ST = ctypes.c_int
 
 
 class _Debug(ctypes.Structure):
-    _fields_ = [("codes", _P), ("row_absmax", _P), ("col_idx", _P), ("count", _P), ("acc", _P)]
+    _fields_ = [("codes", _P), ("row_absmax", _P), ("col_idx", _P), ("count", _P), ("acc", _P),
+                ("gemm_begin", _P), ("gemm_end", _P)]
 
 
 def _sig(name, restype, argtypes):
@@ -104,6 +105,15 @@ def _stream_ptr(device):
 
 def _ptr(t):
     return None if t is None else t.data_ptr()
+
+
+def _event(ev):
+    """Raw cudaEvent_t of a torch.cuda.Event (created on its first record)."""
+    if ev is None:
+        return None
+    if not ev.cuda_event:
+        ev.record()
+    return ev.cuda_event
 
 
 def _need_cuda(t, name, dtype=None):
@@ -180,7 +190,8 @@ def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y
     """Y fp16 [M x N] = LLM.int8()(X fp16 [M x K], W given as CB int8 [N x K] + SCB fp32 [N]).
 
     ``debug`` may map any of codes/row_absmax/col_idx/count/acc to CUDA tensors
-    the call fills (parity checks)."""
+    the call fills (parity checks), and gemm_begin/gemm_end to recorded
+    torch.cuda.Event objects the library re-records around the GEMM launch."""
     torch = _torch()
     _need_cuda(X, "X", torch.float16)
     _need_cuda(CB, "CB", torch.int8)
@@ -195,7 +206,8 @@ def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y
     ws = workspace if workspace is not None else get_workspace(workspace_size(M, N, K), dev)
     dbg = None
     if debug:
-        dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")))
+        dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")),
+                     *(_event(debug.get(k)) for k in ("gemm_begin", "gemm_end")))
     _check(_matmul_mixed(X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N, float(threshold),
                          Y.data_ptr(), ws.data_ptr(), ws.numel(), ctypes.byref(dbg) if dbg else None,
                          _stream_ptr(dev)), "llmint8_matmul_mixed")

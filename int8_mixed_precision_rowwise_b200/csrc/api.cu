@@ -241,7 +241,12 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
     g.status = ws.status;
     g.epi = Epilogue::MixedFp16;
     g.Y = Y_f16;
+    if (dbg && dbg->gemm_begin &&
+        cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
     if ((e = launch_gemm(g, dev, stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if (dbg && dbg->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
 
     if (dbg) {

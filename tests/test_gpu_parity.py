@@ -133,13 +133,12 @@ def test_quantize_worked_example(lib, dev):
 
 
 def test_quantize_edge_rows(lib, dev, oracle_mod):
-    """Zero rows, rows made only of outliers, exact-threshold values, .5 ties,
-    and rows whose maximum sits in a column that is an outlier only because
-    of another row (the fix-up path)."""
+    """Zero rows, exact-threshold values, .5 ties, values just below the
+    threshold, and rows whose maximum sits in a column that is an outlier only
+    because of another row (the fix-up path)."""
     rng = np.random.default_rng(5)
     X = rng.standard_normal((200, 256)).astype(np.float32)
     X[3] = 0.0
-    X[4] = 7.0
     X[5, 10] = 6.0                       # exactly the threshold: outlier column 10
     X[6] = 0.0
     X[6, :3] = [127.0, 2.5, 3.5]         # ties: s = 1
@@ -155,6 +154,16 @@ def test_quantize_edge_rows(lib, dev, oracle_mod):
     assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 256), mask)
     assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
     assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_quantize_row_of_outliers(lib, dev, oracle_mod):
+    """One row >= t everywhere makes every column an outlier: all codes 0,
+    every absmax 0 (the int8 part is empty)."""
+    X16 = make_random((40, 64), seed=6)
+    X16[2] = 7.0
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 64), np.ones(64, np.uint8))
+    assert not codes.cpu().numpy().any() and not absmax.cpu().numpy().any()
 
 
 def test_find_outlier_cols(lib, dev):
@@ -224,7 +233,8 @@ def test_matmul_mixed_matches_oracle(lib, dev, oracle_mod, M, N, K, nout, give_w
     X16, cols = make_activations(lin, seed=M + N)
     W16 = make_weight(lin, seed=K)
     g, r = check_full(lib, dev, oracle_mod, X16, W16, 6.0, give_w16)
-    assert set(cols.tolist()) <= set(r["O"].tolist())
+    if M >= 16:  # with few tokens a planted x60 column can stay below 6 (|z| < 0.1)
+        assert set(cols.tolist()) <= set(r["O"].tolist())
 
 
 def test_threshold_off_and_no_outliers(lib, dev, oracle_mod):
@@ -340,7 +350,8 @@ def test_decode_workload_sampled(lib, dev, oracle_mod, M):
     X, W, cols = synthetic.torch_device_problem(lin, seed=M, device=dev)
     rows, jcols = _samples(lin.M, lin.N, M, ncols=160)
     O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, False, rows, jcols)
-    assert set(cols.tolist()) <= set(O.tolist())
+    if M >= 16:
+        assert set(cols.tolist()) <= set(O.tolist())
 
 
 @pytest.mark.parametrize("name", ["qkv", "attn_out", "fc1", "fc2"])
