@@ -176,6 +176,33 @@ LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, cons
                                     int64_t K, int32_t *acc, void *workspace, size_t ws_bytes,
                                     llmint8_stream_t stream);
 
+/*
+ * Allocation-free row-wise quantizer. The source page has no counterpart: it
+ * exists for callers that cannot allocate device memory, such as a server
+ * that reserved all device memory for its own pool at start-up, a plugin in a
+ * host process that forbids device allocations after initialisation, or a
+ * latency-critical loop that cannot afford an allocation's implicit
+ * synchronisation.
+ *
+ * Same arguments and results as llmint8_quantize_rowwise, without the
+ * workspace: the scratch sits in a fixed array inside the library (about
+ * 512 KB, held by every GPU that uses this call until the process exits).
+ *   - rows <= LLMINT8_NOALLOC_MAX_ROWS and cols <= LLMINT8_NOALLOC_MAX_COLS;
+ *     larger sizes return LLMINT8_ERR_UNSUPPORTED_SHAPE before any work.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture on the device.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents. Calls ordered on one stream are safe; calls whose work
+ *     overlaps on the GPU (unordered streams) race and give wrong results.
+ */
+#define LLMINT8_NOALLOC_MAX_ROWS 65536
+#define LLMINT8_NOALLOC_MAX_COLS 65536
+LLMINT8_API llmint8_status llmint8_quantize_rowwise_noalloc(const void *X_f16, int64_t rows, int64_t cols,
+                                                float threshold, int8_t *codes, float *row_absmax,
+                                                uint32_t *outlier_bitmap, llmint8_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

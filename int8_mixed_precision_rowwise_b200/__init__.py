@@ -18,7 +18,7 @@ import os
 __all__ = [
     "LIB_PATH", "LLMInt8Error", "status_string", "quantize_workspace_size", "workspace_size",
     "workspace_init", "read_status", "quantize_rowwise", "find_outlier_cols", "matmul_mixed",
-    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD",
+    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
@@ -26,46 +26,57 @@ DEFAULT_THRESHOLD = 6.0
 
 OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(7)
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m int8_mixed_precision_rowwise_b200.build` "
-        "(nvcc, sm_100a). There is no CPU fallback.")
+class _Debug(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("row_absmax", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
+                ("count", ctypes.c_void_p), ("acc", ctypes.c_void_p), ("gemm_begin", ctypes.c_void_p),
+                ("gemm_end", ctypes.c_void_p)]
 
-_lib = ctypes.CDLL(LIB_PATH)
+
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _ST = ctypes.c_int
+# ctypes signatures of the C entry points (name -> (restype, argtypes)).
+_SIGNATURES = {
+    "llmint8_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "llmint8_quantize_workspace_size": (ctypes.c_size_t, [_I64, _I64]),
+    "llmint8_workspace_size": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "llmint8_workspace_init": (_ST, [_P, ctypes.c_size_t, _P]),
+    "llmint8_read_status": (_ST, [_P, ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]),
+    "llmint8_quantize_rowwise": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "llmint8_find_outlier_cols": (_ST, [_P, _I64, _P, _P, _P, _P]),
+    "llmint8_matmul_mixed": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, ctypes.c_float, _P, _P, ctypes.c_size_t,
+                                   ctypes.POINTER(_Debug), _P]),
+    "llmint8_gemm_s8s8s32": (_ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
+    "llmint8_quantize_rowwise_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
+}
+EXPORTED = tuple(_SIGNATURES)
+NOALLOC_MAX_ROWS = NOALLOC_MAX_COLS = 65536
+_fns: dict = {}
 
 
-class _Debug(ctypes.Structure):
-    _fields_ = [("codes", _P), ("row_absmax", _P), ("col_idx", _P), ("count", _P), ("acc", _P),
-                ("gemm_begin", _P), ("gemm_end", _P)]
+def load():
+    """Load libllmint8.so (once) and bind its entry points. Raises ImportError
+    when the library has not been built: there is no CPU fallback."""
+    if not _fns:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m int8_mixed_precision_rowwise_b200.build` "
+                "(nvcc, sm_100a). There is no CPU fallback.")
+        cdll = ctypes.CDLL(LIB_PATH)
+        fns = {}
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(cdll, name)
+            f.restype, f.argtypes = res, args
+            fns["_" + name[len("llmint8_"):]] = f
+        _fns.update(fns)
+    return _fns
 
 
-def _sig(name, restype, argtypes):
-    f = getattr(_lib, name)
-    f.restype = restype
-    f.argtypes = argtypes
-    return f
-
-
-_status_string = _sig("llmint8_status_string", ctypes.c_char_p, [ctypes.c_int])
-_quantize_workspace_size = _sig("llmint8_quantize_workspace_size", ctypes.c_size_t, [_I64, _I64])
-_workspace_size = _sig("llmint8_workspace_size", ctypes.c_size_t, [_I64, _I64, _I64])
-_workspace_init = _sig("llmint8_workspace_init", _ST, [_P, ctypes.c_size_t, _P])
-_read_status = _sig("llmint8_read_status", _ST, [_P, ctypes.c_size_t, ctypes.c_int,
-                                                  ctypes.POINTER(ctypes.c_uint32)])
-_quantize_rowwise = _sig("llmint8_quantize_rowwise", _ST,
-                         [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P])
-_find_outlier_cols = _sig("llmint8_find_outlier_cols", _ST, [_P, _I64, _P, _P, _P, _P])
-_matmul_mixed = _sig("llmint8_matmul_mixed", _ST,
-                     [_P, _I64, _I64, _P, _P, _P, _I64, ctypes.c_float, _P, _P, ctypes.c_size_t,
-                      ctypes.POINTER(_Debug), _P])
-_gemm_s8s8s32 = _sig("llmint8_gemm_s8s8s32", _ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P])
-
-EXPORTED = ("llmint8_status_string", "llmint8_quantize_workspace_size", "llmint8_workspace_size",
-            "llmint8_workspace_init", "llmint8_read_status", "llmint8_quantize_rowwise",
-            "llmint8_find_outlier_cols", "llmint8_matmul_mixed", "llmint8_gemm_s8s8s32")
+def __getattr__(name):
+    # _matmul_mixed, _quantize_rowwise, ...: the raw ctypes entry points.
+    if name.startswith("_") and "llmint8" + name in _SIGNATURES:
+        return load()[name]
+    raise AttributeError(name)
 
 
 class LLMInt8Error(RuntimeError):
@@ -75,7 +86,7 @@ class LLMInt8Error(RuntimeError):
 
 
 def status_string(status: int) -> str:
-    return _status_string(int(status)).decode()
+    return load()["_status_string"](int(status)).decode()
 
 
 def _check(status: int, where: str):
@@ -84,11 +95,11 @@ def _check(status: int, where: str):
 
 
 def quantize_workspace_size(rows: int, cols: int) -> int:
-    return int(_quantize_workspace_size(rows, cols))
+    return int(load()["_quantize_workspace_size"](rows, cols))
 
 
 def workspace_size(M: int, N: int, K: int) -> int:
-    return int(_workspace_size(M, N, K))
+    return int(load()["_workspace_size"](M, N, K))
 
 
 # --------------------------------------------------------------------- torch glue
@@ -141,12 +152,12 @@ def get_workspace(nbytes: int, device):
 
 
 def workspace_init(ws) -> None:
-    _check(_workspace_init(ws.data_ptr(), ws.numel(), _stream_ptr(ws.device)), "llmint8_workspace_init")
+    _check(load()["_workspace_init"](ws.data_ptr(), ws.numel(), _stream_ptr(ws.device)), "llmint8_workspace_init")
 
 
 def read_status(ws, clear: bool = True) -> int:
     out = ctypes.c_uint32(0)
-    _check(_read_status(ws.data_ptr(), ws.numel(), int(clear), ctypes.byref(out)), "llmint8_read_status")
+    _check(load()["_read_status"](ws.data_ptr(), ws.numel(), int(clear), ctypes.byref(out)), "llmint8_read_status")
     return int(out.value)
 
 
@@ -164,9 +175,30 @@ def quantize_rowwise(X, threshold: float = 0.0, codes=None, row_absmax=None, out
     if outlier_bitmap is None and threshold > 0:
         outlier_bitmap = torch.empty((cols + 31) // 32, dtype=torch.int32, device=dev)
     ws = workspace if workspace is not None else get_workspace(quantize_workspace_size(rows, cols), dev)
-    _check(_quantize_rowwise(X.data_ptr(), rows, cols, float(threshold), codes.data_ptr(),
+    _check(load()["_quantize_rowwise"](X.data_ptr(), rows, cols, float(threshold), codes.data_ptr(),
                              row_absmax.data_ptr(), _ptr(outlier_bitmap), ws.data_ptr(), ws.numel(),
                              _stream_ptr(dev)), "llmint8_quantize_rowwise")
+    return codes, row_absmax, outlier_bitmap
+
+
+def quantize_rowwise_noalloc(X, threshold: float = 0.0, codes=None, row_absmax=None, outlier_bitmap=None):
+    """quantize_rowwise without a workspace, for callers that cannot allocate
+    device memory: the library's fixed scratch array (rows and cols up to
+    65536) replaces it. Pass preallocated outputs to allocate nothing here
+    either. Calls that overlap on the GPU share that scratch and race."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    rows, cols = X.shape
+    dev = X.device
+    if codes is None:
+        codes = torch.empty((rows, cols), dtype=torch.int8, device=dev)
+    if row_absmax is None:
+        row_absmax = torch.empty(rows, dtype=torch.float32, device=dev)
+    if outlier_bitmap is None and threshold > 0:
+        outlier_bitmap = torch.empty((cols + 31) // 32, dtype=torch.int32, device=dev)
+    _check(load()["_quantize_rowwise_noalloc"](X.data_ptr(), rows, cols, float(threshold), codes.data_ptr(),
+                                     row_absmax.data_ptr(), _ptr(outlier_bitmap), _stream_ptr(dev)),
+           "llmint8_quantize_rowwise_noalloc")
     return codes, row_absmax, outlier_bitmap
 
 
@@ -179,7 +211,7 @@ def find_outlier_cols(outlier_bitmap, cols: int, col_idx=None, d_count=None, syn
     if d_count is None:
         d_count = torch.empty(1, dtype=torch.int32, device=dev)
     h = ctypes.c_int32(-1)
-    _check(_find_outlier_cols(outlier_bitmap.data_ptr(), cols, col_idx.data_ptr(), d_count.data_ptr(),
+    _check(load()["_find_outlier_cols"](outlier_bitmap.data_ptr(), cols, col_idx.data_ptr(), d_count.data_ptr(),
                               ctypes.byref(h) if sync_count else None, _stream_ptr(dev)),
            "llmint8_find_outlier_cols")
     return col_idx, d_count, (int(h.value) if sync_count else None)
@@ -208,7 +240,7 @@ def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y
     if debug:
         dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")),
                      *(_event(debug.get(k)) for k in ("gemm_begin", "gemm_end")))
-    _check(_matmul_mixed(X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N, float(threshold),
+    _check(load()["_matmul_mixed"](X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N, float(threshold),
                          Y.data_ptr(), ws.data_ptr(), ws.numel(), ctypes.byref(dbg) if dbg else None,
                          _stream_ptr(dev)), "llmint8_matmul_mixed")
     return Y
@@ -224,7 +256,7 @@ def gemm_s8s8s32(A, B, acc=None, workspace=None):
     if acc is None:
         acc = torch.empty((M, N), dtype=torch.int32, device=A.device)
     ws = workspace if workspace is not None else get_workspace(workspace_size(M, N, K), A.device)
-    _check(_gemm_s8s8s32(A.data_ptr(), M, B.data_ptr(), N, K, acc.data_ptr(), ws.data_ptr(), ws.numel(),
+    _check(load()["_gemm_s8s8s32"](A.data_ptr(), M, B.data_ptr(), N, K, acc.data_ptr(), ws.data_ptr(), ws.numel(),
                          _stream_ptr(A.device)), "llmint8_gemm_s8s8s32")
     return acc
 

@@ -1,0 +1,66 @@
+"""The allocation-free quantizer entry point, llmint8_quantize_rowwise_noalloc.
+
+It serves callers that cannot allocate device memory (a server whose memory
+pool owns the whole GPU, a plugin barred from allocating after start-up, a
+loop that cannot afford an allocation's synchronisation): its scratch is a
+fixed array inside the library instead of a caller workspace. These tests
+call it through the C ABI and compare it with llmint8_quantize_rowwise, the
+entry point that takes a workspace, on two calls in a row; codes, row absmax
+bits and outlier bitmap must match exactly, as everywhere else in the tests.
+This file is collected last so that a run stopping at the first failure has
+already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from synthetic import Linear, make_activations
+
+
+def _noalloc_fn(lib_path):
+    cdll = ctypes.CDLL(lib_path)
+    f = cdll.llmint8_quantize_rowwise_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    return f
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    """Sizes past the fixed array are refused before any GPU work (no GPU needed)."""
+    import int8_mixed_precision_rowwise_b200 as L
+    f = _noalloc_fn(L.LIB_PATH)
+    A = 0x10000
+    assert f(A, 65537, 1024, 6.0, A, A, A, None) == L.ERR_UNSUPPORTED_SHAPE
+    assert f(A, 16, 65536 + 16, 6.0, A, A, A, None) == L.ERR_UNSUPPORTED_SHAPE
+    assert f(A, 16, 1000, 6.0, A, A, A, None) == L.ERR_UNSUPPORTED_SHAPE   # cols % 16
+    assert f(A, 16, 1024, 6.0, A, A, None, None) == L.ERR_INVALID_ARG      # bitmap needed for t > 0
+    assert f(A, 0, 1024, 6.0, A, A, A, None) == L.OK                       # empty: nothing queued
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import int8_mixed_precision_rowwise_b200 as L
+    f = _noalloc_fn(L.LIB_PATH)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    # Two calls in a row; the second is smaller, so stale scratch from the
+    # first (argmax rows, outlier list, count) would show up in its result.
+    for M, K, n_out, seed in [(700, 4096, 8, 1), (333, 1024, 5, 2)]:
+        X16, _ = make_activations(Linear("q", M, 0, K, n_out, 40.0), seed=seed)
+        X = torch.from_numpy(X16).to(dev)
+        ref_codes, ref_absmax, ref_bm = L.quantize_rowwise(X, 6.0)
+        codes = torch.empty((M, K), dtype=torch.int8, device=dev)
+        absmax = torch.empty(M, dtype=torch.float32, device=dev)
+        bm = torch.full(((K + 31) // 32,), -1, dtype=torch.int32, device=dev)
+        st = f(X.data_ptr(), M, K, 6.0, codes.data_ptr(), absmax.data_ptr(), bm.data_ptr(), stream)
+        assert st == L.OK, L.status_string(st)
+        torch.cuda.synchronize()
+        assert torch.equal(codes, ref_codes)
+        assert np.array_equal(absmax.cpu().numpy().view(np.uint32), ref_absmax.cpu().numpy().view(np.uint32))
+        assert torch.equal(bm, ref_bm)
+        assert int(bm.ne(0).sum()) > 0  # the outlier columns were found
