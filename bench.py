@@ -282,51 +282,73 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def graph_time_ms(fns, reps):
+    """Average device time per call of `fns` (called in turn, `reps` times),
+    captured into one CUDA graph so host launch overhead is excluded; the
+    calls rotate over inputs larger than L2 together."""
+    import torch
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for f in fns:  # first calls outside capture (per-device set-up)
+            f()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            for f in fns:
+                f()
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / (reps * len(fns)))
+    del g
+    return statistics.median(ts)
+
+
 def measure_secondary(L, dev):
     """The quantizer (4096 x 4096, 8 columns x40) and the decode path (BLOOM
-    width, M = 1, 8, 32) in HBM GB/s of algorithmic bytes, CUDA-event timed."""
+    width, M = 1, 8, 32) in HBM GB/s of algorithmic bytes. Each is timed as a
+    CUDA graph of back-to-back calls; the quantizer rotates over 8 inputs
+    (256 MB, twice L2), the decode weights (205 MB) exceed L2 by themselves."""
     import torch
 
     peaks, _ = load_peaks()
     hbm = peaks["hbm_gbs"]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
-    def timed(fn, iters=30):
-        for _ in range(3):
-            fn()
-        ts = []
-        for _ in range(iters):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
-
-    out = {"l2": "256 MB buffer written between iterations", "hbm_peak_gbs": hbm}
+    out = {"timing": "CUDA graph of back-to-back calls; inputs larger than L2", "hbm_peak_gbs": hbm}
     lin = synthetic.QUANT_4096.linears[0]
-    X, _, _ = synthetic.torch_device_problem(synthetic.Linear("q", lin.M, 1, lin.K, lin.n_outlier_cols,
-                                                              lin.outlier_scale), 0, dev)
-    codes = torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev)
-    am = torch.empty(lin.M, dtype=torch.float32, device=dev)
-    bm = torch.empty((lin.K + 31) // 32, dtype=torch.int32, device=dev)
-    ms = timed(lambda: L.quantize_rowwise(X, 6.0, codes, am, bm))
+    bufs = []
+    for k in range(8):
+        X, _, _ = synthetic.torch_device_problem(
+            synthetic.Linear("q", lin.M, 1, lin.K, lin.n_outlier_cols, lin.outlier_scale), k, dev)
+        bufs.append((X, torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
+                     torch.empty(lin.M, dtype=torch.float32, device=dev),
+                     torch.empty((lin.K + 31) // 32, dtype=torch.int32, device=dev)))
+    fns = [lambda b=b: L.quantize_rowwise(b[0], 6.0, b[1], b[2], b[3]) for b in bufs]
+    ms = graph_time_ms(fns, reps=4)
     byts = 2 * lin.M * lin.K + lin.M * lin.K + 4 * lin.M + lin.K // 8
     out["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
                                   "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+    del bufs, fns
     for M in (1, 8, 32):
         lin = synthetic.decode_bloom(M).linears[0]
         X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
         layer = L.Int8MixedLinear.from_fp16(W, keep_fp16_weights=False)
         del W
         Y = torch.empty((M, lin.N), dtype=torch.float16, device=dev)
-        ms = timed(lambda: layer(X, Y))
+        ms = graph_time_ms([lambda: layer(X, Y)], reps=20)
         byts = lin.N * lin.K + 4 * lin.N + 2 * M * lin.K + 2 * M * lin.N
         out[f"decode_M{M}"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
                                "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
-    del flush
+        del layer, X, Y
     torch.cuda.empty_cache()
     return out
 
@@ -394,13 +416,48 @@ def run_reference(args, rank, world):
     }
 
 
+def run_profile_case(args):
+    """A minimal driver for ncu captures: set up the named BLOOM linear (or
+    'all' four), run one warm-up pass, then --steps passes inside an NVTX
+    range 'timed_steps'. Prints nothing; exits 0 on success."""
+    import torch
+
+    import int8_mixed_precision_rowwise_b200 as L
+
+    dev = torch.device("cuda", 0)
+    lins = [l for l in WORKLOAD.linears if args.profile_case in ("all", l.name)]
+    if not lins:
+        raise SystemExit(f"unknown linear {args.profile_case!r}")
+    layers, xs, ys = [], [], []
+    for li, lin in enumerate(lins):
+        X, W, _ = synthetic.torch_device_problem(lin, seed=100 + li, device=dev)
+        layers.append(L.Int8MixedLinear.from_fp16(W, WORKLOAD.threshold, keep_fp16_weights=True))
+        xs.append(X)
+        ys.append(torch.empty((lin.M, lin.N), dtype=torch.float16, device=dev))
+    for i, layer in enumerate(layers):
+        layer(xs[i], ys[i])
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed_steps")
+    for _ in range(args.steps):
+        for i, layer in enumerate(layers):
+            layer(xs[i], ys[i])
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    assert L.read_status(L._workspaces[0], clear=False) == 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--profile-case", default=None,
+                    help="ncu driver: run only this BLOOM linear ('qkv', 'attn_out', 'fc1', 'fc2' or 'all')")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

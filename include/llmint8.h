@@ -67,6 +67,7 @@ typedef enum llmint8_status {
 #define LLMINT8_DEV_TIMEOUT_PRODUCER 0x1u
 #define LLMINT8_DEV_TIMEOUT_MMA 0x2u
 #define LLMINT8_DEV_TIMEOUT_EPILOGUE 0x4u
+#define LLMINT8_DEV_TIMEOUT_QUANT 0x8u
 
 /* Human-readable name of a status code. Never NULL. */
 LLMINT8_API const char *llmint8_status_string(int status);
@@ -186,7 +187,7 @@ LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, cons
  *
  * Same arguments and results as llmint8_quantize_rowwise, without the
  * workspace: the scratch sits in a fixed array inside the library (about
- * 512 KB, held by every GPU that uses this call until the process exits).
+ * 256 KB, held by every GPU that uses this call until the process exits).
  *   - rows <= LLMINT8_NOALLOC_MAX_ROWS and cols <= LLMINT8_NOALLOC_MAX_COLS;
  *     larger sizes return LLMINT8_ERR_UNSUPPORTED_SHAPE before any work.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.

@@ -153,8 +153,11 @@ llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t
         if ((e = cudaMemsetAsync(outlier_bitmap, 0, nwords * 4, stream)) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
     }
-    e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.argmax, ws.col_idx,
-                        ws.count, dev, stream);
+    // |O| and the kernel's sync words (header bytes 4..23); the status word stays.
+    if ((e = cudaMemsetAsync(ws.count, 0, 20, stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.col_idx, ws.count, ws.sync,
+                        ws.status, dev, stream);
     return cuda_status(e);
 }
 
@@ -222,8 +225,8 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
     const size_t clear_bytes = (reinterpret_cast<char *>(ws.bitmap) - clear_from) + (size_t)((K + 31) / 32) * 4;
     if ((e = cudaMemsetAsync(clear_from, 0, clear_bytes, stream)) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    if ((e = launch_quantize(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws.argmax, ws.col_idx, ws.count, dev,
-                             stream)) != cudaSuccess)
+    if ((e = launch_quantize(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws.col_idx, ws.count, ws.sync, ws.status,
+                             dev, stream)) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
 
     GemmArgs g{};

@@ -91,6 +91,254 @@ __device__ __forceinline__ void report(const KParams &p, volatile int *s_abort, 
     *s_abort = 1;
 }
 
+// Epilogue of one CTA (warps 2..5): for each of its output tiles, stage the
+// outlier operands and scales while the tile's MMAs run, wait for the
+// accumulator, then dequantize, add the outlier product and store (or store
+// the raw int32 accumulators), and hand the TMEM buffer back to the MMA
+// issuer. Tiles are first_tile, first_tile + tile_step, ...; this CTA's
+// accumulator rows are a_row_off .. a_row_off + 127 of each a_tile_rows-row
+// A tile.
+template <int BN, bool SWAP, bool RAW, bool PAIR>
+__device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lane, float *s_side, float *s_scale,
+                                             uint32_t tfull0, uint32_t tempty0, volatile int *s_abort,
+                                             uint32_t tmem_base, int first_tile, int tile_step, int num_tiles,
+                                             int a_tile_rows, int a_row_off)
+{
+    auto tfull_bar = [&](int b) { return tfull0 + 8u * b; };
+    auto tempty_bar = [&](int b) { return tempty0 + 8u * b; };
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int et = threadIdx.x - 64;        // 0..127
+    const int r_in_tile = q * 32 + lane;    // accumulator row (A-side row in the tile)
+    const int cnt = RAW ? 0 : min(*p.count, p.K);
+    const bool fast = cnt <= OC;
+    uint32_t tph[2] = {0u, 0u};
+    int local = 0;
+    for (int tile = first_tile; tile < num_tiles; tile += tile_step, ++local) {
+        const int b = local & 1;
+        const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
+        const int arow = mb * a_tile_rows + a_row_off + r_in_tile; // A-operand row of this thread
+        const int brow0 = nb * BN;               // first B-operand row of the tile
+        float own_scale = 0.f;
+        float own_side[OC];
+#pragma unroll
+        for (int k = 0; k < OC; ++k)
+            own_side[k] = 0.f;
+        if (!RAW) {
+            // Stage the outlier operands and scales while the MMAs run.
+            named_barrier_sync(1, 128);
+            for (int idx = et; idx < BN; idx += 128) {
+                const int r = brow0 + idx;
+                s_scale[idx] = SWAP ? (r < p.M ? p.sx[r] : 0.f) : (r < p.N ? p.sb[r] : 0.f);
+            }
+            if (fast) {
+                for (int idx = et; idx < cnt * BN; idx += 128) {
+                    const int k = idx / BN, c = idx - k * BN;
+                    const int r = brow0 + c;
+                    const int col = p.col_idx[k];
+                    float v = 0.f;
+                    if (SWAP) {
+                        if (r < p.M)
+                            v = __half2float(p.X16[(int64_t)r * p.K + col]);
+                    } else {
+                        if (r < p.N)
+                            v = wtilde(p, r, col);
+                    }
+                    s_side[idx] = v;
+                }
+            }
+            if (SWAP) {
+                if (arow < p.N) {
+                    own_scale = p.sb[arow];
+                    if (fast) {
+#pragma unroll
+                        for (int k = 0; k < OC; ++k)
+                            if (k < cnt)
+                                own_side[k] = wtilde(p, arow, p.col_idx[k]);
+                    }
+                }
+            } else {
+                if (arow < p.M) {
+                    own_scale = p.sx[arow];
+                    if (fast) {
+#pragma unroll
+                        for (int k = 0; k < OC; ++k)
+                            if (k < cnt)
+                                own_side[k] = __half2float(p.X16[(int64_t)arow * p.K + p.col_idx[k]]);
+                    }
+                }
+            }
+            named_barrier_sync(1, 128);
+        }
+
+        // All 128 epilogue threads leave together if any of them gave up,
+        // so no thread is left waiting at a named barrier.
+        const bool got = mbar_wait(tfull_bar(b), tph[b]);
+        if (named_barrier_or(1, 128, !got)) {
+            if (!got)
+                report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+            break;
+        }
+        tph[b] ^= 1u;
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
+
+        if constexpr (!SWAP) {
+            const int i = arow;
+#pragma unroll 1
+            for (int g = 0; g < BN / 32; ++g) {
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(tbase + g * 32, acc);
+                tmem_wait_ld();
+                const int j0 = brow0 + g * 32;
+                if constexpr (RAW) {
+                    int32_t *Yr = reinterpret_cast<int32_t *>(p.Y) + (int64_t)i * p.N;
+                    if (i < p.M) {
+                        if (j0 + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+                            for (int c = 0; c < 32; c += 4)
+                                *reinterpret_cast<uint4 *>(Yr + j0 + c) =
+                                    make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                        } else {
+                            for (int c = 0; c < 32; ++c)
+                                if (j0 + c < p.N)
+                                    Yr[j0 + c] = (int32_t)acc[c];
+                        }
+                    }
+                    continue;
+                }
+                float y[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
+                if (fast) {
+#pragma unroll
+                    for (int k = 0; k < OC; ++k) {
+                        if (k < cnt) {
+                            const float xv = own_side[k];
+                            const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                            for (int c4 = 0; c4 < 8; ++c4) {
+                                const float4 w = wrow[c4];
+                                y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                            }
+                        }
+                    }
+                } else {
+                    // More outlier columns than one staged chunk holds.
+                    for (int ch = 0; ch < cnt; ch += OC) {
+                        const int nk = min(OC, cnt - ch);
+                        named_barrier_sync(1, 128);
+                        for (int idx = et; idx < nk * 32; idx += 128) {
+                            const int k = idx >> 5, c = idx & 31;
+                            const int j = j0 + c;
+                            s_side[idx] = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
+                        }
+                        named_barrier_sync(1, 128);
+                        for (int k = 0; k < nk; ++k) {
+                            const float xv =
+                                i < p.M ? __half2float(p.X16[(int64_t)i * p.K + p.col_idx[ch + k]]) : 0.f;
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                y[c] = fmaf(xv, s_side[k * 32 + c], y[c]);
+                        }
+                    }
+                }
+                if (i < p.M) {
+                    __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
+                    if (j0 + 32 <= p.N && (p.N & 7) == 0) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 8) {
+                            uint4 pk;
+                            __half2 *h = reinterpret_cast<__half2 *>(&pk);
+                            h[0] = __floats2half2_rn(y[c + 0], y[c + 1]);
+                            h[1] = __floats2half2_rn(y[c + 2], y[c + 3]);
+                            h[2] = __floats2half2_rn(y[c + 4], y[c + 5]);
+                            h[3] = __floats2half2_rn(y[c + 6], y[c + 7]);
+                            *reinterpret_cast<uint4 *>(Yr + j0 + c) = pk;
+                        }
+                    } else {
+                        for (int c = 0; c < 32; ++c)
+                            if (j0 + c < p.N)
+                                Yr[j0 + c] = __float2half_rn(y[c]);
+                    }
+                }
+            }
+        } else {
+            // Decode form: this thread owns output feature j = arow; the
+            // accumulator columns are tokens brow0 .. brow0 + BN - 1.
+            const int j = arow;
+            uint32_t acc[BN];
+            if constexpr (BN == 32) {
+                tmem_ld_32x32b_x32(tbase, acc);
+            } else {
+                tmem_ld_32x32b_x16(tbase, acc);
+            }
+            tmem_wait_ld();
+            if constexpr (RAW) {
+                if (j < p.N) {
+                    int32_t *Yc = reinterpret_cast<int32_t *>(p.Y) + j;
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        if (brow0 + c < p.M)
+                            Yc[(int64_t)(brow0 + c) * p.N] = (int32_t)acc[c];
+                }
+            } else {
+                float y[BN];
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
+                if (fast) {
+#pragma unroll
+                    for (int k = 0; k < OC; ++k) {
+                        if (k < cnt) {
+                            const float wv = own_side[k];
+#pragma unroll
+                            for (int c = 0; c < BN; ++c)
+                                y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                        }
+                    }
+                } else {
+                    for (int ch = 0; ch < cnt; ch += OC) {
+                        const int nk = min(OC, cnt - ch);
+                        named_barrier_sync(1, 128);
+                        for (int idx = et; idx < nk * BN; idx += 128) {
+                            const int k = idx / BN, c = idx - k * BN;
+                            const int r = brow0 + c;
+                            s_side[idx] =
+                                r < p.M ? __half2float(p.X16[(int64_t)r * p.K + p.col_idx[ch + k]]) : 0.f;
+                        }
+                        named_barrier_sync(1, 128);
+                        for (int k = 0; k < nk; ++k) {
+                            const float wv = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
+#pragma unroll
+                            for (int c = 0; c < BN; ++c)
+                                y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                        }
+                    }
+                }
+                if (j < p.N) {
+                    __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        if (brow0 + c < p.M)
+                            Yc[(int64_t)(brow0 + c) * p.N] = __float2half_rn(y[c]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            if constexpr (PAIR)
+                mbar_arrive_cluster(tempty_bar(b), 0); // the pair's MMA runs in CTA 0
+            else
+                mbar_arrive(tempty_bar(b));
+        }
+    }
+}
+
 template <int BN, int STAGES, bool SWAP, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_gemm_i8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const KParams p)
@@ -222,240 +470,184 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;                 // TMEM lane quarter this warp may read
-        const int et = threadIdx.x - 64;        // 0..127
-        const int r_in_tile = q * 32 + lane;    // accumulator row (A-side row in the tile)
-        const int cnt = RAW ? 0 : min(*p.count, p.K);
-        const bool fast = cnt <= OC;
-        uint32_t tph[2] = {0u, 0u};
-        int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            const int b = local & 1;
-            const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
-            const int arow = mb * BM + r_in_tile;   // A-operand row of this thread
-            const int brow0 = nb * BN;               // first B-operand row of the tile
-            float own_scale = 0.f;
-            float own_side[OC];
-#pragma unroll
-            for (int k = 0; k < OC; ++k)
-                own_side[k] = 0.f;
-            if (!RAW) {
-                // Stage the outlier operands and scales while the MMAs run.
-                named_barrier_sync(1, 128);
-                for (int idx = et; idx < BN; idx += 128) {
-                    const int r = brow0 + idx;
-                    s_scale[idx] = SWAP ? (r < p.M ? p.sx[r] : 0.f) : (r < p.N ? p.sb[r] : 0.f);
-                }
-                if (fast) {
-                    for (int idx = et; idx < cnt * BN; idx += 128) {
-                        const int k = idx / BN, c = idx - k * BN;
-                        const int r = brow0 + c;
-                        const int col = p.col_idx[k];
-                        float v = 0.f;
-                        if (SWAP) {
-                            if (r < p.M)
-                                v = __half2float(p.X16[(int64_t)r * p.K + col]);
-                        } else {
-                            if (r < p.N)
-                                v = wtilde(p, r, col);
-                        }
-                        s_side[idx] = v;
-                    }
-                }
-                if (SWAP) {
-                    if (arow < p.N) {
-                        own_scale = p.sb[arow];
-                        if (fast) {
-#pragma unroll
-                            for (int k = 0; k < OC; ++k)
-                                if (k < cnt)
-                                    own_side[k] = wtilde(p, arow, p.col_idx[k]);
-                        }
-                    }
-                } else {
-                    if (arow < p.M) {
-                        own_scale = p.sx[arow];
-                        if (fast) {
-#pragma unroll
-                            for (int k = 0; k < OC; ++k)
-                                if (k < cnt)
-                                    own_side[k] = __half2float(p.X16[(int64_t)arow * p.K + p.col_idx[k]]);
-                        }
-                    }
-                }
-                named_barrier_sync(1, 128);
-            }
-
-            // All 128 epilogue threads leave together if any of them gave up,
-            // so no thread is left waiting at a named barrier.
-            const bool got = mbar_wait(tfull_bar(b), tph[b]);
-            if (named_barrier_or(1, 128, !got)) {
-                if (!got)
-                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
-                break;
-            }
-            tph[b] ^= 1u;
-            tc_fence_after();
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
-
-            if constexpr (!SWAP) {
-                const int i = arow;
-#pragma unroll 1
-                for (int g = 0; g < BN / 32; ++g) {
-                    uint32_t acc[32];
-                    tmem_ld_32x32b_x32(tbase + g * 32, acc);
-                    tmem_wait_ld();
-                    const int j0 = brow0 + g * 32;
-                    if constexpr (RAW) {
-                        int32_t *Yr = reinterpret_cast<int32_t *>(p.Y) + (int64_t)i * p.N;
-                        if (i < p.M) {
-                            if (j0 + 32 <= p.N && (p.N & 3) == 0) {
-#pragma unroll
-                                for (int c = 0; c < 32; c += 4)
-                                    *reinterpret_cast<uint4 *>(Yr + j0 + c) =
-                                        make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-                            } else {
-                                for (int c = 0; c < 32; ++c)
-                                    if (j0 + c < p.N)
-                                        Yr[j0 + c] = (int32_t)acc[c];
-                            }
-                        }
-                        continue;
-                    }
-                    float y[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
-                    if (fast) {
-#pragma unroll
-                        for (int k = 0; k < OC; ++k) {
-                            if (k < cnt) {
-                                const float xv = own_side[k];
-                                const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
-#pragma unroll
-                                for (int c4 = 0; c4 < 8; ++c4) {
-                                    const float4 w = wrow[c4];
-                                    y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
-                                    y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
-                                    y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
-                                    y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
-                                }
-                            }
-                        }
-                    } else {
-                        // More outlier columns than one staged chunk holds.
-                        for (int ch = 0; ch < cnt; ch += OC) {
-                            const int nk = min(OC, cnt - ch);
-                            named_barrier_sync(1, 128);
-                            for (int idx = et; idx < nk * 32; idx += 128) {
-                                const int k = idx >> 5, c = idx & 31;
-                                const int j = j0 + c;
-                                s_side[idx] = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
-                            }
-                            named_barrier_sync(1, 128);
-                            for (int k = 0; k < nk; ++k) {
-                                const float xv =
-                                    i < p.M ? __half2float(p.X16[(int64_t)i * p.K + p.col_idx[ch + k]]) : 0.f;
-#pragma unroll
-                                for (int c = 0; c < 32; ++c)
-                                    y[c] = fmaf(xv, s_side[k * 32 + c], y[c]);
-                            }
-                        }
-                    }
-                    if (i < p.M) {
-                        __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
-                        if (j0 + 32 <= p.N && (p.N & 7) == 0) {
-#pragma unroll
-                            for (int c = 0; c < 32; c += 8) {
-                                uint4 pk;
-                                __half2 *h = reinterpret_cast<__half2 *>(&pk);
-                                h[0] = __floats2half2_rn(y[c + 0], y[c + 1]);
-                                h[1] = __floats2half2_rn(y[c + 2], y[c + 3]);
-                                h[2] = __floats2half2_rn(y[c + 4], y[c + 5]);
-                                h[3] = __floats2half2_rn(y[c + 6], y[c + 7]);
-                                *reinterpret_cast<uint4 *>(Yr + j0 + c) = pk;
-                            }
-                        } else {
-                            for (int c = 0; c < 32; ++c)
-                                if (j0 + c < p.N)
-                                    Yr[j0 + c] = __float2half_rn(y[c]);
-                        }
-                    }
-                }
-            } else {
-                // Decode form: this thread owns output feature j = arow; the
-                // accumulator columns are tokens brow0 .. brow0 + BN - 1.
-                const int j = arow;
-                uint32_t acc[BN];
-                if constexpr (BN == 32) {
-                    tmem_ld_32x32b_x32(tbase, acc);
-                } else {
-                    tmem_ld_32x32b_x16(tbase, acc);
-                }
-                tmem_wait_ld();
-                if constexpr (RAW) {
-                    if (j < p.N) {
-                        int32_t *Yc = reinterpret_cast<int32_t *>(p.Y) + j;
-#pragma unroll
-                        for (int c = 0; c < BN; ++c)
-                            if (brow0 + c < p.M)
-                                Yc[(int64_t)(brow0 + c) * p.N] = (int32_t)acc[c];
-                    }
-                } else {
-                    float y[BN];
-#pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
-                    if (fast) {
-#pragma unroll
-                        for (int k = 0; k < OC; ++k) {
-                            if (k < cnt) {
-                                const float wv = own_side[k];
-#pragma unroll
-                                for (int c = 0; c < BN; ++c)
-                                    y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
-                            }
-                        }
-                    } else {
-                        for (int ch = 0; ch < cnt; ch += OC) {
-                            const int nk = min(OC, cnt - ch);
-                            named_barrier_sync(1, 128);
-                            for (int idx = et; idx < nk * BN; idx += 128) {
-                                const int k = idx / BN, c = idx - k * BN;
-                                const int r = brow0 + c;
-                                s_side[idx] =
-                                    r < p.M ? __half2float(p.X16[(int64_t)r * p.K + p.col_idx[ch + k]]) : 0.f;
-                            }
-                            named_barrier_sync(1, 128);
-                            for (int k = 0; k < nk; ++k) {
-                                const float wv = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
-#pragma unroll
-                                for (int c = 0; c < BN; ++c)
-                                    y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
-                            }
-                        }
-                    }
-                    if (j < p.N) {
-                        __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
-#pragma unroll
-                        for (int c = 0; c < BN; ++c)
-                            if (brow0 + c < p.M)
-                                Yc[(int64_t)(brow0 + c) * p.N] = __float2half_rn(y[c]);
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(tempty_bar(b));
-        }
+        run_epilogue<BN, SWAP, RAW, false>(p, warp, lane, s_side, s_scale, tfull_bar(0), tempty_bar(0), s_abort,
+                                           tmem_base, blockIdx.x, gridDim.x, num_tiles, BM, 0);
     }
 
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
+}
+
+// Shared-memory layout of one CTA of a pair: A holds this CTA's 128 rows,
+// B its BN/2 rows, per stage.
+template <int BN, int STAGES>
+struct SmemPair {
+    static constexpr int A_BYTES = BM * BK;
+    static constexpr int B_BYTES = (BN / 2) * BK;
+    static constexpr int A_OFF = 0;
+    static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
+    static constexpr int SIDE_OFF = B_OFF + STAGES * B_BYTES;
+    static constexpr int SCALE_OFF = SIDE_OFF + OC * BN * 4;
+    static constexpr int BAR_OFF = SCALE_OFF + BN * 4;
+    static constexpr int NBARS = 2 * STAGES + 5;
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr uint32_t TMEM_COLS = (2 * BN) <= 256 ? 256 : 512;
+    static_assert(ALLOC <= 232448, "shared memory over the 227 KB per-CTA limit");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+    static_assert(BN % 32 == 0 && BN <= 256, "pair MMA needs N a multiple of 32, at most 256");
+};
+
+// The prefill GEMM on CTA pairs (a cluster of two CTAs on one TPC). Each pair
+// computes 256 x BN output tiles with tcgen05.mma.cta_group::2 (M = 256):
+// every CTA TMA-loads its own 128 A rows and BN/2 B rows per stage (no
+// multicast) and counts the bytes on the even CTA's barrier; the even CTA's
+// MMA thread waits there, issues the MMAs for the pair, and multicasts its
+// commits (stage free, accumulator ready) to both CTAs. Each CTA's epilogue
+// reads its own 128 accumulator rows from its TMEM and reports back to the
+// even CTA. Per MAC this moves half the operand bytes of the single-CTA form.
+template <int BN, int STAGES, bool RAW>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    k_gemm_i8_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const KParams p)
+{
+    using L = SmemPair<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    float *s_side = reinterpret_cast<float *>(smem + L::SIDE_OFF);
+    float *s_scale = reinterpret_cast<float *>(smem + L::SCALE_OFF);
+    const uint32_t bar0 = sbase + L::BAR_OFF;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);  // the even CTA's producer arms it for both CTAs' bytes
+            mbar_init(empty_bar(s), 1); // the pair's MMA commit
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 8); // 4 epilogue warps in each CTA
+        }
+        mbar_init(drain_bar, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(s_tmem), L::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    tc_fence_before();
+    cluster_sync_all(); // barriers and TMEM of both CTAs ready before any cross-CTA traffic
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int num_tiles = p.num_m_blk * p.num_n_blk;
+    const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            constexpr uint32_t TX = 2u * (uint32_t)(L::A_BYTES + L::B_BYTES);
+            for (int tile = pair_id; tile < num_tiles && !*s_abort; tile += num_pairs) {
+                const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
+                const int a_row = mb * 2 * BM + (int)rank * BM;
+                const int b_row = nb * BN + (int)rank * (BN / 2);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_PRODUCER);
+                        break;
+                    }
+                    if (*s_abort)
+                        break;
+                    if (leader)
+                        mbar_arrive_expect_tx(full_bar(stage), TX);
+                    tma_load_2d_pair(sbase + L::A_OFF + stage * L::A_BYTES, &tmA, full_bar(stage), kb * BK, a_row);
+                    tma_load_2d_pair(sbase + L::B_OFF + stage * L::B_BYTES, &tmB, full_bar(stage), kb * BK, b_row);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (leader && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t tph[2] = {0u, 0u};
+            constexpr uint32_t IDESC = idesc_i8(2 * BM, BN);
+            int local = 0;
+            for (int tile = pair_id; tile < num_tiles && !*s_abort; tile += num_pairs, ++local) {
+                const int b = local & 1;
+                if (!mbar_wait_cluster(tempty_bar(b), tph[b] ^ 1u)) {
+                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
+                    break;
+                }
+                tph[b] ^= 1u;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+                bool ok = true;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase)) {
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = sbase + L::A_OFF + stage * L::A_BYTES;
+                    const uint32_t b0 = sbase + L::B_OFF + stage * L::B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UK; ++k)
+                        mma_i8_pair(d_tmem, smem_desc_k128(a0 + k * UK), smem_desc_k128(b0 + k * UK), IDESC,
+                                    (kb | k) != 0 ? 1u : 0u);
+                    mma_commit_pair_mc(empty_bar(stage), 0x3); // both CTAs' stage is free
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                mma_commit_pair_mc(tfull_bar(b), 0x3); // both halves of accumulator b are ready
+            }
+            mma_commit_pair(drain_bar);
+            if (!mbar_wait(drain_bar, 0u))
+                report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
+        }
+        __syncwarp();
+    } else {
+        run_epilogue<BN, false, RAW, true>(p, warp, lane, s_side, s_scale, tfull_bar(0), tempty_bar(0), s_abort,
+                                           tmem_base, pair_id, num_pairs, num_tiles, 2 * BM, (int)rank * BM);
+    }
+
+    tc_fence_before();
+    cluster_sync_all(); // both CTAs done with TMEM and with each other's barriers
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
     }
 }
 
@@ -541,6 +733,104 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+template <int BN, int STAGES, bool RAW>
+cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+{
+    using L = SmemPair<BN, STAGES>;
+    auto kern = k_gemm_i8_pair<BN, STAGES, RAW>;
+    static std::atomic<uint64_t> configured{0};
+    const uint64_t bit = 1ull << (dev.device & 63);
+    if (!(configured.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+        if (e != cudaSuccess)
+            return e;
+        configured.fetch_or(bit);
+    }
+    CUtensorMap ta, tb;
+    if (!make_map_i8(&ta, a.A, a.M, a.K, BM) || !make_map_i8(&tb, a.B, a.N, a.K, BN / 2))
+        return cudaErrorInvalidValue;
+    KParams p;
+    p.rows_a = (int)a.M;
+    p.rows_b = (int)a.N;
+    p.K = (int)a.K;
+    p.num_m_blk = (int)((a.M + 2 * BM - 1) / (2 * BM));
+    p.num_n_blk = (int)((a.N + BN - 1) / BN);
+    p.num_kb = (int)((a.K + BK - 1) / BK);
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.sx = a.sx;
+    p.sb = a.sb;
+    p.X16 = reinterpret_cast<const __half *>(a.X16);
+    p.W16 = reinterpret_cast<const __half *>(a.W16);
+    p.CB = a.B;
+    p.col_idx = a.col_idx;
+    p.count = a.count;
+    p.Y = a.Y;
+    p.status = a.status;
+    const int tiles = p.num_m_blk * p.num_n_blk;
+    const int pairs = std::min(tiles, dev.num_sms / 2);
+    kern<<<2 * pairs, NTHREADS, L::ALLOC, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+// Tile width for CTA-pair tiles (256 x BN), chosen like pick_bn over the
+// number of pairs.
+int pick_bn_pair(int64_t M, int64_t N, int num_pairs)
+{
+    static const int cands[] = {256, 224, 192, 128};
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int bn : cands) {
+        const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + bn - 1) / bn);
+        const int64_t cost = ((tiles + num_pairs - 1) / num_pairs) * bn;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+// Tile width for the persistent prefill GEMM: the one that minimises the
+// number of tile waves times the tile width (a tile's main loop is
+// proportional to its width), preferring wider tiles on ties. 224 divides
+// 14336, 43008 and 57344 exactly, which removes the ragged last wave.
+int pick_bn(int64_t M, int64_t N, int num_sms)
+{
+    static const int cands[] = {256, 224, 192, 128};
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int bn : cands) {
+        const int64_t tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+        const int64_t waves = (tiles + num_sms - 1) / num_sms;
+        const int64_t cost = waves * bn;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+template <bool RAW>
+cudaError_t run_prefill(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (a.M >= 2 * BM && dev.num_sms >= 2) {
+        switch (pick_bn_pair(a.M, a.N, dev.num_sms / 2)) {
+        case 224: return run_pair<224, 6, RAW>(a, dev, stream);
+        case 192: return run_pair<192, 6, RAW>(a, dev, stream);
+        case 128: return run_pair<128, 8, RAW>(a, dev, stream);
+        default: return run_pair<256, 6, RAW>(a, dev, stream);
+        }
+    }
+    switch (pick_bn(a.M, a.N, dev.num_sms)) {
+    case 224: return run<224, 4, false, RAW>(a, dev, stream);
+    case 192: return run<192, 5, false, RAW>(a, dev, stream);
+    case 128: return run<128, 6, false, RAW>(a, dev, stream);
+    default: return run<256, 4, false, RAW>(a, dev, stream);
+    }
+}
+
 } // namespace
 
 cudaError_t launch_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
@@ -549,10 +839,10 @@ cudaError_t launch_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t s
         return cudaSuccess;
     const bool raw = a.epi == Epilogue::RawInt32;
     if (a.M <= 16)
-        return raw ? run<16, 8, true, true>(a, dev, stream) : run<16, 8, true, false>(a, dev, stream);
+        return raw ? run<16, 10, true, true>(a, dev, stream) : run<16, 10, true, false>(a, dev, stream);
     if (a.M <= 32)
-        return raw ? run<32, 8, true, true>(a, dev, stream) : run<32, 8, true, false>(a, dev, stream);
-    return raw ? run<256, 4, false, true>(a, dev, stream) : run<256, 4, false, false>(a, dev, stream);
+        return raw ? run<32, 10, true, true>(a, dev, stream) : run<32, 10, true, false>(a, dev, stream);
+    return raw ? run_prefill<true>(a, dev, stream) : run_prefill<false>(a, dev, stream);
 }
 
 } // namespace llmint8

@@ -10,17 +10,17 @@ namespace llmint8 {
 // Workspace layout (byte offsets; every region 256-byte aligned):
 //   [0]      uint32 status word (bits LLMINT8_DEV_*)
 //   [4]      int32  |O| (outlier column count)
+//   [8]      uint32 grid-barrier counter and generation, late-outlier flag
 //   [256]    uint32 outlier bitmap [ceil(K/32)]
 //   ...      int32  ascending outlier columns [K]
-//   ...      int32  per-row argmax column of the masked absmax [M]
 //   ...      fp32   SX [M]
 //   ...      int8   CX [M x K]
 struct Workspace {
     uint32_t *status;
     int32_t *count;
+    uint32_t *sync;
     uint32_t *bitmap;
     int32_t *col_idx;
-    int32_t *argmax;
     float *sx;
     int8_t *cx;
     size_t bytes;
@@ -40,15 +40,14 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, Workspace
     size_t nwords = (size_t)((K + 31) / 32);
     char *bm = take(nwords * 4);
     char *ci = take((size_t)K * 4);
-    char *am = take((size_t)M * 4);
     char *sx = with_codes ? take((size_t)M * 4) : nullptr;
     char *cx = with_codes ? take((size_t)M * (size_t)K) : nullptr;
     if (ws) {
         ws->status = reinterpret_cast<uint32_t *>(hdr);
         ws->count = hdr ? reinterpret_cast<int32_t *>(hdr + 4) : nullptr;
+        ws->sync = hdr ? reinterpret_cast<uint32_t *>(hdr + 8) : nullptr;
         ws->bitmap = reinterpret_cast<uint32_t *>(bm);
         ws->col_idx = reinterpret_cast<int32_t *>(ci);
-        ws->argmax = reinterpret_cast<int32_t *>(am);
         ws->sx = reinterpret_cast<float *>(sx);
         ws->cx = reinterpret_cast<int8_t *>(cx);
         ws->bytes = off;
@@ -65,14 +64,14 @@ struct DeviceInfo {
 // Cached per-device properties (first call per device queries them).
 cudaError_t device_info(DeviceInfo *out);
 
-// K1 + K2: quantize rows of X (fp16) with outlier detection at threshold t.
-// Writes codes, absmax, the outlier bitmap and (when t > 0) fixes up rows whose
-// masked maximum sat in a column that turned out to be an outlier, zeroes the
-// codes of every outlier column, and compacts the bitmap into col_idx/count.
-// `bitmap` and `count` must be zeroed on the stream before the call.
+// Quantize rows of X (fp16) with outlier detection at threshold t: codes,
+// absmax over the non-outlier columns, the outlier bitmap and (t > 0) its
+// compaction into col_idx/count. `bitmap` must be zeroed before the call.
+// `sync` is two zeroed uint32 words (grid barrier); `status` receives
+// LLMINT8_DEV_* bits.
 cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes,
-                            float *absmax, uint32_t *bitmap, int32_t *argmax, int32_t *col_idx,
-                            int32_t *count, const DeviceInfo &dev, cudaStream_t stream);
+                            float *absmax, uint32_t *bitmap, int32_t *col_idx, int32_t *count, uint32_t *sync,
+                            uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
 
 // Bitmap -> ascending column list and count (one CTA).
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

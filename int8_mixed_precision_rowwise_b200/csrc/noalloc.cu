@@ -7,11 +7,11 @@
 // running inside a host process that forbids device allocations after
 // initialisation, or a latency-critical loop where an allocation's implicit
 // device synchronisation is not acceptable. They still own the inputs and
-// outputs; only the quantizer's small scratch (per-row argmax columns, the
-// compacted outlier list and its count) moves into the fixed array below.
+// outputs; only the quantizer's small scratch (the compacted outlier list,
+// its count and the kernel's barrier words) moves into the fixed array below.
 //
 // The array lives in this library's module, so every GPU that uses this entry
-// point holds it (about 512 KB) from its first call until the process exits.
+// point holds it (about 256 KB) from its first call until the process exits.
 // All calls on a device share it and it keeps the last call's contents, so
 // two calls whose work overlaps on the GPU (different streams, no ordering
 // between them) race on it; calls ordered on one stream are safe.
@@ -29,9 +29,8 @@ namespace {
 
 constexpr int64_t kMaxRows = LLMINT8_NOALLOC_MAX_ROWS;
 constexpr int64_t kMaxCols = LLMINT8_NOALLOC_MAX_COLS;
-constexpr size_t kHeaderBytes = 256; // int32 |O| at offset 0
-constexpr size_t kArgmaxOff = kHeaderBytes;
-constexpr size_t kColIdxOff = kArgmaxOff + (size_t)kMaxRows * 4;
+constexpr size_t kHeaderBytes = 256; // int32 |O| at 0, uint32 status at 4, grid-barrier words at 8
+constexpr size_t kColIdxOff = kHeaderBytes;
 constexpr size_t kScratchBytes = kColIdxOff + (size_t)kMaxCols * 4;
 
 // The scratch. In host code this name is only a stand-in: the device address
@@ -92,16 +91,17 @@ extern "C" llmint8_status llmint8_quantize_rowwise_noalloc(const void *X_f16, in
         return LLMINT8_ERR_CUDA;
     char *s = static_cast<char *>(base);
     int32_t *count = reinterpret_cast<int32_t *>(s);
-    int32_t *argmax = reinterpret_cast<int32_t *>(s + kArgmaxOff);
+    uint32_t *status = reinterpret_cast<uint32_t *>(s + 4);
+    uint32_t *sync = reinterpret_cast<uint32_t *>(s + 8);
     int32_t *col_idx = reinterpret_cast<int32_t *>(s + kColIdxOff);
-    // The array keeps the previous call's contents: clear the count, and the
-    // caller's bitmap, which the kernels OR into.
-    if (cudaMemsetAsync(count, 0, sizeof(int32_t), stream) != cudaSuccess)
+    // The array keeps the previous call's contents: clear the count, status
+    // and grid-barrier words, and the caller's bitmap, which the kernels OR into.
+    if (cudaMemsetAsync(count, 0, 24, stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     if (outlier_bitmap &&
         cudaMemsetAsync(outlier_bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    cudaError_t e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, argmax, col_idx,
-                                    count, dev, stream);
+    cudaError_t e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, col_idx, count, sync,
+                                    status, dev, stream);
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
 }

@@ -7,21 +7,30 @@
 // quantized per row (sections "LLM.int8() 的简要总结" and "MatMul 内部").
 //
 // The outlier set O is a property of the whole matrix, yet each row's scale
-// must exclude O. K1 reads X exactly once: each CTA keeps a shared-memory copy
-// of the columns already known to be outliers (its own discoveries plus the
-// global bitmap, refreshed at every row) and takes the row maximum over the
-// other columns with |x| < t, recording the column where it sits. That masked
-// maximum is never below the true one (known columns are a subset of O, and
-// every column outside O has |x| < t), and equals it whenever the recorded
-// column is outside the final O. K2 re-quantizes exactly the rows whose
-// recorded column ended up in O, zeroes the codes of every column of O, and
-// compacts the bitmap into ascending column indices.
+// must exclude O. One fused, cooperatively launched kernel does it:
+//   seed      a bounded subset of rows (about 2 MB) is read only to find
+//             outlier columns; systematic outlier columns show up in most
+//             rows, so this almost always finds all of O;
+//   quantize  every row zeroes its known outlier columns, takes its maximum
+//             |x| and writes its codes (seeded rows come back from L2);
+//   finish    compaction of O; only if some column first reached t during
+//             the quantize step are the affected rows re-quantized and the
+//             new columns' codes zeroed.
+// Both paths give exactly the definition's result. The maximum runs on
+// packed fp16 pairs, the outlier test compares against the smallest fp16 >= t
+// (exact for fp16 inputs), and the codes round with the 1.5 * 2^23 trick,
+// which is round-half-even like rintf.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "internal.h"
+#include "llmint8.h"
+#include "ptx.cuh"
 
 namespace llmint8 {
 
@@ -52,250 +61,6 @@ __device__ __forceinline__ uint2 pack8(const int (&q)[8])
     r.y = (uint32_t)(q[4] & 0xFF) | ((uint32_t)(q[5] & 0xFF) << 8) | ((uint32_t)(q[6] & 0xFF) << 16) |
           ((uint32_t)(q[7] & 0xFF) << 24);
     return r;
-}
-
-template <int NT>
-__device__ __forceinline__ unsigned long long block_max_u64(unsigned long long v, unsigned long long *s_red)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-        v = w > v ? w : v;
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0)
-        s_red[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        v = lane < NT / 32 ? s_red[lane] : 0ull;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
-            v = w > v ? w : v;
-        }
-        if (lane == 0)
-            s_red[0] = v;
-    }
-    __syncthreads();
-    v = s_red[0];
-    __syncthreads();
-    return v;
-}
-
-template <int NT>
-__device__ __forceinline__ float block_max_f32(float v, float *s_red)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0)
-        s_red[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        v = lane < NT / 32 ? s_red[lane] : 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0)
-            s_red[0] = v;
-    }
-    __syncthreads();
-    v = s_red[0];
-    __syncthreads();
-    return v;
-}
-
-// Key ordering (value desc, column asc) so a max-reduction returns the
-// largest |x| and, among equal values, the smallest column.
-__device__ __forceinline__ unsigned long long amax_key(float a, int c)
-{
-    return ((unsigned long long)__float_as_uint(a) << 32) | (uint32_t)(~(uint32_t)c);
-}
-
-// Merge the global outlier bitmap into the CTA's known set.
-template <int NT>
-__device__ __forceinline__ void refresh_known(uint32_t *s_known, const uint32_t *bitmap, int nwords)
-{
-    for (int w = threadIdx.x; w < nwords; w += NT) {
-        uint32_t g = *reinterpret_cast<const volatile uint32_t *>(bitmap + w);
-        if (g & ~s_known[w])
-            atomicOr(&s_known[w], g);
-    }
-}
-
-// Record newly seen outlier columns (bits of word w) in the CTA set and, if
-// they were new to this CTA, in the global bitmap.
-__device__ __forceinline__ void publish_outliers(uint32_t *s_known, uint32_t *bitmap, int w, uint32_t bits)
-{
-    uint32_t old = atomicOr(&s_known[w], bits);
-    uint32_t fresh = bits & ~old;
-    if (fresh)
-        atomicOr(&bitmap[w], fresh);
-}
-
-// K1, register-resident rows: NT threads per row, V 16-byte vectors each
-// (NT * V * 8 >= cols). One CTA walks rows blockIdx.x, +gridDim.x, ...
-template <int NT, int V>
-__global__ void __launch_bounds__(NT) k_quantize_rows(const uint4 *__restrict__ X, int64_t rows, int cols,
-                                                      float t, int8_t *__restrict__ codes,
-                                                      float *__restrict__ absmax,
-                                                      int32_t *__restrict__ argmax,
-                                                      uint32_t *__restrict__ bitmap)
-{
-    extern __shared__ uint32_t s_known[];
-    __shared__ unsigned long long s_red[NT / 32];
-    const int tid = threadIdx.x;
-    const int nvec = cols >> 3;
-    const int nwords = (cols + 31) >> 5;
-    const bool thr = t > 0.f;
-
-    if (thr) {
-        for (int w = tid; w < nwords; w += NT)
-            s_known[w] = 0u;
-    }
-
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const uint4 *xr = X + r * (int64_t)nvec;
-        uint4 v[V];
-#pragma unroll
-        for (int u = 0; u < V; ++u) {
-            const int vi = u * NT + tid;
-            v[u] = vi < nvec ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        uint32_t kbits[V];
-#pragma unroll
-        for (int u = 0; u < V; ++u)
-            kbits[u] = 0u;
-        if (thr) {
-            __syncthreads(); // s_known initialised / previous row's readers done
-            refresh_known<NT>(s_known, bitmap, nwords);
-            __syncthreads();
-#pragma unroll
-            for (int u = 0; u < V; ++u) {
-                const int vi = u * NT + tid;
-                if (vi < nvec)
-                    kbits[u] = (s_known[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
-            }
-        }
-
-        unsigned long long key = 0ull;
-#pragma unroll
-        for (int u = 0; u < V; ++u) {
-            const int vi = u * NT + tid;
-            if (vi >= nvec)
-                continue;
-            float x[8];
-            unpack8(v[u], x);
-            uint32_t hit = 0u;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float a = fabsf(x[e]);
-                if (thr && a >= t) {
-                    hit |= 1u << e;
-                } else if (!((kbits[u] >> e) & 1u)) {
-                    const unsigned long long k = amax_key(a, vi * 8 + e);
-                    key = k > key ? k : key;
-                }
-            }
-            if (hit & ~kbits[u])
-                publish_outliers(s_known, bitmap, vi >> 2, (hit & ~kbits[u]) << ((vi & 3) * 8));
-            kbits[u] |= hit;
-        }
-
-        key = block_max_u64<NT>(key, s_red);
-        const float amax = __uint_as_float((uint32_t)(key >> 32));
-        const int acol = (int)(~(uint32_t)key);
-        const float s = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-
-        int8_t *cr = codes + r * (int64_t)cols;
-#pragma unroll
-        for (int u = 0; u < V; ++u) {
-            const int vi = u * NT + tid;
-            if (vi >= nvec)
-                continue;
-            float x[8];
-            unpack8(v[u], x);
-            int q[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                q[e] = ((kbits[u] >> e) & 1u) ? 0 : quant1(x[e], s);
-            *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) = pack8(q);
-        }
-        if (tid == 0) {
-            absmax[r] = amax;
-            argmax[r] = amax > 0.f ? acol : -1;
-        }
-    }
-}
-
-// K1 for rows too long to hold in registers (cols > 65536): the same
-// arithmetic, with the row read twice (the second read is served by L2).
-template <int NT>
-__global__ void __launch_bounds__(NT) k_quantize_rows_loop(const uint4 *__restrict__ X, int64_t rows,
-                                                           int cols, float t, int8_t *__restrict__ codes,
-                                                           float *__restrict__ absmax,
-                                                           int32_t *__restrict__ argmax,
-                                                           uint32_t *__restrict__ bitmap)
-{
-    extern __shared__ uint32_t s_known[];
-    __shared__ unsigned long long s_red[NT / 32];
-    const int tid = threadIdx.x;
-    const int nvec = cols >> 3;
-    const int nwords = (cols + 31) >> 5;
-    const bool thr = t > 0.f;
-    if (thr) {
-        for (int w = tid; w < nwords; w += NT)
-            s_known[w] = 0u;
-    }
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const uint4 *xr = X + r * (int64_t)nvec;
-        if (thr) {
-            __syncthreads();
-            refresh_known<NT>(s_known, bitmap, nwords);
-            __syncthreads();
-        }
-        unsigned long long key = 0ull;
-        for (int vi = tid; vi < nvec; vi += NT) {
-            float x[8];
-            unpack8(__ldg(xr + vi), x);
-            uint32_t kb = thr ? (s_known[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu : 0u;
-            uint32_t hit = 0u;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float a = fabsf(x[e]);
-                if (thr && a >= t) {
-                    hit |= 1u << e;
-                } else if (!((kb >> e) & 1u)) {
-                    const unsigned long long k = amax_key(a, vi * 8 + e);
-                    key = k > key ? k : key;
-                }
-            }
-            if (hit & ~kb)
-                publish_outliers(s_known, bitmap, vi >> 2, (hit & ~kb) << ((vi & 3) * 8));
-        }
-        key = block_max_u64<NT>(key, s_red);
-        const float amax = __uint_as_float((uint32_t)(key >> 32));
-        const int acol = (int)(~(uint32_t)key);
-        const float s = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-        int8_t *cr = codes + r * (int64_t)cols;
-        for (int vi = tid; vi < nvec; vi += NT) {
-            float x[8];
-            unpack8(__ldg(xr + vi), x);
-            // Within one row the known set only gains columns whose element in
-            // this row is itself >= t, so this mask agrees with the first pass.
-            uint32_t kb = thr ? (s_known[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu : 0u;
-            int q[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                q[e] = (((kb >> e) & 1u) || (thr && fabsf(x[e]) >= t)) ? 0 : quant1(x[e], s);
-            *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) = pack8(q);
-        }
-        if (tid == 0) {
-            absmax[r] = amax;
-            argmax[r] = amax > 0.f ? acol : -1;
-        }
-    }
 }
 
 // Ascending list of the set bits of s_bm[0..nwords) written by one CTA.
@@ -357,141 +122,498 @@ __global__ void __launch_bounds__(NT) k_compact(const uint32_t *__restrict__ bit
     compact_block<NT>(s_bm, nwords, col_idx, count);
 }
 
-// K2: with the final outlier set known, (a) CTA 0 compacts it, (b) rows whose
-// masked maximum sat in an outlier column are re-quantized over the
-// non-outlier columns, and (c) every other row gets its outlier-column codes
-// zeroed.
-template <int NT>
-__global__ void __launch_bounds__(NT) k_fixup_rows(const uint4 *__restrict__ X, int64_t rows, int cols,
-                                                   int8_t *__restrict__ codes, float *__restrict__ absmax,
-                                                   const int32_t *__restrict__ argmax,
-                                                   const uint32_t *__restrict__ bitmap,
-                                                   int32_t *__restrict__ col_idx, int32_t *__restrict__ count)
+// One bounded grid-wide barrier (all CTAs are co-resident: the kernel is
+// launched cooperatively). sync[0] counts arrivals, sync[1] is the generation.
+__device__ bool grid_barrier(uint32_t *sync, uint32_t nblocks)
 {
-    extern __shared__ uint32_t s_bm[];
-    __shared__ float s_red[NT / 32];
-    const int tid = threadIdx.x;
-    const int nwords = (cols + 31) >> 5;
-    const int nvec = cols >> 3;
-    for (int w = tid; w < nwords; w += NT)
-        s_bm[w] = bitmap[w];
-    __syncthreads();
-    if (blockIdx.x == 0)
-        compact_block<NT>(s_bm, nwords, col_idx, count);
+    uint32_t g, prev;
+    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(g) : "l"(sync + 1) : "memory");
+    asm volatile("atom.acq_rel.gpu.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(sync) : "memory");
+    if (prev + 1 == nblocks) {
+        asm volatile("st.relaxed.gpu.u32 [%0], 0;" ::"l"(sync) : "memory");
+        asm volatile("red.release.gpu.add.u32 [%0], 1;" ::"l"(sync + 1) : "memory");
+        return true;
+    }
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        uint32_t cur;
+        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(sync + 1) : "memory");
+        if (cur != g)
+            return true;
+        if (global_timer_ns() - t0 > kWaitLimitNs)
+            return false;
+        __nanosleep(64);
+    }
+}
 
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const int am = argmax[r];
-        int8_t *cr = codes + r * (int64_t)cols;
-        if (am >= 0 && ((s_bm[am >> 5] >> (am & 31)) & 1u)) {
-            const uint4 *xr = X + r * (int64_t)nvec;
-            float m = 0.f;
-            for (int vi = tid; vi < nvec; vi += NT) {
-                float x[8];
-                unpack8(__ldg(xr + vi), x);
-                const uint32_t kb = (s_bm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+// Per 16-byte vector (8 fp16 values): |x| as half2 pairs and their maximum.
+__device__ __forceinline__ __half2 vec_abs_max(const uint4 &v, __half2 (&a)[4])
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (!((kb >> e) & 1u))
-                        m = fmaxf(m, fabsf(x[e]));
-            }
-            const float amax = block_max_f32<NT>(m, s_red);
-            const float s = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-            for (int vi = tid; vi < nvec; vi += NT) {
-                float x[8];
-                unpack8(__ldg(xr + vi), x);
-                const uint32_t kb = (s_bm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
-                int q[8];
+    for (int i = 0; i < 4; ++i)
+        a[i] = __habs2(h[i]);
+    return __hmax2(__hmax2(a[0], a[1]), __hmax2(a[2], a[3]));
+}
+
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Codes of 8 fp16 values with multiplier s: per value the fp32 product x * s
+// rounded to nearest even, then rint() of it by adding 1.5 * 2^23 in
+// round-to-nearest-even (the low byte of the sum is the code). The two
+// roundings must stay separate (no fused multiply-add), as in the definition.
+__device__ __forceinline__ uint2 codes8(const uint4 &v, float s)
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+    uint32_t b[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    q[e] = ((kb >> e) & 1u) ? 0 : quant1(x[e], s);
-                *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) = pack8(q);
-            }
-            if (tid == 0)
-                absmax[r] = amax;
-        } else {
-            for (int w = tid; w < nwords; w += NT) {
-                uint32_t bits = s_bm[w];
-                while (bits) {
-                    const int b = __ffs(bits) - 1;
-                    cr[w * 32 + b] = 0;
-                    bits &= bits - 1u;
-                }
-            }
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        b[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(f.x, s), 12582912.0f));
+        b[2 * i + 1] = __float_as_uint(__fadd_rn(__fmul_rn(f.y, s), 12582912.0f));
+    }
+    return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+}
+
+// Zero the fp16 values of a 16-byte vector whose bit is set in `kbyte`
+// (bit e = element e): known outlier columns drop out of the maximum and get
+// code 0.
+__device__ __forceinline__ void mask_known(uint4 &v, uint32_t kbyte)
+{
+    uint32_t *w = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t m = (kbyte >> (2 * i)) & 3u;
+        w[i] &= ~(((m & 1u) * 0x0000FFFFu) | ((m >> 1) * 0xFFFF0000u));
+    }
+}
+
+__device__ __forceinline__ uint32_t known_byte(const uint32_t *s_known, int vi)
+{
+    return (s_known[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+}
+
+// Record the columns of one vector with |x| >= t16 in the CTA set and the
+// global bitmap; returns true if one of them was new to the bitmap.
+__device__ __forceinline__ bool publish_vector(const uint4 &v, int vi, __half t16, uint32_t *s_known,
+                                               uint32_t *bitmap)
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+    uint32_t hit = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 a = __habs2(h[i]);
+        if (__hge(__low2half(a), t16))
+            hit |= 1u << (2 * i);
+        if (__hge(__high2half(a), t16))
+            hit |= 2u << (2 * i);
+    }
+    if (!hit)
+        return false;
+    const uint32_t bits = hit << ((vi & 3) * 8);
+    const uint32_t old = atomicOr(&s_known[vi >> 2], bits);
+    if (!(bits & ~old))
+        return false;
+    const uint32_t gold = atomicOr(&bitmap[vi >> 2], bits & ~old);
+    return ((bits & ~old) & ~gold) != 0u;
+}
+
+// Seed: find the outlier columns of one row (no codes).
+template <int GS, int V, bool FULL>
+__device__ __forceinline__ void row_seed(const uint4 *__restrict__ xr, int nvec, int gl, __half t16,
+                                         uint32_t *s_known, uint32_t *bitmap)
+{
+    const __half2 t2 = __half2half2(t16);
+    for (int c0 = 0; c0 < nvec; c0 += GS * V) {
+        uint4 v[V];
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int vi = c0 + u * GS + gl;
+            v[u] = (FULL || vi < nvec) ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            __half2 a[4];
+            const __half2 vm = vec_abs_max(v[u], a);
+            if (__hbgt2(t2, vm)) // both halves below t: no outlier in these 8 columns
+                continue;
+            (void)publish_vector(v[u], c0 + u * GS + gl, t16, s_known, bitmap);
         }
     }
 }
 
-template <int NT, int V>
-cudaError_t launch_k1(const void *X, int64_t rows, int cols, float t, int8_t *codes, float *absmax,
-                      int32_t *argmax, uint32_t *bitmap, const DeviceInfo &dev, cudaStream_t stream)
+// Maximum |x| of one row over the columns not known as outliers, for a group
+// of GS threads holding V vectors each per chunk. Known columns are zeroed in
+// `v` in place. `kb4` holds this thread's known-column bytes of the first
+// chunk (resident rows); longer rows read them from s_known.
+template <int GS, int V, bool THR, bool FULL>
+__device__ __forceinline__ float row_max(const uint4 *__restrict__ xr, int nvec, int gl, bool resident,
+                                         const uint32_t *s_known, const uint32_t (&kb4)[(V + 3) / 4],
+                                         uint4 (&v)[V])
 {
-    const size_t smem = (size_t)((cols + 31) / 32) * 4;
-    auto kern = k_quantize_rows<NT, V>;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem);
-    if (e != cudaSuccess)
-        return e;
-    per_sm = std::max(per_sm, 1);
-    const int64_t grid = std::min<int64_t>(rows, (int64_t)per_sm * dev.num_sms);
-    kern<<<(unsigned)grid, NT, smem, stream>>>(reinterpret_cast<const uint4 *>(X), rows, cols, t, codes,
-                                               absmax, argmax, bitmap);
-    return cudaGetLastError();
+    __half2 m2 = __float2half2_rn(0.f);
+    for (int c0 = 0; c0 < nvec; c0 += GS * V) {
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int vi = c0 + u * GS + gl;
+            v[u] = (FULL || vi < nvec) ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            if constexpr (THR) {
+                const int vi = c0 + u * GS + gl;
+                const uint32_t kbyte = resident ? (kb4[u >> 2] >> ((u & 3) * 8)) & 0xFFu
+                                                : ((FULL || vi < nvec) ? known_byte(s_known, vi) : 0u);
+                if (kbyte)
+                    mask_known(v[u], kbyte);
+            }
+            __half2 a[4];
+            m2 = __hmax2(m2, vec_abs_max(v[u], a));
+        }
+    }
+    return fmaxf(__low2float(m2), __high2float(m2));
 }
 
-template <int NT>
-cudaError_t launch_k1_nt(const void *X, int64_t rows, int cols, float t, int8_t *codes, float *absmax,
-                         int32_t *argmax, uint32_t *bitmap, const DeviceInfo &dev, cudaStream_t stream,
-                         int v)
+// Codes of one row with multiplier s: rint(x * s), zero for known outlier
+// columns. Uses `v` (already masked) for resident rows, else reads the row
+// again and masks it.
+template <int GS, int V, bool THR, bool FULL>
+__device__ __forceinline__ void row_codes(const uint4 *__restrict__ xr, int nvec, int gl, bool resident,
+                                          const uint32_t *s_known, float s, uint4 (&v)[V], int8_t *__restrict__ cr)
 {
-    switch (v) {
-    case 1: return launch_k1<NT, 1>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream);
-    case 2: return launch_k1<NT, 2>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream);
-    case 4: return launch_k1<NT, 4>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream);
-    default: return launch_k1<NT, 8>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream);
+    for (int c0 = 0; c0 < nvec; c0 += GS * V) {
+        if (!resident) {
+#pragma unroll
+            for (int u = 0; u < V; ++u) {
+                const int vi = c0 + u * GS + gl;
+                v[u] = (FULL || vi < nvec) ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+                if constexpr (THR) {
+                    if (FULL || vi < nvec) {
+                        const uint32_t kbyte = known_byte(s_known, vi);
+                        if (kbyte)
+                            mask_known(v[u], kbyte);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int vi = c0 + u * GS + gl;
+            if (FULL || vi < nvec)
+                *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) = codes8(v[u], s);
+        }
     }
+}
+
+// Maximum of a float over a row group of WPR warps (WPR = 1: one warp;
+// WPR = 8: the whole CTA, through shared memory; `buf` alternates per row so
+// one __syncthreads per reduction suffices).
+template <int WPR>
+__device__ __forceinline__ float group_max_f32(float v, float *buf)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if constexpr (WPR > 1) {
+        if ((threadIdx.x & 31) == 0)
+            buf[threadIdx.x >> 5] = v;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < WPR; ++i)
+            v = fmaxf(v, buf[i]);
+    }
+    return v;
+}
+
+// Quantize one row with one group of WPR warps: zero its known outlier
+// columns, take the maximum |x|, write codes and absmax. With THR, a row that
+// holds a column >= t not yet in s_known publishes it, raises *new_flag and
+// gets absmax -1 (a marker: the finish step quantizes it again).
+template <int WPR, int V, bool THR, bool FULL>
+__device__ __forceinline__ void quantize_row(const uint4 *__restrict__ xr, int64_t r, int cols, float t, __half t16,
+                                             bool resident, uint32_t *s_known, uint32_t *bitmap, uint32_t *new_flag,
+                                             const uint32_t (&kb4)[(V + 3) / 4], uint4 (&v)[V],
+                                             int8_t *__restrict__ codes, float *__restrict__ absmax, float *red)
+{
+    constexpr int GS = 32 * WPR;
+    const int gl = ((threadIdx.x >> 5) % WPR) * 32 + (threadIdx.x & 31);
+    const int nvec = cols >> 3;
+    float amax = row_max<GS, V, THR, FULL>(xr, nvec, gl, resident, s_known, kb4, v);
+    amax = group_max_f32<WPR>(amax, red);
+    if (THR && amax >= t) {
+        for (int vi = gl; vi < nvec; vi += GS)
+            if (publish_vector(__ldg(xr + vi), vi, t16, s_known, bitmap))
+                atomicOr(new_flag, 1u);
+        if (gl == 0) {
+            atomicOr(new_flag, 1u);
+            absmax[r] = -1.f;
+        }
+        return;
+    }
+    const float s = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+    row_codes<GS, V, THR, FULL>(xr, nvec, gl, resident, s_known, s, v, codes + r * (int64_t)cols);
+    if (gl == 0)
+        absmax[r] = amax;
+}
+
+template <int GS, int V>
+__device__ __forceinline__ void load_known_bytes(const uint32_t *s_known, int nvec, int gl, bool resident,
+                                                 uint32_t (&kb4)[(V + 3) / 4])
+{
+#pragma unroll
+    for (int i = 0; i < (V + 3) / 4; ++i)
+        kb4[i] = 0u;
+    if (resident) {
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int vi = u * GS + gl;
+            if (vi < nvec)
+                kb4[u >> 2] |= known_byte(s_known, vi) << ((u & 3) * 8);
+        }
+    }
+}
+
+constexpr int kMaxLate = 64; // late outlier columns handled by the cheap path
+
+// Fused quantizer, one row per group of WPR warps (WPR = 1: a warp per row;
+// WPR = 8: the whole CTA per row). With a threshold (THR):
+//   seed     - every `seed_stride`-th group reads its first row only to find
+//              outlier columns (|x| >= t); these rows come back from L2 in
+//              the next step;
+//   barrier  - then each CTA loads the outlier set found so far (the "seed
+//              set", also kept aside);
+//   quantize - every row: maximum over the columns not known as outliers,
+//              codes and absmax;
+//   barrier  - then CTA 0 compacts the final outlier set. If no column first
+//              reached t during the quantize step (flag sync[2]), every row
+//              was coded against the final set and the kernel is done.
+//              Otherwise, with L = final set minus seed set, each group
+//              re-quantizes those of its rows that were marked, or whose
+//              maximum equals |x| at a column of L, and zeroes the L-column
+//              codes of its other rows (every row, when |L| > kMaxLate).
+// Without a threshold only the quantize step runs. FULL: the row length is a
+// multiple of the chunk (no bounds checks). A row of at most 32 * WPR * V
+// 16-byte vectors stays in registers between its maximum and its codes; a
+// longer one is read twice.
+template <int WPR, int V, bool THR, bool FULL>
+__global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X, int64_t rows, int cols, float t,
+                                                     __half t16, int8_t *__restrict__ codes,
+                                                     float *__restrict__ absmax, uint32_t *__restrict__ bitmap,
+                                                     int32_t *__restrict__ col_idx, int32_t *__restrict__ count,
+                                                     uint32_t *__restrict__ sync, uint32_t *__restrict__ status,
+                                                     int seed_stride)
+{
+    constexpr int GROUPS = 8 / WPR; // row groups per CTA
+    constexpr int GS = 32 * WPR;    // threads per group
+    extern __shared__ uint32_t s_dyn[];
+    __shared__ float s_red[2][8];
+    __shared__ int s_flag, s_nlate;
+    __shared__ int s_late[kMaxLate];
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int grp = warp / WPR, gl = (warp % WPR) * 32 + (tid & 31);
+    const int64_t gid = (int64_t)blockIdx.x * GROUPS + grp;
+    const int64_t G = (int64_t)gridDim.x * GROUPS;
+    const int nvec = cols >> 3, nwords = (cols + 31) >> 5;
+    const bool resident = nvec <= GS * V;
+    uint32_t *s_known = s_dyn;         // [nwords]
+    uint32_t *s_seed = s_dyn + nwords; // [nwords]
+    uint32_t kb4[(V + 3) / 4];
+    uint4 v[V];
+
+    if constexpr (THR) {
+        for (int w = tid; w < nwords; w += 256)
+            s_known[w] = 0u;
+        __syncthreads();
+        if (gid < rows && gid % seed_stride == 0)
+            row_seed<GS, V, FULL>(X + gid * (int64_t)nvec, nvec, gl, t16, s_known, bitmap);
+        __syncthreads();
+        if (tid == 0) {
+            s_flag = grid_barrier(sync, gridDim.x) ? 1 : 0;
+            if (!s_flag)
+                atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
+        }
+        __syncthreads();
+        if (!s_flag)
+            return;
+        for (int w = tid; w < nwords; w += 256)
+            s_known[w] = s_seed[w] = __ldcg(bitmap + w);
+        __syncthreads();
+    }
+
+    load_known_bytes<GS, V>(s_known, nvec, gl, THR && resident, kb4);
+    int it = 0;
+    for (int64_t r = gid; r < rows; r += G, ++it)
+        quantize_row<WPR, V, THR, FULL>(X + r * (int64_t)nvec, r, cols, t, t16, resident, s_known, bitmap,
+                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1]);
+    if constexpr (!THR)
+        return;
+
+    // ---- finish
+    __syncthreads();
+    if (tid == 0) {
+        s_flag = grid_barrier(sync, gridDim.x) ? 1 : 0;
+        if (!s_flag)
+            atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
+    }
+    __syncthreads();
+    if (!s_flag)
+        return;
+    for (int w = tid; w < nwords; w += 256)
+        s_known[w] = __ldcg(bitmap + w);
+    __syncthreads();
+    if (blockIdx.x == 0)
+        compact_block<256>(s_known, nwords, col_idx, count);
+    if (__ldcg(sync + 2) == 0u)
+        return; // every row was coded against the complete outlier set
+
+    // Late columns: in the final set but not in the seed set.
+    if (tid == 0)
+        s_nlate = 0;
+    __syncthreads();
+    for (int w = tid; w < nwords; w += 256) {
+        uint32_t bits = s_known[w] & ~s_seed[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            const int k = atomicAdd(&s_nlate, 1);
+            if (k < kMaxLate)
+                s_late[k] = w * 32 + b;
+            bits &= bits - 1u;
+        }
+    }
+    __syncthreads();
+    const int nlate = s_nlate;
+    load_known_bytes<GS, V>(s_known, nvec, gl, resident, kb4);
+    it = 0;
+    for (int64_t r = gid; r < rows; r += G, ++it) {
+        const float a = __ldcg(absmax + r);
+        const __half *xh = reinterpret_cast<const __half *>(X + r * (int64_t)nvec);
+        bool redo = a < 0.f || nlate > kMaxLate;
+        if (!redo) {
+            for (int k = gl; k < nlate; k += GS)
+                redo |= a > 0.f && __half2float(__habs(xh[s_late[k]])) == a;
+        }
+        if constexpr (WPR == 1)
+            redo = __any_sync(0xffffffffu, redo);
+        else
+            redo = __syncthreads_or(redo);
+        if (redo) {
+            quantize_row<WPR, V, true, FULL>(X + r * (int64_t)nvec, r, cols, t, t16, resident, s_known, bitmap,
+                                             sync + 2, kb4, v, codes, absmax, s_red[it & 1]);
+        } else {
+            for (int k = gl; k < nlate; k += GS)
+                codes[r * (int64_t)cols + s_late[k]] = 0;
+        }
+    }
+}
+
+// The smallest fp16 value >= t, so that for fp16 x, |x| >= t exactly when
+// |x| >= t16 (t above the fp16 range: no finite value qualifies).
+__half threshold_fp16(float t)
+{
+    if (!(t > 0.f))
+        return __float2half(0.f);
+    if (t > 65504.f)
+        return __ushort_as_half((unsigned short)0x7C00u); // +inf
+    __half h = __float2half_rn(t);
+    if (__half2float(h) < t)
+        h = __ushort_as_half((unsigned short)(__half_as_ushort(h) + 1u));
+    return h;
+}
+
+template <int WPR, int V, bool THR, bool FULL>
+cudaError_t launch_fused(const void *X, int64_t rows, int cols, float t, int8_t *codes, float *absmax,
+                         uint32_t *bitmap, int32_t *col_idx, int32_t *count, uint32_t *sync, uint32_t *status,
+                         const DeviceInfo &dev, cudaStream_t stream)
+{
+    constexpr int GROUPS = 8 / WPR;
+    const size_t smem = THR ? (size_t)((cols + 31) / 32) * 4 * 2 : 0;
+    auto kern = k_quant_fused<WPR, V, THR, FULL>;
+    // Resident CTAs per SM, cached per (kernel, device, shared memory in 1 KB steps).
+    static std::mutex mu;
+    static std::map<std::pair<int, size_t>, int> occ;
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto key = std::make_pair(dev.device, (smem + 1023) / 1024);
+        auto it = occ.find(key);
+        if (it != occ.end()) {
+            per_sm = it->second;
+        } else {
+            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, key.second * 1024);
+            if (e != cudaSuccess)
+                return e;
+            occ[key] = per_sm;
+        }
+    }
+    if (per_sm < 1)
+        return cudaErrorInvalidConfiguration;
+    const int64_t want = (rows + GROUPS - 1) / GROUPS;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)per_sm * dev.num_sms);
+    // Seed about 2 MB of rows (at least 64 rows, all rows when fewer): every
+    // seed_stride-th row group seeds its first row. A column that misses the
+    // seed is still handled exactly, by the finish step.
+    const int64_t groups = std::min<int64_t>(rows, (int64_t)grid * GROUPS);
+    const int64_t row_bytes = (int64_t)cols * 2;
+    const int64_t seed_rows = std::min<int64_t>(groups, std::max<int64_t>(64, (2ll << 20) / row_bytes));
+    const int seed_stride = (int)std::max<int64_t>(1, groups / std::max<int64_t>(1, seed_rows));
+    const __half t16 = threshold_fp16(t);
+    const uint4 *xp = reinterpret_cast<const uint4 *>(X);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative; // the barriers need every CTA resident
+    attr[0].val.cooperative = THR ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, xp, rows, cols, t, t16, codes, absmax, bitmap, col_idx, count, sync,
+                              status, seed_stride);
+}
+
+template <int WPR, int V>
+cudaError_t launch_fused_v(const void *X, int64_t rows, int cols, float t, int8_t *codes, float *absmax,
+                           uint32_t *bitmap, int32_t *col_idx, int32_t *count, uint32_t *sync, uint32_t *status,
+                           const DeviceInfo &dev, cudaStream_t stream)
+{
+    const bool thr = t > 0.f;
+    const bool full = ((cols >> 3) % (32 * WPR * V)) == 0;
+    if (thr)
+        return full ? launch_fused<WPR, V, true, true>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count,
+                                                       sync, status, dev, stream)
+                    : launch_fused<WPR, V, true, false>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count,
+                                                        sync, status, dev, stream);
+    return full ? launch_fused<WPR, V, false, true>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync,
+                                                    status, dev, stream)
+                : launch_fused<WPR, V, false, false>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync,
+                                                     status, dev, stream);
 }
 
 } // namespace
 
 cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols64, float t, int8_t *codes,
-                            float *absmax, uint32_t *bitmap, int32_t *argmax, int32_t *col_idx,
-                            int32_t *count, const DeviceInfo &dev, cudaStream_t stream)
+                            float *absmax, uint32_t *bitmap, int32_t *col_idx, int32_t *count, uint32_t *sync,
+                            uint32_t *status, const DeviceInfo &dev, cudaStream_t stream)
 {
     if (rows <= 0 || cols64 <= 0)
         return cudaSuccess;
     const int cols = (int)cols64;
     const int nvec = cols / 8;
-    const size_t smem = (size_t)((cols + 31) / 32) * 4;
-    cudaError_t e;
-    // K1: pick the narrowest block whose registers hold a whole row.
-    int nt = 0, v = 0;
-    for (int cand_nt : {128, 256, 512, 1024}) {
-        int need = (nvec + cand_nt - 1) / cand_nt;
-        if (need <= 8) {
-            nt = cand_nt;
-            v = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
-            break;
-        }
+    // Many rows: one warp per row, with 16 vectors per thread (a row of up to
+    // 4096 columns stays in registers) unless 8 divides the row into whole
+    // chunks where 16 does not. Few rows: the whole CTA on each row.
+    if (rows >= (int64_t)dev.num_sms * 8) {
+        if (nvec > 512 && nvec % 512 != 0 && nvec % 256 == 0)
+            return launch_fused_v<1, 8>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
+                                        stream);
+        return launch_fused_v<1, 16>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
+                                     stream);
     }
-    switch (nt) {
-    case 128: e = launch_k1_nt<128>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream, v); break;
-    case 256: e = launch_k1_nt<256>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream, v); break;
-    case 512: e = launch_k1_nt<512>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream, v); break;
-    case 1024: e = launch_k1_nt<1024>(X, rows, cols, t, codes, absmax, argmax, bitmap, dev, stream, v); break;
-    default: {
-        const int64_t grid = std::min<int64_t>(rows, (int64_t)dev.num_sms * 2);
-        k_quantize_rows_loop<1024><<<(unsigned)grid, 1024, smem, stream>>>(
-            reinterpret_cast<const uint4 *>(X), rows, cols, t, codes, absmax, argmax, bitmap);
-        e = cudaGetLastError();
-    }
-    }
-    if (e != cudaSuccess || !(t > 0.f))
-        return e;
-    // K2: fix-up, zeroing, compaction.
-    const int64_t grid2 = std::min<int64_t>(rows, (int64_t)dev.num_sms * 8);
-    k_fixup_rows<256><<<(unsigned)grid2, 256, smem, stream>>>(reinterpret_cast<const uint4 *>(X), rows, cols,
-                                                             codes, absmax, argmax, bitmap, col_idx, count);
-    return cudaGetLastError();
+    return launch_fused_v<8, 8>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev, stream);
 }
 
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

@@ -156,6 +156,25 @@ def test_quantize_edge_rows(lib, dev, oracle_mod):
     assert np.array_equal(codes.cpu().numpy(), c_ref)
 
 
+def test_quantize_late_outlier_column(lib, dev, oracle_mod):
+    """8192 rows: the outlier-column seed reads only the first rows, so a
+    column that crosses the threshold only in row 8100 is found late, while
+    rows 7000.. already took their maximum (5.5) in it. The result must still
+    be the definition's (every row re-quantized against the final set)."""
+    X = np.random.default_rng(8).standard_normal((8192, 2048)).astype(np.float32)
+    X[:, 100] *= 0.1
+    X[7000:, 100] = 5.5
+    X[8100, 100] = 50.0
+    X16 = X.astype(np.float16)
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
+    mask = oracle_mod.outlier_mask(X16, 6.0)
+    assert mask[100]
+    c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 2048), mask)
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
 def test_quantize_row_of_outliers(lib, dev, oracle_mod):
     """One row >= t everywhere makes every column an outlier: all codes 0,
     every absmax 0 (the int8 part is empty)."""
