@@ -425,9 +425,34 @@ def run_profile_case(args):
     import int8_mixed_precision_rowwise_b200 as L
 
     dev = torch.device("cuda", 0)
+    if args.profile_case == "quantizer":
+        lin = synthetic.QUANT_4096.linears[0]
+        X, _, _ = synthetic.torch_device_problem(
+            synthetic.Linear("q", lin.M, 1, lin.K, lin.n_outlier_cols, lin.outlier_scale), 0, dev)
+        L.quantize_rowwise(X, 6.0)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("timed_steps")
+        for _ in range(args.steps):
+            L.quantize_rowwise(X, 6.0)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        return
+    if args.profile_case.startswith("decode_M"):
+        lin = synthetic.decode_bloom(int(args.profile_case[len("decode_M"):])).linears[0]
+        X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
+        layer = L.Int8MixedLinear.from_fp16(W, keep_fp16_weights=False)
+        del W
+        layer(X)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("timed_steps")
+        for _ in range(args.steps):
+            layer(X)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        return
     lins = [l for l in WORKLOAD.linears if args.profile_case in ("all", l.name)]
     if not lins:
-        raise SystemExit(f"unknown linear {args.profile_case!r}")
+        raise SystemExit(f"unknown case {args.profile_case!r}")
     layers, xs, ys = [], [], []
     for li, lin in enumerate(lins):
         X, W, _ = synthetic.torch_device_problem(lin, seed=100 + li, device=dev)
@@ -453,7 +478,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--profile-case", default=None,
-                    help="ncu driver: run only this BLOOM linear ('qkv', 'attn_out', 'fc1', 'fc2' or 'all')")
+                    help="ncu driver: run only this BLOOM linear ('qkv', 'attn_out', 'fc1', 'fc2' or 'all'), "
+                         "the 4096 x 4096 'quantizer', or 'decode_M1' / 'decode_M8' / 'decode_M32'")
     args = ap.parse_args()
     if args.profile_case:
         run_profile_case(args)
