@@ -264,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {
             "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "k_gemm_i8<256,4,false,false> (fused dequant + outlier epilogue)",
+            "kernel": "k_gemm_i8_pair (CTA-pair tcgen05 int8 GEMM, fused dequant + outlier epilogue)",
             "peak_source": f"2 x bf16 sustained of {peak_kind} ({peaks.get('bf16_tflops_sustained')} TF/s), "
                            f"nominal int8:bf16 = 4.5:2.25; burst equivalent {round(int8_peak_burst, 1)}, "
                            "spec 4500",
