@@ -408,9 +408,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int stage = 0;
             uint32_t phase = 0, armed = 0, armed_phase = 0;
             constexpr uint32_t TX = (uint32_t)(L::A_BYTES + L::B_BYTES);
+            // The weight operand (A when SWAP, else B) does not depend on the
+            // kernel before this one: start streaming the first tile's weight
+            // tiles before waiting for the quantizer's output. (Hinting more of
+            // them into L2 here was measured to slow the quantizer down by
+            // queueing its few reads behind the flood.)
+            const CUtensorMap *wmap = SWAP ? &tmA : &tmB;
+            int pre = 0;
+            if ((int)blockIdx.x < num_tiles) {
+                const int mb = (int)blockIdx.x % p.num_m_blk, nb = (int)blockIdx.x / p.num_m_blk;
+                const int wrow = SWAP ? mb * BM : nb * BN;
+                const uint32_t woff = SWAP ? L::A_OFF : L::B_OFF;
+                const uint32_t wbytes = SWAP ? L::A_BYTES : L::B_BYTES;
+                pre = min(STAGES, p.num_kb);
+                for (int s = 0; s < pre; ++s) {
+                    mbar_arrive_expect_tx(full_bar(s), TX);
+                    tma_load_2d(sbase + woff + s * wbytes, wmap, full_bar(s), s * BK, wrow);
+                    armed |= 1u << s; // phase 0
+                }
+            }
+            griddep_wait();
             for (int tile = blockIdx.x; tile < num_tiles && !*s_abort; tile += gridDim.x) {
                 const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (tile == (int)blockIdx.x && kb < pre) {
+                        // Weight tile already in flight on this stage's barrier.
+                        if (SWAP)
+                            tma_load_2d(sbase + L::B_OFF + stage * L::B_BYTES, &tmB, full_bar(stage), kb * BK,
+                                        nb * BN);
+                        else
+                            tma_load_2d(sbase + L::A_OFF + stage * L::A_BYTES, &tmA, full_bar(stage), kb * BK,
+                                        mb * BM);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
                         report(p, s_abort, LLMINT8_DEV_TIMEOUT_PRODUCER);
                         break;
@@ -484,6 +518,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         __syncwarp();
     } else {
+        griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
         run_epilogue<BN, SWAP, RAW, false>(p, warp, lane, s_side, s_scale, tfull_bar(0), tempty_bar(0), s_abort,
                                            tmem_base, blockIdx.x, gridDim.x, num_tiles, BM, 0);
     }
@@ -583,11 +618,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             constexpr uint32_t TX = 2u * (uint32_t)(L::A_BYTES + L::B_BYTES);
+            // The weight half (B) of the first stages goes out before the wait
+            // for the quantizer's codes (A).
+            int pre = 0;
+            if (pair_id < num_tiles) {
+                const int nb = pair_id / p.num_m_blk;
+                const int b_row = nb * BN + (int)rank * (BN / 2);
+                pre = min(STAGES, p.num_kb);
+                for (int s = 0; s < pre; ++s) {
+                    if (leader)
+                        mbar_arrive_expect_tx(full_bar(s), TX);
+                    tma_load_2d_pair(sbase + L::B_OFF + s * L::B_BYTES, &tmB, full_bar(s), s * BK, b_row);
+                }
+            }
+            griddep_wait();
             for (int tile = pair_id; tile < num_tiles && !*s_abort; tile += num_pairs) {
                 const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
                 const int a_row = mb * 2 * BM + (int)rank * BM;
                 const int b_row = nb * BN + (int)rank * (BN / 2);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (tile == pair_id && kb < pre) {
+                        tma_load_2d_pair(sbase + L::A_OFF + stage * L::A_BYTES, &tmA, full_bar(stage), kb * BK,
+                                         a_row);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
                         report(p, s_abort, LLMINT8_DEV_TIMEOUT_PRODUCER);
                         break;
@@ -653,6 +711,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         }
         __syncwarp();
     } else {
+        griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
         run_epilogue<BN, false, RAW, true>(p, warp, lane, s_side, s_scale, tfull_bar(0), tempty_bar(0), s_abort,
                                            tmem_base, pair_id, num_pairs, num_tiles, 2 * BM, (int)rank * BM);
     }
@@ -666,6 +725,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 // ---------------------------------------------------------------- host side
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream finishes (it waits with griddep_wait()
+// before reading that kernel's output).
+template <typename Kern>
+cudaError_t launch_dependent(Kern kern, int grid, int smem, cudaStream_t stream, const CUtensorMap &ta,
+                             const CUtensorMap &tb, const KParams &p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
@@ -687,7 +766,9 @@ EncodeTiledFn encode_fn()
 }
 
 // Row-major int8 [rows x K] as a 2-D tensor map with a 128-byte x box_rows box.
-bool make_map_i8(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows)
+// Encoded maps are cached (keyed on device, address, shape and box) so that
+// repeated calls on the same buffers skip the driver call between launches.
+bool encode_map_i8(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
@@ -700,6 +781,39 @@ bool make_map_i8(CUtensorMap *map, const void *base, int64_t rows, int64_t K, in
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_map_i8(CUtensorMap *map, int device, const void *base, int64_t rows, int64_t K, int box_rows)
+{
+    struct Entry {
+        int device;
+        const void *base;
+        int64_t rows, K;
+        int box_rows;
+        CUtensorMap map;
+    };
+    constexpr int kCache = 32;
+    static std::mutex mu;
+    static Entry cache[kCache];
+    static int used = 0, next = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i) {
+            const Entry &e = cache[i];
+            if (e.device == device && e.base == base && e.rows == rows && e.K == K && e.box_rows == box_rows) {
+                *map = e.map;
+                return true;
+            }
+        }
+    }
+    if (!encode_map_i8(map, base, rows, K, box_rows))
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry &e = cache[next];
+    e = Entry{device, base, rows, K, box_rows, *map};
+    next = (next + 1) % kCache;
+    used = used < kCache ? used + 1 : kCache;
+    return true;
 }
 
 template <int BN, int STAGES, bool SWAP, bool RAW>
@@ -721,7 +835,7 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     const int64_t rows_a = SWAP ? a.N : a.M;
     const int64_t rows_b = SWAP ? a.M : a.N;
     CUtensorMap ta, tb;
-    if (!make_map_i8(&ta, Aop, rows_a, a.K, BM) || !make_map_i8(&tb, Bop, rows_b, a.K, BN))
+    if (!make_map_i8(&ta, dev.device, Aop, rows_a, a.K, BM) || !make_map_i8(&tb, dev.device, Bop, rows_b, a.K, BN))
         return cudaErrorInvalidValue;
     KParams p;
     p.rows_a = (int)rows_a;
@@ -743,8 +857,7 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     p.status = a.status;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int grid = std::min(tiles, dev.num_sms);
-    kern<<<grid, NTHREADS, L::ALLOC, stream>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_dependent(kern, grid, L::ALLOC, stream, ta, tb, p);
 }
 
 template <int BN, int STAGES, bool RAW>
@@ -761,7 +874,7 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
         configured.fetch_or(bit);
     }
     CUtensorMap ta, tb;
-    if (!make_map_i8(&ta, a.A, a.M, a.K, BM) || !make_map_i8(&tb, a.B, a.N, a.K, BN / 2))
+    if (!make_map_i8(&ta, dev.device, a.A, a.M, a.K, BM) || !make_map_i8(&tb, dev.device, a.B, a.N, a.K, BN / 2))
         return cudaErrorInvalidValue;
     KParams p;
     p.rows_a = (int)a.M;
@@ -783,8 +896,7 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.status = a.status;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int pairs = std::min(tiles, dev.num_sms / 2);
-    kern<<<2 * pairs, NTHREADS, L::ALLOC, stream>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, p);
 }
 
 // Tile width for CTA-pair tiles (256 x BN): the one that minimises tile
@@ -857,7 +969,7 @@ cudaError_t launch_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t s
         return cudaSuccess;
     const bool raw = a.epi == Epilogue::RawInt32;
     if (a.M <= 16)
-        return raw ? run<16, 10, true, true>(a, dev, stream) : run<16, 10, true, false>(a, dev, stream);
+        return raw ? run<16, 12, true, true>(a, dev, stream) : run<16, 12, true, false>(a, dev, stream);
     if (a.M <= 32)
         return raw ? run<32, 10, true, true>(a, dev, stream) : run<32, 10, true, false>(a, dev, stream);
     return raw ? run_prefill<true>(a, dev, stream) : run_prefill<false>(a, dev, stream);

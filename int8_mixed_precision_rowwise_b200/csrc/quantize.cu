@@ -221,14 +221,14 @@ __device__ __forceinline__ bool publish_vector(const uint4 &v, int vi, __half t1
     return ((bits & ~old) & ~gold) != 0u;
 }
 
-// Seed: find the outlier columns of one row (no codes).
+// Seed: find the outlier columns of one row (no codes). The last chunk read
+// stays in `v` (the whole row when it fits in one chunk).
 template <int GS, int V, bool FULL>
 __device__ __forceinline__ void row_seed(const uint4 *__restrict__ xr, int nvec, int gl, __half t16,
-                                         uint32_t *s_known, uint32_t *bitmap)
+                                         uint32_t *s_known, uint32_t *bitmap, uint4 (&v)[V])
 {
     const __half2 t2 = __half2half2(t16);
     for (int c0 = 0; c0 < nvec; c0 += GS * V) {
-        uint4 v[V];
 #pragma unroll
         for (int u = 0; u < V; ++u) {
             const int vi = c0 + u * GS + gl;
@@ -252,14 +252,16 @@ __device__ __forceinline__ void row_seed(const uint4 *__restrict__ xr, int nvec,
 template <int GS, int V, bool THR, bool FULL>
 __device__ __forceinline__ float row_max(const uint4 *__restrict__ xr, int nvec, int gl, bool resident,
                                          const uint32_t *s_known, const uint32_t (&kb4)[(V + 3) / 4],
-                                         uint4 (&v)[V])
+                                         uint4 (&v)[V], bool preloaded)
 {
     __half2 m2 = __float2half2_rn(0.f);
     for (int c0 = 0; c0 < nvec; c0 += GS * V) {
+        if (!(preloaded && resident)) {
 #pragma unroll
-        for (int u = 0; u < V; ++u) {
-            const int vi = c0 + u * GS + gl;
-            v[u] = (FULL || vi < nvec) ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+            for (int u = 0; u < V; ++u) {
+                const int vi = c0 + u * GS + gl;
+                v[u] = (FULL || vi < nvec) ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+            }
         }
 #pragma unroll
         for (int u = 0; u < V; ++u) {
@@ -336,12 +338,13 @@ template <int WPR, int V, bool THR, bool FULL>
 __device__ __forceinline__ void quantize_row(const uint4 *__restrict__ xr, int64_t r, int cols, float t, __half t16,
                                              bool resident, uint32_t *s_known, uint32_t *bitmap, uint32_t *new_flag,
                                              const uint32_t (&kb4)[(V + 3) / 4], uint4 (&v)[V],
-                                             int8_t *__restrict__ codes, float *__restrict__ absmax, float *red)
+                                             int8_t *__restrict__ codes, float *__restrict__ absmax, float *red,
+                                             bool preloaded = false)
 {
     constexpr int GS = 32 * WPR;
     const int gl = ((threadIdx.x >> 5) % WPR) * 32 + (threadIdx.x & 31);
     const int nvec = cols >> 3;
-    float amax = row_max<GS, V, THR, FULL>(xr, nvec, gl, resident, s_known, kb4, v);
+    float amax = row_max<GS, V, THR, FULL>(xr, nvec, gl, resident, s_known, kb4, v, preloaded);
     amax = group_max_f32<WPR>(amax, red);
     if (THR && amax >= t) {
         for (int vi = gl; vi < nvec; vi += GS)
@@ -394,6 +397,9 @@ constexpr int kMaxLate = 64; // late outlier columns handled by the cheap path
 //              re-quantizes those of its rows that were marked, or whose
 //              maximum equals |x| at a column of L, and zeroes the L-column
 //              codes of its other rows (every row, when |L| > kMaxLate).
+// When every row is seeded (rows <= groups), the set after the first barrier
+// is final: CTA 0 compacts it there, each row stays in registers from the
+// seed to its codes, and the second barrier is skipped.
 // Without a threshold only the quantize step runs. FULL: the row length is a
 // multiple of the chunk (no bounds checks). A row of at most 32 * WPR * V
 // 16-byte vectors stays in registers between its maximum and its codes; a
@@ -404,7 +410,7 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
                                                      float *__restrict__ absmax, uint32_t *__restrict__ bitmap,
                                                      int32_t *__restrict__ col_idx, int32_t *__restrict__ count,
                                                      uint32_t *__restrict__ sync, uint32_t *__restrict__ status,
-                                                     int seed_stride)
+                                                     int seed_stride, bool all_seeded)
 {
     constexpr int GROUPS = 8 / WPR; // row groups per CTA
     constexpr int GS = 32 * WPR;    // threads per group
@@ -422,13 +428,14 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     uint32_t *s_seed = s_dyn + nwords; // [nwords]
     uint32_t kb4[(V + 3) / 4];
     uint4 v[V];
+    griddep_release(); // the GEMM may start its weight stream now; it waits for this kernel's output
 
     if constexpr (THR) {
         for (int w = tid; w < nwords; w += 256)
             s_known[w] = 0u;
         __syncthreads();
         if (gid < rows && gid % seed_stride == 0)
-            row_seed<GS, V, FULL>(X + gid * (int64_t)nvec, nvec, gl, t16, s_known, bitmap);
+            row_seed<GS, V, FULL>(X + gid * (int64_t)nvec, nvec, gl, t16, s_known, bitmap, v);
         __syncthreads();
         if (tid == 0) {
             s_flag = grid_barrier(sync, gridDim.x) ? 1 : 0;
@@ -441,15 +448,20 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
         for (int w = tid; w < nwords; w += 256)
             s_known[w] = s_seed[w] = __ldcg(bitmap + w);
         __syncthreads();
+        // Every row seeded (one row per group): the set is final already.
+        if (all_seeded && blockIdx.x == 0)
+            compact_block<256>(s_known, nwords, col_idx, count);
     }
 
     load_known_bytes<GS, V>(s_known, nvec, gl, THR && resident, kb4);
     int it = 0;
     for (int64_t r = gid; r < rows; r += G, ++it)
         quantize_row<WPR, V, THR, FULL>(X + r * (int64_t)nvec, r, cols, t, t16, resident, s_known, bitmap,
-                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1]);
+                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1], THR && all_seeded);
     if constexpr (!THR)
         return;
+    if (all_seeded)
+        return; // no row can hold a column the seed did not see
 
     // ---- finish
     __syncthreads();
@@ -571,8 +583,9 @@ cudaError_t launch_fused(const void *X, int64_t rows, int cols, float t, int8_t 
     attr[0].val.cooperative = THR ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const bool all_seeded = seed_stride == 1 && rows <= groups;
     return cudaLaunchKernelEx(&cfg, kern, xp, rows, cols, t, t16, codes, absmax, bitmap, col_idx, count, sync,
-                              status, seed_stride);
+                              status, seed_stride, all_seeded);
 }
 
 template <int WPR, int V>
