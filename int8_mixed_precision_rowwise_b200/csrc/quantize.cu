@@ -36,33 +36,6 @@ namespace llmint8 {
 
 namespace {
 
-__device__ __forceinline__ void unpack8(const uint4 &v, float (&x)[8])
-{
-    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 f = __half22float2(h[i]);
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-    }
-}
-
-// Quantize one value with the row multiplier s = 127 / absmax (fp32, RN).
-__device__ __forceinline__ int quant1(float x, float s)
-{
-    return __float2int_rn(__fmul_rn(x, s));
-}
-
-__device__ __forceinline__ uint2 pack8(const int (&q)[8])
-{
-    uint2 r;
-    r.x = (uint32_t)(q[0] & 0xFF) | ((uint32_t)(q[1] & 0xFF) << 8) | ((uint32_t)(q[2] & 0xFF) << 16) |
-          ((uint32_t)(q[3] & 0xFF) << 24);
-    r.y = (uint32_t)(q[4] & 0xFF) | ((uint32_t)(q[5] & 0xFF) << 8) | ((uint32_t)(q[6] & 0xFF) << 16) |
-          ((uint32_t)(q[7] & 0xFF) << 24);
-    return r;
-}
-
 // Ascending list of the set bits of s_bm[0..nwords) written by one CTA.
 template <int NT>
 __device__ void compact_block(const uint32_t *s_bm, int nwords, int32_t *col_idx, int32_t *count)
