@@ -133,8 +133,10 @@ typedef struct llmint8_debug {
     float *row_absmax;  /* [M]     SX: X's row absmax over non-outlier columns */
     int32_t *col_idx;   /* [K]     ascending outlier columns (first |O| valid) */
     int32_t *count;     /* [1]     |O| */
-    int32_t *acc;       /* [M x N] int32 accumulators of the int8 part (runs the
-                           int8 GEMM a second time with a raw int32 epilogue) */
+    int32_t *acc;       /* [M x N] int32 accumulators of the int8 part (M <= 32:
+                           written by the fused decode kernel itself; larger M:
+                           the int8 GEMM runs a second time with a raw int32
+                           epilogue) */
     void *gemm_begin;   /* cudaEvent_t or NULL: recorded on `stream` right before */
     void *gemm_end;     /* and right after the fused GEMM launch (kernel timing)  */
 } llmint8_debug;
@@ -155,10 +157,16 @@ typedef struct llmint8_debug {
  *              absmax, from llmint8_quantize_rowwise(W, t <= 0).
  *   W_f16      (device, may be NULL) fp16 [N x K]
  *   Y_f16      (device) fp16 [M x N] out
- *   workspace  (device) >= llmint8_workspace_size(M, N, K) bytes, zeroed once.
+ *   workspace  (device) >= llmint8_workspace_size(M, N, K) bytes, zeroed once
+ *              (llmint8_workspace_init). After a call that left an error bit in
+ *              the status word, zero it again before the next call.
  *   dbg        (host struct of device pointers, may be NULL)
- * M <= 32 runs the decode kernel (W streamed once, tokens on the MMA N side);
- * larger M runs the persistent prefill GEMM.
+ * M <= 32 (and N <= 122880) runs one fused, cooperatively launched decode
+ * kernel: the outlier columns and codes of X are computed across all SMs
+ * while the weight codes already stream in, W is split evenly over the SMs
+ * and split tiles are summed exactly in int32. Larger M runs the quantizer
+ * and then the persistent prefill GEMM (CTA pairs from M = 256).
+ * Calls that share a workspace must be ordered (one stream, or events).
  */
 LLMINT8_API llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
                                     const float *SCB, const void *W_f16, int64_t N,

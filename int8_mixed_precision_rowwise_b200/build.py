@@ -16,8 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libllmint8.so")
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "noalloc.cu"]
-HEADERS = ["internal.h", "ptx.cuh"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "decode.cu", "noalloc.cu"]
+HEADERS = ["internal.h", "ptx.cuh", "common.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -65,6 +65,49 @@ llmint8_status check_k(int64_t K)
 
 llmint8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA; }
 
+// The intermediate results a caller asked for in `dbg`: the raw int32
+// accumulators (with `run_acc`, one more int8 GEMM of the same codes; the
+// decode kernel writes them itself) and copies of the codes, row absmax and
+// outlier columns from the workspace.
+llmint8_status copy_debug(const llmint8_debug *dbg, const Workspace &ws, int64_t M, int64_t N, int64_t K,
+                          const int8_t *CB, const float *SCB, const void *X_f16, const void *W_f16, bool run_acc,
+                          const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (!dbg)
+        return LLMINT8_OK;
+    if (dbg->acc && run_acc) {
+        GemmArgs r{};
+        r.A = ws.cx;
+        r.B = CB;
+        r.M = M;
+        r.N = N;
+        r.K = K;
+        r.sx = ws.sx;
+        r.sb = SCB;
+        r.X16 = X_f16;
+        r.W16 = W_f16;
+        r.col_idx = ws.col_idx;
+        r.count = ws.count;
+        r.status = ws.status;
+        r.epi = Epilogue::RawInt32;
+        r.Y = dbg->acc;
+        if (launch_gemm(r, dev, stream) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    }
+    if (dbg->codes &&
+        cudaMemcpyAsync(dbg->codes, ws.cx, (size_t)M * K, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if (dbg->row_absmax &&
+        cudaMemcpyAsync(dbg->row_absmax, ws.sx, (size_t)M * 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if (dbg->col_idx &&
+        cudaMemcpyAsync(dbg->col_idx, ws.col_idx, (size_t)K * 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if (dbg->count && cudaMemcpyAsync(dbg->count, ws.count, 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return LLMINT8_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -89,15 +132,14 @@ size_t llmint8_quantize_workspace_size(int64_t rows, int64_t cols)
 {
     if (rows < 0 || cols < 0)
         return 0;
-    return carve(nullptr, rows, cols, false, nullptr);
+    return carve(nullptr, rows, cols, false, false, nullptr);
 }
 
 size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K)
 {
-    (void)N;
     if (M < 0 || N < 0 || K < 0)
         return 0;
-    return carve(nullptr, M, K, true, nullptr);
+    return carve(nullptr, M, K, true, decode_shape(M, N), nullptr);
 }
 
 llmint8_status llmint8_workspace_init(void *workspace, size_t ws_bytes, llmint8_stream_t stream)
@@ -139,7 +181,7 @@ llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t
         (outlier_bitmap && !aligned16(outlier_bitmap)))
         return LLMINT8_ERR_ALIGNMENT;
     Workspace ws;
-    const size_t need = carve(static_cast<char *>(workspace), rows, cols, false, &ws);
+    const size_t need = carve(static_cast<char *>(workspace), rows, cols, false, false, &ws);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
     if (rows == 0)
@@ -209,7 +251,7 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
             return LLMINT8_ERR_ALIGNMENT;
     }
     Workspace ws;
-    const size_t need = carve(static_cast<char *>(workspace), M, K, true, &ws);
+    const size_t need = carve(static_cast<char *>(workspace), M, K, true, decode_shape(M, N), &ws);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
     if (M == 0 || N == 0)
@@ -219,6 +261,20 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
     if (e != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     const float t = effective_threshold(threshold);
+
+    if (decode_fused_fits(M, N, K, dev)) {
+        // A few tokens: the whole layer in one kernel.
+        DecodeArgs d{X_f16, M, N, K, t, CB, SCB, W_f16, Y_f16, dbg ? dbg->acc : nullptr, ws};
+        if (dbg && dbg->gemm_begin &&
+            cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if ((e = launch_decode(d, dev, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if (dbg && dbg->gemm_end &&
+            cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        return copy_debug(dbg, ws, M, N, K, CB, SCB, X_f16, W_f16, false, dev, stream);
+    }
 
     // Clear |O| and the bitmap (one memset: they sit next to each other).
     char *clear_from = reinterpret_cast<char *>(ws.count);
@@ -252,28 +308,7 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
     if (dbg && dbg->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
 
-    if (dbg) {
-        if (dbg->acc) {
-            GemmArgs r = g;
-            r.epi = Epilogue::RawInt32;
-            r.Y = dbg->acc;
-            if ((e = launch_gemm(r, dev, stream)) != cudaSuccess)
-                return LLMINT8_ERR_CUDA;
-        }
-        if (dbg->codes && (e = cudaMemcpyAsync(dbg->codes, ws.cx, (size_t)M * K, cudaMemcpyDeviceToDevice,
-                                               stream)) != cudaSuccess)
-            return LLMINT8_ERR_CUDA;
-        if (dbg->row_absmax && (e = cudaMemcpyAsync(dbg->row_absmax, ws.sx, (size_t)M * 4,
-                                                    cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
-            return LLMINT8_ERR_CUDA;
-        if (dbg->col_idx && (e = cudaMemcpyAsync(dbg->col_idx, ws.col_idx, (size_t)K * 4,
-                                                 cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
-            return LLMINT8_ERR_CUDA;
-        if (dbg->count && (e = cudaMemcpyAsync(dbg->count, ws.count, 4, cudaMemcpyDeviceToDevice, stream)) !=
-                              cudaSuccess)
-            return LLMINT8_ERR_CUDA;
-    }
-    return LLMINT8_OK;
+    return copy_debug(dbg, ws, M, N, K, CB, SCB, X_f16, W_f16, true, dev, stream);
 }
 
 llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B, int64_t N, int64_t K,
@@ -291,7 +326,7 @@ llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B,
     if (!aligned16(A) || !aligned16(B) || !aligned16(acc) || !aligned16(workspace))
         return LLMINT8_ERR_ALIGNMENT;
     Workspace ws;
-    const size_t need = carve(static_cast<char *>(workspace), M, K, true, &ws);
+    const size_t need = carve(static_cast<char *>(workspace), M, K, true, false, &ws);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
     if (M == 0 || N == 0)

@@ -771,6 +771,8 @@ cudaError_t launch_dependent(Kern kern, int grid, int smem, cudaStream_t stream,
     return cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
 }
 
+} // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -840,6 +842,8 @@ bool make_map_i8(CUtensorMap *map, int device, const void *base, int64_t rows, i
     used = used < kCache ? used + 1 : kCache;
     return true;
 }
+
+namespace {
 
 template <int BN, int STAGES, bool SWAP, bool RAW>
 cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)

@@ -3,18 +3,33 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace llmint8 {
 
+// Decode (M <= kDecodeMaxM tokens) runs as one fused kernel with at most
+// kDecodeMaxCtas CTAs.
+constexpr int kDecodeMaxM = 32;
+constexpr int kDecodeMaxCtas = 160;
+constexpr int kHeaderBytes = 256;
+
 // Workspace layout (byte offsets; every region 256-byte aligned):
 //   [0]      uint32 status word (bits LLMINT8_DEV_*)
 //   [4]      int32  |O| (outlier column count)
-//   [8]      uint32 grid-barrier counter and generation, late-outlier flag
+//   [8]      uint32 grid-barrier counter and generation, late-outlier flag,
+//            decode outlier-list flag
 //   [256]    uint32 outlier bitmap [ceil(K/32)]
 //   ...      int32  ascending outlier columns [K]
 //   ...      fp32   SX [M]
 //   ...      int8   CX [M x K]
+//   decode only (1 <= M <= kDecodeMaxM), every entry rewritten by each call:
+//   ...      uint8  outlier mask per 8 columns [K/8]
+//   ...      fp32   partial row maxima [kDecodeMaxM x kDecodeMaxCtas]
+//   ...      int32  partial accumulators per CTA [kDecodeMaxCtas x kDecodeMaxM x 128]
+//   ...      uint32 partial-ready flags per CTA [kDecodeMaxCtas] (tagged with the
+//            call's grid-barrier generation, so never cleared)
 struct Workspace {
     uint32_t *status;
     int32_t *count;
@@ -23,12 +38,21 @@ struct Workspace {
     int32_t *col_idx;
     float *sx;
     int8_t *cx;
+    uint8_t *hitmask;
+    float *prow;
+    int32_t *slots;
+    uint32_t *pflags;
     size_t bytes;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, Workspace *ws)
+// Shapes that llmint8_matmul_mixed runs with the fused decode kernel.
+inline bool decode_shape(int64_t M, int64_t N) { return M >= 1 && M <= kDecodeMaxM && N >= 1; }
+
+// Lay out (base != null) or size a workspace; `decode` adds the regions of
+// the fused decode kernel.
+inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool decode, Workspace *ws)
 {
     size_t off = 0;
     auto take = [&](size_t n) {
@@ -36,12 +60,16 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, Workspace
         off = align256(off + n);
         return base ? base + o : nullptr;
     };
-    char *hdr = take(256);
+    char *hdr = take(kHeaderBytes);
     size_t nwords = (size_t)((K + 31) / 32);
     char *bm = take(nwords * 4);
     char *ci = take((size_t)K * 4);
     char *sx = with_codes ? take((size_t)M * 4) : nullptr;
     char *cx = with_codes ? take((size_t)M * (size_t)K) : nullptr;
+    char *hm = decode ? take((size_t)(K / 8)) : nullptr;
+    char *pr = decode ? take((size_t)kDecodeMaxCtas * kDecodeMaxM * 4) : nullptr;
+    char *sl = decode ? take((size_t)kDecodeMaxCtas * kDecodeMaxM * 128 * 4) : nullptr;
+    char *pf = decode ? take((size_t)kDecodeMaxCtas * 4) : nullptr;
     if (ws) {
         ws->status = reinterpret_cast<uint32_t *>(hdr);
         ws->count = hdr ? reinterpret_cast<int32_t *>(hdr + 4) : nullptr;
@@ -50,6 +78,10 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, Workspace
         ws->col_idx = reinterpret_cast<int32_t *>(ci);
         ws->sx = reinterpret_cast<float *>(sx);
         ws->cx = reinterpret_cast<int8_t *>(cx);
+        ws->hitmask = reinterpret_cast<uint8_t *>(hm);
+        ws->prow = reinterpret_cast<float *>(pr);
+        ws->slots = reinterpret_cast<int32_t *>(sl);
+        ws->pflags = reinterpret_cast<uint32_t *>(pf);
         ws->bytes = off;
     }
     return off;
@@ -72,6 +104,10 @@ cudaError_t device_info(DeviceInfo *out);
 cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes,
                             float *absmax, uint32_t *bitmap, int32_t *col_idx, int32_t *count, uint32_t *sync,
                             uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
+
+// The smallest fp16 value >= t, so that for fp16 x, |x| >= t exactly when
+// |x| >= threshold_fp16(t) (+inf when no finite value qualifies, 0 for t <= 0).
+__half threshold_fp16(float t);
 
 // Bitmap -> ascending column list and count (one CTA).
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,
@@ -96,5 +132,27 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, const DeviceInfo &dev, cudaStream_t stream);
+
+// The whole LLM.int8() linear for at most kDecodeMaxM tokens in one kernel:
+// outlier detection, quantization of X, the int8 product streamed over all
+// SMs, dequantization and the outlier product.
+struct DecodeArgs {
+    const void *X;       // [M x K] fp16
+    int64_t M, N, K;
+    float t;             // threshold (0: no decomposition)
+    const int8_t *CB;    // [N x K]
+    const float *sb;     // [N]
+    const void *W16;     // [N x K] fp16 or null
+    void *Y;             // [M x N] fp16
+    int32_t *acc_out;    // [M x N] int32 products (before dequantization), or null
+    Workspace ws;
+};
+
+bool decode_fused_fits(int64_t M, int64_t N, int64_t K, const DeviceInfo &dev);
+cudaError_t launch_decode(const DecodeArgs &args, const DeviceInfo &dev, cudaStream_t stream);
+
+// Row-major int8 [rows x K] as a 2-D TMA tensor map (128-byte x box_rows box,
+// 128-byte swizzle, zero fill out of bounds); cached per device and buffer.
+bool make_map_i8(CUtensorMap *map, int device, const void *base, int64_t rows, int64_t K, int box_rows);
 
 } // namespace llmint8

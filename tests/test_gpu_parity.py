@@ -274,6 +274,65 @@ def test_all_columns_outliers(lib, dev, oracle_mod, M):
     assert g["O"].size == 96 and not g["CX"].any()
 
 
+# ------------------------------------------------------------------ fused decode kernel (M <= 32)
+
+@pytest.mark.parametrize("M,N,K", [(1, 100, 16), (3, 129, 80), (16, 300, 1040), (21, 1000, 4096),
+                                   (2, 4000, 1024), (32, 256, 57344)])
+def test_decode_split_tiles(lib, dev, oracle_mod, M, N, K):
+    """The decode kernel spreads (weight tile, 128-byte K slice) units over
+    the SMs: from a single unit (one CTA) up to tiles split over dozens of
+    CTAs. The split products are summed exactly: acc is compared bit for bit."""
+    lin = Linear("d", M, N, K, 3, 60.0)
+    X16, _ = make_activations(lin, seed=M * 7 + K)
+    W16 = make_weight(lin, seed=N)
+    check_full(lib, dev, oracle_mod, X16, W16, 6.0, give_w16=False)
+
+
+def test_decode_threshold_off(lib, dev, oracle_mod):
+    X16 = make_random((5, 2048), seed=21)
+    W16 = make_random((700, 2048), seed=22, scale=0.02)
+    g, _ = check_full(lib, dev, oracle_mod, X16, W16, 0.0)
+    assert g["O"].size == 0
+
+
+def test_decode_after_prefill_same_workspace(lib, dev, oracle_mod):
+    """A prefill call leaves its bitmap and codes in the shared workspace; the
+    decode call after it must not depend on them (and the reverse)."""
+    lin = Linear("t", 300, 640, 1024, 6, 60.0)
+    X16, _ = make_activations(lin, seed=5)
+    W16 = make_weight(lin, seed=5)
+    check_full(lib, dev, oracle_mod, X16, W16, 6.0)
+    check_full(lib, dev, oracle_mod, X16[:9], W16, 6.0)
+    check_full(lib, dev, oracle_mod, X16[100:], W16, 6.0)
+
+
+def test_decode_repeat_and_graph(lib, dev):
+    """Tile counters return to zero after each call: repeated calls and CUDA
+    graph replays give identical results."""
+    lin = Linear("t", 4, 3000, 2048, 4, 60.0)
+    X16, _ = make_activations(lin, seed=8)
+    W16 = make_weight(lin, seed=8)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    layer = lib.Int8MixedLinear.from_fp16(W)
+    ref = layer(X).clone()
+    for _ in range(3):
+        assert torch.equal(layer(X), ref)
+    Y = torch.empty_like(ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer(X, Y=Y)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer(X, Y=Y)
+    for _ in range(2):
+        Y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(Y, ref)
+
+
 def test_repeat_calls_identical(lib, dev):
     lin = Linear("t", 300, 600, 1024, 4, 60.0)
     X16, _ = make_activations(lin, seed=1)
