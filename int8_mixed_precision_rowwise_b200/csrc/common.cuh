@@ -10,35 +10,37 @@
 namespace llmint8 {
 
 // One bounded grid-wide barrier (all CTAs are co-resident: the kernel is
-// launched cooperatively). sync[0] counts arrivals, sync[1] is the
-// generation; *gen (if given) receives the generation this barrier opened.
-// The arrival is a release and the wait an acquire at GPU scope, so writes
-// that the calling thread made, or that its CTA made before a CTA barrier,
-// are visible to every CTA after the barrier.
+// launched cooperatively). sync[0] counts arrivals and sync[1] is the
+// generation, read and written together as one 64-bit word (8-byte
+// aligned), so that an arrival learns both in a single atomic round trip.
+// The last arrival moves to the next generation and clears the count in
+// one add; the others wait for the generation to change. *gen (if given)
+// receives the generation this barrier opened. The arrival is a release
+// and the wait an acquire at GPU scope, so writes that the calling thread
+// made, or that its CTA made before a CTA barrier, are visible to every
+// CTA after the barrier.
 __device__ __forceinline__ bool grid_barrier(uint32_t *sync, uint32_t nblocks, uint32_t *gen = nullptr)
 {
-    uint32_t g, prev;
-    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(g) : "l"(sync + 1) : "memory");
-    asm volatile("atom.acq_rel.gpu.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(sync) : "memory");
-    if (prev + 1 == nblocks) {
-        asm volatile("st.relaxed.gpu.u32 [%0], 0;" ::"l"(sync) : "memory");
-        asm volatile("red.release.gpu.add.u32 [%0], 1;" ::"l"(sync + 1) : "memory");
-        if (gen)
-            *gen = g + 1;
+    unsigned long long *word = reinterpret_cast<unsigned long long *>(sync);
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.add.u64 %0, [%1], 1;" : "=l"(old) : "l"(word) : "memory");
+    const uint32_t g = (uint32_t)(old >> 32);
+    if (gen)
+        *gen = g + 1;
+    if ((uint32_t)old + 1u == nblocks) {
+        const unsigned long long next = (1ull << 32) - nblocks; // generation + 1, count back to 0
+        asm volatile("red.release.gpu.add.u64 [%0], %1;" ::"l"(word), "l"(next) : "memory");
         return true;
     }
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-        uint32_t cur;
-        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(sync + 1) : "memory");
-        if (cur != g) {
-            if (gen)
-                *gen = g + 1;
+        unsigned long long cur;
+        asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(cur) : "l"(word) : "memory");
+        if ((uint32_t)(cur >> 32) != g)
             return true;
-        }
         if (global_timer_ns() - t0 > kWaitLimitNs)
             return false;
-        __nanosleep(64);
+        __nanosleep(32);
     }
 }
 

@@ -279,9 +279,10 @@ constexpr int kMaxLate = 64; // late outlier columns handled by the cheap path
 
 // Fused quantizer, one row per group of WPR warps (WPR = 1: a warp per row;
 // WPR = 8: the whole CTA per row). With a threshold (THR):
-//   seed     - every `seed_stride`-th group reads its first row only to find
-//              outlier columns (|x| >= t); these rows come back from L2 in
-//              the next step;
+//   seed     - the first row of every group (rows that fit in registers,
+//              kept there for the quantize step), or of every
+//              `seed_stride`-th group (longer rows, read again from L2 in the
+//              next step), is searched for outlier columns (|x| >= t);
 //   barrier  - then each CTA loads the outlier set found so far (the "seed
 //              set", also kept aside);
 //   quantize - every row: maximum over the columns not known as outliers,
@@ -293,9 +294,10 @@ constexpr int kMaxLate = 64; // late outlier columns handled by the cheap path
 //              re-quantizes those of its rows that were marked, or whose
 //              maximum equals |x| at a column of L, and zeroes the L-column
 //              codes of its other rows (every row, when |L| > kMaxLate).
-// When every row is seeded (rows <= groups), the set after the first barrier
-// is final: CTA 0 compacts it there, each row stays in registers from the
-// seed to its codes, and the second barrier is skipped.
+// Rows that fit in registers: every group seeds its first row, which stays
+// in registers from the seed to its codes. When every row is seeded (rows
+// <= groups), the set after the first barrier is final: CTA 0 compacts it
+// there and the second barrier is skipped.
 // Without a threshold only the quantize step runs. FULL: the row length is a
 // multiple of the chunk (no bounds checks). A row of at most 32 * WPR * V
 // 16-byte vectors stays in registers between its maximum and its codes; a
@@ -330,7 +332,11 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
         for (int w = tid; w < nwords; w += 256)
             s_known[w] = 0u;
         __syncthreads();
-        if (gid < rows && gid % seed_stride == 0)
+        // A row that fits in registers is read here once and for all: every
+        // group seeds its first row and keeps it for the quantize step, so
+        // those reads overlap the barrier. Longer rows: every
+        // seed_stride-th group reads its first row only to seed.
+        if (gid < rows && (resident || gid % seed_stride == 0))
             row_seed<GS, V, FULL>(X + gid * (int64_t)nvec, nvec, gl, t16, s_known, bitmap, v);
         __syncthreads();
         if (tid == 0) {
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     int it = 0;
     for (int64_t r = gid; r < rows; r += G, ++it)
         quantize_row<WPR, V, THR, FULL>(X + r * (int64_t)nvec, r, cols, t, t16, resident, s_known, bitmap,
-                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1], THR && all_seeded);
+                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1], THR && resident && it == 0);
     if constexpr (!THR)
         return;
     if (all_seeded)
@@ -465,7 +471,8 @@ cudaError_t launch_fused(const void *X, int64_t rows, int cols, float t, int8_t 
     attr[0].val.cooperative = THR ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const bool all_seeded = seed_stride == 1 && rows <= groups;
+    const bool resident = (cols >> 3) <= 32 * WPR * V;
+    const bool all_seeded = rows <= groups && (resident || seed_stride == 1);
     return cudaLaunchKernelEx(&cfg, kern, xp, rows, cols, t, t16, codes, absmax, bitmap, col_idx, count, sync,
                               status, seed_stride, all_seeded);
 }
