@@ -23,10 +23,10 @@
 //     is read with an evict-first L2 policy (it is used once), so X, the
 //     partial buffers and this kernel's own instructions stay in L2;
 //   - a tile whose K range is split between CTAs is summed exactly in int32:
-//     its first CTA (for which it is the last segment, reached at the end of
-//     the stream) finishes it; the others, for which it is the first segment,
-//     park their partial sums at the start of their stream and raise a flag
-//     tagged with this call's barrier generation.
+//     every CTA processes its segments from the last to the first, so the
+//     head of a tile (the end of one CTA's range) is done early and parked
+//     with a flag tagged with this call's barrier generation; the CTA that
+//     holds the tile's tail finishes it at the end of its stream.
 // The MMA is the swapped form: the weight tile is the M = 128 side, tokens
 // the N = 16 or 32 side. The code that runs once per launch (scales, codes,
 // epilogue) is written as short loops over the M real tokens rather than
@@ -139,6 +139,24 @@ __device__ __forceinline__ int owner_of(int64_t u, int64_t units, int64_t G)
     return (int)c;
 }
 
+// The i-th unit a CTA with units [u0, u1) processes: its segments (maximal
+// runs of units in one tile) from the last to the first, the units of each
+// in ascending order. The last segment of a range is a tile's head, whose
+// tile is finished by another CTA; processing it first lets that partial be
+// parked early.
+__device__ __forceinline__ int64_t unit_order(int64_t u0, int64_t u1, int KB, int64_t i)
+{
+    int64_t se = u1;
+    for (;;) {
+        const int64_t ts = ((se - 1) / KB) * KB;
+        const int64_t su = ts > u0 ? ts : u0;
+        if (i < se - su)
+            return su + i;
+        i -= se - su;
+        se = su;
+    }
+}
+
 // Ascending list of the outlier columns from the per-8-column masks
 // hitmask[0 .. nvec), by the NHELP helper threads of one CTA.
 __device__ void compact_masks(const uint8_t *hitmask, int nvec, int32_t *col_idx, int32_t *count, int et,
@@ -222,9 +240,7 @@ __device__ __forceinline__ void store_codes(const DParams &p, uint4 x, int r, in
 //   weight stream may start);
 //   2. absmax per row = maximum of the partial maxima (s_amax) and the
 //      multiplier 127 / absmax; the slice's codes go to p.cx; CTA 0 writes SX;
-//   grid barrier (codes complete before any CTA's TMA reads them);
-//   3. CTA 0 compacts the outlier columns and then sets the list flag
-//      sync[3] to the generation of the first barrier (*gen).
+//   grid barrier (codes complete before any CTA's TMA reads them).
 // Each thread keeps its first PC vectors of X in registers; the rest is read
 // again (from L2). Returns false if a grid barrier gave up.
 template <bool THR>
@@ -331,22 +347,24 @@ __device__ bool row_scales(const DParams &p, int et, uint32_t xloaded_bar, uint3
     if (et == 0)
         *s_flag = grid_barrier(p.sync, (uint32_t)G) ? 1 : 0;
     named_barrier_sync(1, NHELP);
-    if (!*s_flag)
-        return false;
-    if (c == 0) {
-        // Off the critical path: the epilogues need the list much later and
-        // wait for the flag.
-        if constexpr (THR) {
-            compact_masks(p.hitmask, nvec, p.col_idx, p.count, et, s_pfx);
-        } else if (et == 0) {
-            *p.count = 0;
-        }
-        if (et == NHELP - 1 || (!THR && et == 0)) {
-            __threadfence();
-            asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p.sync + 3), "r"(*gen) : "memory");
-        }
+    return *s_flag != 0;
+}
+
+// The ascending outlier columns and their count, by CTA 0's helper warps
+// after the codes are out (off the critical path: the epilogues need the
+// list much later); then the list flag sync[3] is set to `gen`.
+template <bool THR>
+__device__ void publish_outlier_list(const DParams &p, int et, int *s_pfx, uint32_t gen)
+{
+    if constexpr (THR) {
+        compact_masks(p.hitmask, p.K >> 3, p.col_idx, p.count, et, s_pfx);
+    } else if (et == 0) {
+        *p.count = 0;
     }
-    return true;
+    if (et == NHELP - 1 || (!THR && et == 0)) {
+        __threadfence();
+        asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p.sync + 3), "r"(gen) : "memory");
+    }
 }
 
 // Outlier weights W~[j, cols[k]] of this thread's weight row j for k < nk
@@ -417,14 +435,16 @@ __device__ void finalize_row(const DParams &p, int j, int r, int32_t *acc, const
 
 // Epilogue of one segment [su, se) of tile t = su / num_kb, held in TMEM
 // accumulator buffer seg & 1. A whole tile is finished here. A split tile is
-// finished by its first CTA c_lo, for which it is the last segment: it reads
-// the partials that the tile's other CTAs parked (after their ready flags,
-// normally long set) before its own accumulator is complete, then adds it;
-// for each other CTA the tile is its first segment, which it parks in its
-// slot before raising its flag to `gen`. All NHELP helper threads call it
-// together; returns false on a timeout (nothing written).
+// finished by the CTA holding its last unit, c_hi: the tile is that CTA's
+// first segment, which it processes last, and before its own accumulator is
+// complete it reads the partials that the tile's other CTAs parked (after
+// their ready flags). For each other CTA the tile is its last segment, which
+// it processes first and parks in its slot before raising its flag to
+// `gen`. All NHELP helper threads call it together; returns false on a
+// timeout (nothing written).
 template <int BN>
-__device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, int64_t u0, int64_t su, int64_t se,
+__device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, int64_t u0, int64_t u1, int64_t su,
+                                 int64_t se,
                                  int seg, uint32_t tmem_base, uint32_t tfull_b, uint32_t tempty_b, uint32_t &tph_b,
                                  const float *s_amax, float *s_side, int *s_cols, int32_t *s_acc, float *s_wv,
                                  int cnt, uint32_t gen, volatile int *s_abort, volatile int *s_last)
@@ -436,7 +456,9 @@ __device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, i
     const bool whole = su == tile_u0 && se == tile_u0 + KB;
     const int c_lo = whole ? (int)cta : owner_of(tile_u0, p.units, G);
     const int c_hi = whole ? (int)cta : owner_of(tile_u0 + KB - 1, p.units, G);
-    const bool finisher = cta == c_lo;
+    const bool finisher = cta == c_hi;
+    (void)u0;
+    (void)u1;
     const int q = warp & 3;      // TMEM lane quarter this warp may read
     const int r = q * 32 + lane; // weight row within the tile
     const int j = t * TM + r;
@@ -453,7 +475,7 @@ __device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, i
             if (et == 0) {
                 bool all = true;
                 const uint64_t t0 = global_timer_ns();
-                for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
+                for (int cc = c_lo; cc < c_hi; ++cc) {
                     uint32_t f;
                     for (;;) {
                         asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(f) : "l"(p.pflags + cc) : "memory");
@@ -471,18 +493,16 @@ __device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, i
                     report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
                 return false;
             }
-            for (int cc = c_lo + 1; cc <= c_hi; ++cc) {
+            for (int cc = c_lo; cc < c_hi; ++cc) {
                 const int32_t *src = p.slots + ((int64_t)cc * kDecodeMaxM) * TM + r;
-                for (int c0 = 0; c0 < M; c0 += 8) {
-                    int32_t v[8];
+                int32_t v[BN];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        v[u] = c0 + u < M ? __ldcg(src + (c0 + u) * TM) : 0;
+                for (int c = 0; c < BN; ++c) // every load in flight at once
+                    v[c] = c < M ? __ldcg(src + c * TM) : 0;
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (c0 + u < M)
-                            acc[c0 + u] += v[u];
-                }
+                for (int c = 0; c < BN; ++c)
+                    if (c < M)
+                        acc[c] += v[c];
             }
         }
     }
@@ -506,7 +526,8 @@ __device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, i
     if (lane == 0)
         mbar_arrive(tempty_b); // the accumulator is in registers now
     if (!finisher) {
-        // This tile is this CTA's first segment: park it for the finisher.
+        // This tile is this CTA's last segment (processed first): park it
+        // for the finisher.
         int32_t *dst = p.slots + (cta * kDecodeMaxM) * TM + r;
 #pragma unroll
         for (int c = 0; c < BN; ++c)
@@ -607,7 +628,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(xloaded_bar, 0u))
                 report(p, s_abort, LLMINT8_DEV_TIMEOUT_PRODUCER);
             for (int s = 0; s < pre; ++s) {
-                const int64_t u = u0 + s;
+                const int64_t u = unit_order(u0, u1, KB, s);
                 const int t = (int)(u / KB), kb = (int)(u - (int64_t)t * KB);
                 const int ns = slices(kb);
                 mbar_arrive_expect_tx(full_bar(s), tx(ns));
@@ -618,7 +639,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             // The next units into L2, so that HBM stays busy until the codes
             // are ready and the ring turns over.
-            for (int64_t u = u0 + pre; u < u1 && u < u0 + pre + kL2Ahead; ++u) {
+            for (int64_t i = pre; i < n && i < pre + kL2Ahead; ++i) {
+                const int64_t u = unit_order(u0, u1, KB, i);
                 const int t = (int)(u / KB), kb = (int)(u - (int64_t)t * KB);
                 for (int j = 0; j < slices(kb); ++j)
                     tma_prefetch_l2_2d(&tmW, (kb * KS + j) * SK, t * TM);
@@ -627,7 +649,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 report(p, s_abort, LLMINT8_DEV_TIMEOUT_PRODUCER);
             asm volatile("fence.proxy.async.global;" ::: "memory"); // codes written by other CTAs
             for (int64_t i = 0; i < n; ++i) {
-                const int64_t u = u0 + i;
+                const int64_t u = unit_order(u0, u1, KB, i);
                 const int t = (int)(u / KB), kb = (int)(u - (int64_t)t * KB);
                 const int ns = slices(kb);
                 if (i < pre) {
@@ -676,10 +698,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t tph[2] = {0u, 0u};
             constexpr uint32_t IDESC = idesc_i8(TM, BN);
             int seg = 0;
-            int64_t u = u0;
-            while (u < u1 && !*s_abort) {
-                const int t = (int)(u / KB);
-                const int64_t seg_end = min(u1, (int64_t)(t + 1) * KB);
+            int64_t seg_end = u1; // segments from the last to the first
+            while (seg_end > u0 && !*s_abort) {
+                const int64_t u = max(u0, ((seg_end - 1) / KB) * KB);
                 const int b = seg & 1;
                 if (!mbar_wait(tempty_bar(b), tph[b] ^ 1u)) {
                     report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
@@ -714,7 +735,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!ok)
                     break;
                 mma_commit(tfull_bar(b)); // this segment's product is complete
-                u = seg_end;
+                seg_end = u;
                 ++seg;
             }
             // Wait for every MMA this thread issued before TMEM is released.
@@ -734,6 +755,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 report(p, s_abort, LLMINT8_DEV_TIMEOUT_QUANT);
             mbar_arrive(ready_bar); // the producer may add the codes to its stages
         }
+        if (ok && blockIdx.x == 0)
+            publish_outlier_list<THR>(p, et, s_pfx, gen);
         if (ok) {
             // The outlier list of CTA 0 (ready long before the first segment ends).
             if (et == 0) {
@@ -767,14 +790,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             named_barrier_sync(1, NHELP);
             uint32_t tph[2] = {0u, 0u};
             int seg = 0;
-            for (int64_t u = u0; u < u1; ++seg) {
-                const int64_t seg_end = min(u1, (u / KB + 1) * KB);
+            for (int64_t seg_end = u1; seg_end > u0; ++seg) { // segments from the last to the first
+                const int64_t su = max(u0, ((seg_end - 1) / KB) * KB);
                 const int b = seg & 1;
-                if (!epilogue_segment<BN>(p, et, warp, lane, u0, u, seg_end, seg, tmem_base, tfull_bar(b),
+                if (!epilogue_segment<BN>(p, et, warp, lane, u0, u1, su, seg_end, seg, tmem_base, tfull_bar(b),
                                           tempty_bar(b), tph[b], s_amax, s_side, s_cols, s_acc, s_wv, cnt, gen,
                                           s_abort, s_last))
                     break;
-                u = seg_end;
+                seg_end = su;
             }
         }
     }
