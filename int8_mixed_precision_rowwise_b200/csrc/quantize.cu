@@ -356,10 +356,41 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     }
 
     load_known_bytes<GS, V>(s_known, nvec, gl, THR && resident, kb4);
+    // With the whole CTA on a row that fits in registers (at most 16 vectors
+    // a thread), the next row is read into a second register set while this
+    // one is reduced and coded: two rows in flight per CTA.
+    constexpr bool PREFETCH = WPR > 1 && V <= 16;
+    auto load_row = [&](int64_t r, uint4(&dst)[V]) {
+        const uint4 *xr = X + r * (int64_t)nvec;
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int vi = u * GS + gl;
+            dst[u] = (FULL || vi < nvec) ? __ldg(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    uint4 vn[PREFETCH ? V : 1];
     int it = 0;
-    for (int64_t r = gid; r < rows; r += G, ++it)
+    for (int64_t r = gid; r < rows; r += G, ++it) {
+        bool pre = THR && resident && it == 0; // the seed step left the first row in v
+        if constexpr (PREFETCH) {
+            if (resident) {
+                if (it == 0 && !pre)
+                    load_row(r, v);
+                pre = true;
+                if (r + G < rows)
+                    load_row(r + G, vn);
+            }
+        }
         quantize_row<WPR, V, THR, FULL>(X + r * (int64_t)nvec, r, cols, t, t16, resident, s_known, bitmap,
-                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1], THR && resident && it == 0);
+                                        sync + 2, kb4, v, codes, absmax, s_red[it & 1], pre);
+        if constexpr (PREFETCH) {
+            if (resident) {
+#pragma unroll
+                for (int u = 0; u < V; ++u)
+                    v[u] = vn[u];
+            }
+        }
+    }
     if constexpr (!THR)
         return;
     if (all_seeded)
@@ -519,16 +550,19 @@ cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols64, float t
         return cudaSuccess;
     const int cols = (int)cols64;
     const int nvec = cols / 8;
-    // Many rows: one warp per row, with 16 vectors per thread (a row of up to
-    // 4096 columns stays in registers) unless 8 divides the row into whole
-    // chunks where 16 does not. Few rows: the whole CTA on each row.
-    if (rows >= (int64_t)dev.num_sms * 8) {
-        if (nvec > 512 && nvec % 512 != 0 && nvec % 256 == 0)
-            return launch_fused_v<1, 8>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
-                                        stream);
+    // Many rows of up to 4096 columns: one warp per row, the row in registers
+    // (16 vectors a thread). Otherwise the whole CTA on each row, with 8, 16
+    // or 32 vectors a thread, so that rows of up to 65536 columns stay in
+    // registers and are read from HBM once; longer rows are read twice.
+    if (rows >= (int64_t)dev.num_sms * 8 && nvec <= 32 * 16)
         return launch_fused_v<1, 16>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
                                      stream);
-    }
+    if (nvec <= 256 * 16 && nvec > 256 * 8)
+        return launch_fused_v<8, 16>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
+                                     stream);
+    if (nvec <= 256 * 32 && nvec > 256 * 16)
+        return launch_fused_v<8, 32>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
+                                     stream);
     return launch_fused_v<8, 8>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev, stream);
 }
 
