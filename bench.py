@@ -275,11 +275,47 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(world * step_ops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "h2d_bytes_per_step": int(sum(x.numel() * 2 for x in xs)),
                 "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in ys))},
-        "gpu_launches": 3 * gemm_launches,
+        "gpu_launches": 2 * gemm_launches,  # per linear: the fused quantizer and the GEMM
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
         "secondary": secondary,
     }
     return line
+
+
+def per_linear_times(L, dev, reps=10):
+    """For each BLOOM linear and the 2048 x 16384 x 4096 prefill linear: the
+    GEMM alone (events around its launch) and the whole llmint8_matmul_mixed
+    call (quantizer, GEMM), median of `reps` calls; int8 TOPS of each."""
+    import torch
+
+    res = {}
+    lins = list(WORKLOAD.linears) + list(synthetic.PREFILL_7B.linears)
+    for li, lin in enumerate(lins):
+        X, W, _ = synthetic.torch_device_problem(lin, seed=200 + li, device=dev)
+        layer = L.Int8MixedLinear.from_fp16(W, WORKLOAD.threshold, keep_fp16_weights=True)
+        Y = torch.empty((lin.M, lin.N), dtype=torch.float16, device=dev)
+        gb = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        cb = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        ce = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        for _ in range(2):
+            L.matmul_mixed(X, layer.CB, layer.SCB, layer.W_f16, layer.threshold, Y=Y)
+        torch.cuda.synchronize()
+        for k in range(reps):
+            cb[k].record()
+            L.matmul_mixed(X, layer.CB, layer.SCB, layer.W_f16, layer.threshold, Y=Y,
+                           debug={"gemm_begin": gb[k], "gemm_end": ge[k]})
+            ce[k].record()
+        torch.cuda.synchronize()
+        gemm_us = statistics.median(gb[k].elapsed_time(ge[k]) for k in range(reps)) * 1e3
+        call_us = statistics.median(cb[k].elapsed_time(ce[k]) for k in range(reps)) * 1e3
+        ops = ops_of(lin)
+        name = lin.name if lin in WORKLOAD.linears else f"prefill_{lin.M}x{lin.N}x{lin.K}"
+        res[name] = {"gemm_us": round(gemm_us, 1), "gemm_tops": round(ops / (gemm_us * 1e-6) / 1e12, 1),
+                     "call_us": round(call_us, 1), "call_tops": round(ops / (call_us * 1e-6) / 1e12, 1)}
+        del layer, X, W, Y
+    torch.cuda.empty_cache()
+    return res
 
 
 def graph_time_ms(fns, reps):
@@ -338,6 +374,7 @@ def measure_secondary(L, dev):
     out["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
                                   "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
     del bufs, fns
+    out["per_linear"] = per_linear_times(L, dev)
     for M in (1, 8, 32):
         lin = synthetic.decode_bloom(M).linears[0]
         X, W, _ = synthetic.torch_device_problem(lin, 0, dev)

@@ -161,7 +161,7 @@ typedef struct llmint8_debug {
  *              (llmint8_workspace_init). After a call that left an error bit in
  *              the status word, zero it again before the next call.
  *   dbg        (host struct of device pointers, may be NULL)
- * M <= 32 (and N <= 122880) runs one fused, cooperatively launched decode
+ * M <= 32 runs one fused, cooperatively launched decode
  * kernel: the outlier columns and codes of X are computed across all SMs
  * while the weight codes already stream in, W is split evenly over the SMs
  * and split tiles are summed exactly in int32. Larger M runs the quantizer
@@ -173,6 +173,35 @@ LLMINT8_API llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, in
                                     float threshold, void *Y_f16, void *workspace,
                                     size_t ws_bytes, const llmint8_debug *dbg,
                                     llmint8_stream_t stream);
+
+/* Activations the epilogue can apply after the bias. */
+typedef enum {
+    LLMINT8_ACT_NONE = 0,
+    /* BLOOM's GELU, tanh form (page "优化故事：Bloom 推理", section
+     * "唾手可得的优化"): g(y) = 0.5 y (1 + tanh(0.79788456 y (1 + 0.044715 y^2))). */
+    LLMINT8_ACT_GELU_TANH = 1
+} llmint8_activation;
+
+/*
+ * llmint8_matmul_mixed with the two steps that follow the linear in a
+ * transformer block fused into its epilogue. The output is
+ *   Y[i,j] = fp16( act( y[i,j] + bias[j] ) )
+ * where y[i,j] is the fp32 value llmint8_matmul_mixed rounds, bias is added
+ * in fp32 (nn.Linear's bias, which the Linear8bitLt replacing each nn.Linear
+ * keeps: page "Hugging Face 将 LLM.int8() 8-bit 量化集成进 transformers 与
+ * accelerate", section "accelerate 就是你需要的一切"), and
+ * act is evaluated in fp32 (tanhf). Rounding to fp16 happens once, at the end.
+ *   bias_f16   (device, may be NULL) fp16 [N]
+ *   activation LLMINT8_ACT_NONE or LLMINT8_ACT_GELU_TANH; anything else
+ *              returns LLMINT8_ERR_INVALID_ARG.
+ * Every other argument, and the behaviour on errors, as for
+ * llmint8_matmul_mixed (which is this call with bias NULL and no activation).
+ */
+LLMINT8_API llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
+                                       const float *SCB, const void *W_f16, int64_t N,
+                                       float threshold, const void *bias_f16, int activation,
+                                       void *Y_f16, void *workspace, size_t ws_bytes,
+                                       const llmint8_debug *dbg, llmint8_stream_t stream);
 
 /*
  * Plain int8 GEMM with int32 output: acc[i,j] = sum_k A[i,k] * B[j,k]

@@ -46,6 +46,8 @@ _SIGNATURES = {
     "llmint8_find_outlier_cols": (_ST, [_P, _I64, _P, _P, _P, _P]),
     "llmint8_matmul_mixed": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, ctypes.c_float, _P, _P, ctypes.c_size_t,
                                    ctypes.POINTER(_Debug), _P]),
+    "llmint8_matmul_mixed_ex": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, ctypes.c_float, _P, ctypes.c_int, _P, _P,
+                                      ctypes.c_size_t, ctypes.POINTER(_Debug), _P]),
     "llmint8_gemm_s8s8s32": (_ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
     "llmint8_quantize_rowwise_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
 }
@@ -217,10 +219,15 @@ def find_outlier_cols(outlier_bitmap, cols: int, col_idx=None, d_count=None, syn
     return col_idx, d_count, (int(h.value) if sync_count else None)
 
 
+ACTIVATIONS = {None: 0, "none": 0, "gelu_tanh": 1}
+
+
 def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y=None, workspace=None,
-                 debug: dict | None = None):
+                 debug: dict | None = None, bias=None, activation=None):
     """Y fp16 [M x N] = LLM.int8()(X fp16 [M x K], W given as CB int8 [N x K] + SCB fp32 [N]).
 
+    ``bias`` (fp16 [N]) and ``activation`` (None or "gelu_tanh") are applied
+    in the epilogue before the fp16 rounding (llmint8_matmul_mixed_ex).
     ``debug`` may map any of codes/row_absmax/col_idx/count/acc to CUDA tensors
     the call fills (parity checks), and gemm_begin/gemm_end to recorded
     torch.cuda.Event objects the library re-records around the GEMM launch."""
@@ -230,6 +237,10 @@ def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y
     _need_cuda(SCB, "SCB", torch.float32)
     if W_f16 is not None:
         _need_cuda(W_f16, "W_f16", torch.float16)
+    if bias is not None:
+        _need_cuda(bias, "bias", torch.float16)
+    if activation not in ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(k for k in ACTIVATIONS if k)} or None")
     M, K = X.shape
     N = CB.shape[0]
     dev = X.device
@@ -240,9 +251,15 @@ def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y
     if debug:
         dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")),
                      *(_event(debug.get(k)) for k in ("gemm_begin", "gemm_end")))
-    _check(load()["_matmul_mixed"](X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N, float(threshold),
-                         Y.data_ptr(), ws.data_ptr(), ws.numel(), ctypes.byref(dbg) if dbg else None,
-                         _stream_ptr(dev)), "llmint8_matmul_mixed")
+    if bias is None and not ACTIVATIONS[activation]:
+        _check(load()["_matmul_mixed"](X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N,
+                                       float(threshold), Y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                       ctypes.byref(dbg) if dbg else None, _stream_ptr(dev)), "llmint8_matmul_mixed")
+    else:
+        _check(load()["_matmul_mixed_ex"](X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), _ptr(W_f16), N,
+                                          float(threshold), _ptr(bias), ACTIVATIONS[activation], Y.data_ptr(),
+                                          ws.data_ptr(), ws.numel(), ctypes.byref(dbg) if dbg else None,
+                                          _stream_ptr(dev)), "llmint8_matmul_mixed_ex")
     return Y
 
 
@@ -262,17 +279,21 @@ def gemm_s8s8s32(A, B, acc=None, workspace=None):
 
 
 class Int8MixedLinear:
-    """An LLM.int8() linear layer without bias: holds CB/SCB (and optionally the
-    fp16 weight for the outlier columns) and applies matmul_mixed."""
+    """An LLM.int8() linear layer: holds CB/SCB (and optionally the fp16 weight
+    for the outlier columns), an optional fp16 bias and an optional activation
+    fused after it, and applies matmul_mixed."""
 
-    def __init__(self, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD):
+    def __init__(self, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, bias=None, activation=None):
         self.CB, self.SCB, self.W_f16, self.threshold = CB, SCB, W_f16, threshold
+        self.bias, self.activation = bias, activation
 
     @classmethod
-    def from_fp16(cls, W, threshold: float = DEFAULT_THRESHOLD, keep_fp16_weights: bool = True):
+    def from_fp16(cls, W, threshold: float = DEFAULT_THRESHOLD, keep_fp16_weights: bool = True, bias=None,
+                  activation=None):
         """Quantize W fp16 [N x K] per output row (offline weight preparation)."""
         CB, SCB, _ = quantize_rowwise(W, 0.0)
-        return cls(CB, SCB, W if keep_fp16_weights else None, threshold)
+        return cls(CB, SCB, W if keep_fp16_weights else None, threshold, bias, activation)
 
     def __call__(self, X, Y=None):
-        return matmul_mixed(X, self.CB, self.SCB, self.W_f16, self.threshold, Y=Y)
+        return matmul_mixed(X, self.CB, self.SCB, self.W_f16, self.threshold, Y=Y, bias=self.bias,
+                            activation=self.activation)

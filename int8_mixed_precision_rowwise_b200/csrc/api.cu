@@ -232,6 +232,15 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
                                     void *Y_f16, void *workspace, size_t ws_bytes, const llmint8_debug *dbg,
                                     llmint8_stream_t stream)
 {
+    return llmint8_matmul_mixed_ex(X_f16, M, K, CB, SCB, W_f16, N, threshold, nullptr, LLMINT8_ACT_NONE, Y_f16,
+                                   workspace, ws_bytes, dbg, stream);
+}
+
+llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
+                                       const float *SCB, const void *W_f16, int64_t N, float threshold,
+                                       const void *bias_f16, int activation, void *Y_f16, void *workspace,
+                                       size_t ws_bytes, const llmint8_debug *dbg, llmint8_stream_t stream)
+{
     if (M < 0 || N < 0)
         return LLMINT8_ERR_INVALID_ARG;
     llmint8_status st = check_k(K);
@@ -241,8 +250,10 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
         return LLMINT8_ERR_UNSUPPORTED_SHAPE;
     if (!X_f16 || !CB || !SCB || !Y_f16 || !workspace)
         return LLMINT8_ERR_INVALID_ARG;
+    if (activation != LLMINT8_ACT_NONE && activation != LLMINT8_ACT_GELU_TANH)
+        return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(X_f16) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y_f16) || !aligned16(workspace) ||
-        (W_f16 && !aligned16(W_f16)))
+        (W_f16 && !aligned16(W_f16)) || (bias_f16 && !aligned16(bias_f16)))
         return LLMINT8_ERR_ALIGNMENT;
     if (dbg) {
         if ((dbg->codes && !aligned16(dbg->codes)) || (dbg->row_absmax && !aligned16(dbg->row_absmax)) ||
@@ -264,7 +275,7 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
 
     if (decode_fused_fits(M, N, K, dev)) {
         // A few tokens: the whole layer in one kernel.
-        DecodeArgs d{X_f16, M, N, K, t, CB, SCB, W_f16, Y_f16, dbg ? dbg->acc : nullptr, ws};
+        DecodeArgs d{X_f16, M, N, K, t, CB, SCB, W_f16, bias_f16, activation, Y_f16, dbg ? dbg->acc : nullptr, ws};
         if (dbg && dbg->gemm_begin &&
             cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
@@ -297,6 +308,8 @@ llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, con
     g.W16 = W_f16;
     g.col_idx = ws.col_idx;
     g.count = ws.count;
+    g.bias = bias_f16;
+    g.act = activation;
     g.status = ws.status;
     g.epi = Epilogue::MixedFp16;
     g.Y = Y_f16;

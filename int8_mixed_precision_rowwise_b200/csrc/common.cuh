@@ -105,4 +105,16 @@ __device__ __forceinline__ uint32_t hit_mask8(const uint4 &v, __half t16)
     return hit;
 }
 
+// The last two steps of every epilogue: y + bias (fp32), then the
+// activation (LLMINT8_ACT_GELU_TANH: BLOOM's GELU in tanh form, page
+// "优化故事：Bloom 推理", section "唾手可得的优化"), before the single fp16
+// rounding.
+__device__ __forceinline__ float bias_act(float y, float bias, int act)
+{
+    y += bias;
+    if (act == 1)
+        y = 0.5f * y * (1.0f + tanhf(0.79788456f * y * (1.0f + 0.044715f * y * y)));
+    return y;
+}
+
 } // namespace llmint8

@@ -69,6 +69,8 @@ struct DParams {
     const int8_t *CB;
     const float *sb;
     const __half *W16;
+    const __half *bias;      // fp16 [N] or null
+    int act;                 // LLMINT8_ACT_*
     __half *Y;
     int32_t *acc_out;        // [M x N] int32 products, or null
     uint8_t *hitmask;        // [K/8] outlier mask per 8 columns
@@ -396,6 +398,7 @@ __device__ void finalize_row(const DParams &p, int j, int r, int32_t *acc, const
         for (int c = 0; c < M; ++c)
             p.acc_out[(int64_t)c * p.N + j] = acc[c];
     const float sbj = j < p.N ? p.sb[j] : 0.f;
+    const float bj = (p.bias && j < p.N) ? __half2float(p.bias[j]) : 0.f;
     if (cnt <= OC) {
         // s_side holds X at the outlier columns for all tokens (staged once per
         // CTA), s_wv this row's outlier weights (loaded before the accumulator).
@@ -404,7 +407,7 @@ __device__ void finalize_row(const DParams &p, int j, int r, int32_t *acc, const
             for (int k = 0; k < cnt; ++k)
                 y = fmaf(s_wv[k * TM + r], s_side[k * BN + c], y);
             if (j < p.N)
-                p.Y[(int64_t)c * p.N + j] = __float2half_rn(y);
+                p.Y[(int64_t)c * p.N + j] = __float2half_rn(bias_act(y, bj, p.act));
         }
         return;
     }
@@ -430,7 +433,7 @@ __device__ void finalize_row(const DParams &p, int j, int r, int32_t *acc, const
     }
     if (j < p.N)
         for (int c = 0; c < M; ++c)
-            p.Y[(int64_t)c * p.N + j] = __float2half_rn(yr[c]);
+            p.Y[(int64_t)c * p.N + j] = __float2half_rn(bias_act(yr[c], bj, p.act));
 }
 
 // Epilogue of one segment [su, se) of tile t = su / num_kb, held in TMEM
@@ -846,6 +849,8 @@ cudaError_t run_decode(const DecodeArgs &a, const DeviceInfo &dev, cudaStream_t 
     p.CB = a.CB;
     p.sb = a.sb;
     p.W16 = reinterpret_cast<const __half *>(a.W16);
+    p.bias = reinterpret_cast<const __half *>(a.bias);
+    p.act = a.act;
     p.Y = reinterpret_cast<__half *>(a.Y);
     p.acc_out = a.acc_out;
     p.hitmask = a.ws.hitmask;

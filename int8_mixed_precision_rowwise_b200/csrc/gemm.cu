@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "llmint8.h"
+#include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -53,6 +54,8 @@ struct KParams {
     const __half *X16, *W16;
     const int8_t *CB;
     const int32_t *col_idx, *count;
+    const __half *bias;        // fp16 [N] or null
+    int act;                   // LLMINT8_ACT_*
     void *Y;
     uint32_t *status;
 };
@@ -260,6 +263,14 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                         }
                     }
                 }
+                if (p.bias || p.act) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int j = j0 + c;
+                        const float bv = (p.bias && j < p.N) ? __half2float(__ldg(p.bias + j)) : 0.f;
+                        y[c] = bias_act(y[c], bv, p.act);
+                    }
+                }
                 if (i < p.M) {
                     __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
                     if (j0 + 32 <= p.N && (p.N & 7) == 0) {
@@ -332,6 +343,12 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                                 y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
                         }
                     }
+                }
+                if (p.bias || p.act) {
+                    const float bv = (p.bias && j < p.N) ? __half2float(__ldg(p.bias + j)) : 0.f;
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        y[c] = bias_act(y[c], bv, p.act);
                 }
                 if (j < p.N) {
                     __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
@@ -882,6 +899,8 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     p.CB = a.B;
     p.col_idx = a.col_idx;
     p.count = a.count;
+    p.bias = reinterpret_cast<const __half *>(a.bias);
+    p.act = a.act;
     p.Y = a.Y;
     p.status = a.status;
     const int tiles = p.num_m_blk * p.num_n_blk;
@@ -921,6 +940,8 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.CB = a.B;
     p.col_idx = a.col_idx;
     p.count = a.count;
+    p.bias = reinterpret_cast<const __half *>(a.bias);
+    p.act = a.act;
     p.Y = a.Y;
     p.status = a.status;
     const int tiles = p.num_m_blk * p.num_n_blk;

@@ -127,6 +127,8 @@ struct GemmArgs {
     const void *W16;     // [N x K] fp16 or null (then CB * SB / 127)
     const int32_t *col_idx;
     const int32_t *count;
+    const void *bias;    // fp16 [N] or null, added after dequantization
+    int act;             // LLMINT8_ACT_* applied after the bias
     void *Y;             // fp16 [M x N]  (MixedFp16) or int32 [M x N] (RawInt32)
     uint32_t *status;
 };
@@ -143,6 +145,8 @@ struct DecodeArgs {
     const int8_t *CB;    // [N x K]
     const float *sb;     // [N]
     const void *W16;     // [N x K] fp16 or null
+    const void *bias;    // fp16 [N] or null
+    int act;             // LLMINT8_ACT_*
     void *Y;             // [M x N] fp16
     int32_t *acc_out;    // [M x N] int32 products (before dequantization), or null
     Workspace ws;

@@ -56,6 +56,8 @@ def _load():
         lib.oracle_outlier_weight.argtypes = [P, P, P, I64, I64, P, I64, P]
         lib.oracle_outlier_weight.restype = None
         lib.oracle_mixed_output.argtypes = [P, P, P, I64, I64, P, I64, P, I64, P, P]
+        lib.oracle_bias_act.restype = None
+        lib.oracle_bias_act.argtypes = [P, I64, I64, P, ctypes.c_int]
         lib.oracle_mixed_output.restype = None
         _lib = lib
     return _lib
@@ -151,19 +153,34 @@ def mixed_output(acc, SX, SB, X, cols, Wt) -> np.ndarray:
     return Y
 
 
+ACTIVATIONS = {None: 0, "none": 0, "gelu_tanh": 1}
+
+
+def bias_act(Y, bias=None, activation=None) -> np.ndarray:
+    """fp64 act(Y + bias): bias fp16/fp32 [N] or None, activation None or
+    "gelu_tanh" (BLOOM's tanh-form GELU)."""
+    Y = np.array(Y, dtype=np.float64, order="C")
+    M, N = Y.shape
+    b = None if bias is None else np.ascontiguousarray(np.asarray(bias).astype(np.float32))
+    _load().oracle_bias_act(_ptr(Y), M, N, None if b is None else _ptr(b), ACTIVATIONS[activation])
+    return Y
+
+
 def quantize_weight(W):
     """Offline weight preparation: row-wise absmax over the full row (no outliers)."""
     return quantize_rowwise(W, None)
 
 
-def matmul_mixed(X, threshold: float, W=None, CB=None, SB=None, use_fp16_weight_cols: bool = True):
+def matmul_mixed(X, threshold: float, W=None, CB=None, SB=None, use_fp16_weight_cols: bool = True, bias=None,
+                 activation=None):
     """The whole LLM.int8() linear on the host.
 
     X fp16 [M x K]. The weight is given as fp16 W [N x K] (then CB/SB are made
     from it), or as CB/SB only. ``use_fp16_weight_cols`` picks the source of
     W's outlier columns when W is given (False: recover them from CB*SB/127).
-    Returns a dict with O (ascending columns), CX, SX, CB, SB, acc, Wt and
-    Y (fp64)."""
+    ``bias`` (fp16 [N]) and ``activation`` follow the linear (bias_act).
+    Returns a dict with O (ascending columns), CX, SX, CB, SB, acc, Wt,
+    Y_lin (the linear alone) and Y (after bias and activation), both fp64."""
     x = _f32(X)
     if CB is None:
         CB, SB = quantize_weight(W)
@@ -172,5 +189,6 @@ def matmul_mixed(X, threshold: float, W=None, CB=None, SB=None, use_fp16_weight_
     CX, SX = quantize_rowwise(x, O)
     acc = int8_matmul(CX, CB)
     Wt = outlier_weight(O, N, K, W=W if (W is not None and use_fp16_weight_cols) else None, CB=CB, SB=SB)
-    Y = mixed_output(acc, SX, SB, x, O, Wt)
-    return dict(O=O, CX=CX, SX=SX, CB=CB, SB=SB, acc=acc, Wt=Wt, Y=Y)
+    Y_lin = mixed_output(acc, SX, SB, x, O, Wt)
+    Y = Y_lin if (bias is None and not ACTIVATIONS[activation]) else bias_act(Y_lin, bias, activation)
+    return dict(O=O, CX=CX, SX=SX, CB=CB, SB=SB, acc=acc, Wt=Wt, Y_lin=Y_lin, Y=Y)

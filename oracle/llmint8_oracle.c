@@ -161,3 +161,26 @@ void oracle_mixed_output(const int32_t *acc, const float *SX, const float *SB, i
         }
     }
 }
+
+/* The steps after the linear in a transformer block, on the fp64 output:
+ * Y[i,j] += bias[j] (nn.Linear's bias, kept by the Linear8bitLt that replaces
+ * it: page "Hugging Face 将 LLM.int8() 8-bit 量化集成进 transformers 与
+ * accelerate", section "accelerate 就是你需要的一切"), then, for act == 1,
+ * BLOOM's GELU in its tanh form (page "优化故事：Bloom 推理", section
+ * "唾手可得的优化"): g(y) = y/2 * (1 + tanh(0.79788456 * y * (1 + 0.044715 y^2))).
+ * bias may be NULL. */
+void oracle_bias_act(double *Y, int64_t M, int64_t N, const float *bias, int act)
+{
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t j = 0; j < N; ++j) {
+            double y = Y[i * N + j];
+            if (bias)
+                y += (double)bias[j];
+            if (act == 1) {
+                const double inner = 0.79788456 * y * (1.0 + 0.044715 * y * y);
+                y = 0.5 * y * (1.0 + tanh(inner));
+            }
+            Y[i * N + j] = y;
+        }
+    }
+}

@@ -85,6 +85,23 @@ def test_matmul_argument_errors(lib):
     assert _mm(lib, N=0) == lib.OK
 
 
+def test_matmul_ex_argument_errors(lib):
+    """The bias/activation entry point checks its two extra arguments before
+    anything is queued; the others are checked as for llmint8_matmul_mixed."""
+    f = lib._matmul_mixed_ex
+    M, N, K = 64, 64, 128
+    ws = lib.workspace_size(M, N, K)
+
+    def call(bias=None, act=0, X=A, wsb=ws):
+        return f(X, M, K, A, A, None, N, 6.0, bias, act, A, A, wsb, None, None)
+
+    assert call(act=2) == lib.ERR_INVALID_ARG
+    assert call(act=-1) == lib.ERR_INVALID_ARG
+    assert call(bias=A + 2) == lib.ERR_ALIGNMENT
+    assert call(X=None, act=1) == lib.ERR_INVALID_ARG
+    assert call(wsb=1024, bias=A, act=1) == lib.ERR_WORKSPACE
+
+
 def test_quantize_argument_errors(lib):
     q = lib._quantize_rowwise
     ws = lib.quantize_workspace_size(32, 64)

@@ -333,6 +333,33 @@ def test_decode_repeat_and_graph(lib, dev):
         assert torch.equal(Y, ref)
 
 
+# ------------------------------------------------------------------ bias and GELU fused in the epilogue
+
+@pytest.mark.parametrize("M,N,K,act", [(300, 520, 1040, "gelu_tanh"), (300, 520, 1040, None),
+                                       (100, 384, 512, "gelu_tanh"), (5, 640, 1024, "gelu_tanh"),
+                                       (32, 300, 2048, None), (7, 136, 96, "gelu_tanh")])
+def test_matmul_mixed_bias_activation(lib, dev, oracle_mod, M, N, K, act):
+    """llmint8_matmul_mixed_ex: Y = fp16(act(linear + bias)) on every path
+    (CTA-pair prefill, single-CTA prefill, fused decode; the last shape sends
+    every column to the fp16 side). The tolerance is the linear's, carried
+    through the activation: GELU's slope is at most 1.13, and the fp16
+    rounding now happens after it."""
+    lin = Linear("ba", M, N, K, 5, 60.0)
+    X16, _ = make_activations(lin, seed=M + 3 * N)
+    W16 = make_weight(lin, seed=K + 1)
+    bias = np.random.default_rng(N).standard_normal(N).astype(np.float16)
+    t = 1e-3 if K == 96 else 6.0
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    Y = lib.matmul_mixed(X, CB, SCB, W, t, bias=to_dev(bias, dev), activation=act)
+    r = oracle_mod.matmul_mixed(X16, t, W=W16, bias=bias, activation=act)
+    y = Y.cpu().numpy().astype(np.float64)
+    pre = r["Y_lin"] + bias.astype(np.float64)[None, :]
+    tol = 1.13 * (1e-2 + 2e-3 * np.abs(pre)) + 5e-4 * np.abs(r["Y"])
+    bad = np.abs(y - r["Y"]) > tol
+    assert not bad.any(), f"{bad.sum()} outside tolerance, worst {np.abs(y - r['Y']).max()}"
+
+
 def test_repeat_calls_identical(lib, dev):
     lin = Linear("t", 300, 600, 1024, 4, 60.0)
     X16, _ = make_activations(lin, seed=1)

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from conftest import read_golden
-from synthetic import make_random
+from synthetic import Linear, make_activations, make_random, make_weight
 
 pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
 
@@ -293,3 +293,41 @@ def test_brute_force_tiny_workload(oracle_mod):
     assert r["O"].tolist() == [5, 37]
     exact = X.astype(np.float64) @ W.astype(np.float64).T
     assert np.abs(r["Y"] - exact).max() < 0.05
+
+
+# ------------------------------------------------------------------ bias and activation after the linear
+
+def test_gelu_tanh_matches_library_routine(oracle_mod):
+    """The oracle's BLOOM GELU (page "优化故事：Bloom 推理", section "唾手可得的优化")
+    against torch's tanh-approximated GELU, an independent library routine.
+    The page writes sqrt(2/pi) as 0.79788456 (torch: 0.7978845608...), a
+    relative difference of 1e-9."""
+    import torch
+    y = np.linspace(-12.0, 12.0, 4801).reshape(1, -1)
+    got = oracle_mod.bias_act(y, activation="gelu_tanh")
+    ref = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
+    assert np.all(np.abs(got - ref) <= 1e-8 * (1.0 + np.abs(y)))
+
+
+def test_gelu_tanh_identities(oracle_mod):
+    """g(0) = 0, g(y) - g(-y) = y (tanh is odd), g(y) -> y for large y and
+    -> 0 for very negative y."""
+    y = np.concatenate([np.linspace(-8, 8, 1601), [0.0, 40.0, -40.0]]).reshape(1, -1)
+    g = oracle_mod.bias_act(y, activation="gelu_tanh")[0]
+    gm = oracle_mod.bias_act(-y, activation="gelu_tanh")[0]
+    assert g[-3] == 0.0
+    assert np.all(np.abs((g - gm) - y[0]) <= 1e-12 * (1.0 + np.abs(y[0])))
+    assert abs(g[-2] - 40.0) < 1e-12 and abs(g[-1]) < 1e-12
+
+
+def test_bias_is_added_per_output_feature(oracle_mod):
+    """Y = linear + bias[j]: the bias follows the output feature (column of Y)."""
+    lin = Linear("b", 6, 40, 64, 2, 20.0)
+    X16, _ = make_activations(lin, seed=3)
+    W16 = make_weight(lin, seed=4)
+    bias = np.random.default_rng(5).standard_normal(40).astype(np.float16)
+    r = oracle_mod.matmul_mixed(X16, 6.0, W=W16, bias=bias)
+    diff = r["Y"] - r["Y_lin"]
+    assert np.allclose(diff, np.broadcast_to(bias.astype(np.float64), diff.shape), rtol=0, atol=1e-12)
+    # a per-row (token) bias would be a different matrix
+    assert not np.allclose(diff, bias[:6].astype(np.float64)[:, None], atol=1e-3)
