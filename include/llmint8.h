@@ -203,6 +203,28 @@ LLMINT8_API llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M,
                                        void *Y_f16, void *workspace, size_t ws_bytes,
                                        const llmint8_debug *dbg, llmint8_stream_t stream);
 
+/* Bytes of workspace needed by llmint8_matmul_mixed_fp16w: that of
+ * llmint8_matmul_mixed plus room for W's codes [N x K] and row absmax [N]. */
+LLMINT8_API size_t llmint8_workspace_size_fp16w(int64_t M, int64_t N, int64_t K);
+
+/*
+ * The linear in the "has fp16 weights" mode of Linear8bitLt (page "Hugging
+ * Face 将 LLM.int8() 8-bit 量化集成进 transformers 与 accelerate", section
+ * "用法": the default, meant for mixed int8/fp16 training): W stays in fp16
+ * and is quantized per output row on every call (llmint8_quantize_rowwise
+ * with t <= 0, into the workspace), then the call proceeds as
+ * llmint8_matmul_mixed_ex with W_f16 supplying the outlier columns. The
+ * result is identical to quantizing W once and calling llmint8_matmul_mixed_ex.
+ *   W_f16      (device) fp16 [N x K], required
+ *   workspace  >= llmint8_workspace_size_fp16w(M, N, K) bytes, zeroed once
+ *   dbg        as for llmint8_matmul_mixed
+ * Other arguments and errors as for llmint8_matmul_mixed_ex.
+ */
+LLMINT8_API llmint8_status llmint8_matmul_mixed_fp16w(const void *X_f16, int64_t M, int64_t K, const void *W_f16,
+                                          int64_t N, float threshold, const void *bias_f16, int activation,
+                                          void *Y_f16, void *workspace, size_t ws_bytes,
+                                          const llmint8_debug *dbg, llmint8_stream_t stream);
+
 /*
  * Plain int8 GEMM with int32 output: acc[i,j] = sum_k A[i,k] * B[j,k]
  * (the int8 product of vector-wise quantization, [Q]).

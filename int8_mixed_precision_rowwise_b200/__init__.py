@@ -18,7 +18,8 @@ import os
 __all__ = [
     "LIB_PATH", "LLMInt8Error", "status_string", "quantize_workspace_size", "workspace_size",
     "workspace_init", "read_status", "quantize_rowwise", "find_outlier_cols", "matmul_mixed",
-    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc",
+    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc", "matmul_mixed_fp16w",
+    "workspace_size_fp16w", "ACTIVATIONS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
@@ -48,6 +49,9 @@ _SIGNATURES = {
                                    ctypes.POINTER(_Debug), _P]),
     "llmint8_matmul_mixed_ex": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, ctypes.c_float, _P, ctypes.c_int, _P, _P,
                                       ctypes.c_size_t, ctypes.POINTER(_Debug), _P]),
+    "llmint8_workspace_size_fp16w": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "llmint8_matmul_mixed_fp16w": (_ST, [_P, _I64, _I64, _P, _I64, ctypes.c_float, _P, ctypes.c_int, _P, _P,
+                                         ctypes.c_size_t, ctypes.POINTER(_Debug), _P]),
     "llmint8_gemm_s8s8s32": (_ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
     "llmint8_quantize_rowwise_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
 }
@@ -263,6 +267,39 @@ def matmul_mixed(X, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y
     return Y
 
 
+def workspace_size_fp16w(M: int, N: int, K: int) -> int:
+    return int(load()["_workspace_size_fp16w"](M, N, K))
+
+
+def matmul_mixed_fp16w(X, W_f16, threshold: float = DEFAULT_THRESHOLD, Y=None, workspace=None,
+                       debug: dict | None = None, bias=None, activation=None):
+    """The linear with W kept in fp16 and quantized per output row on every
+    call ("has fp16 weights" mode): Y fp16 [M x N] from X fp16 [M x K] and
+    W_f16 fp16 [N x K]; bias, activation and debug as for matmul_mixed."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    _need_cuda(W_f16, "W_f16", torch.float16)
+    if bias is not None:
+        _need_cuda(bias, "bias", torch.float16)
+    if activation not in ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(k for k in ACTIVATIONS if k)} or None")
+    M, K = X.shape
+    N = W_f16.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    ws = workspace if workspace is not None else get_workspace(workspace_size_fp16w(M, N, K), dev)
+    dbg = None
+    if debug:
+        dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")),
+                     *(_event(debug.get(k)) for k in ("gemm_begin", "gemm_end")))
+    _check(load()["_matmul_mixed_fp16w"](X.data_ptr(), M, K, W_f16.data_ptr(), N, float(threshold), _ptr(bias),
+                                         ACTIVATIONS[activation], Y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                         ctypes.byref(dbg) if dbg else None, _stream_ptr(dev)),
+           "llmint8_matmul_mixed_fp16w")
+    return Y
+
+
 def gemm_s8s8s32(A, B, acc=None, workspace=None):
     """int32 [M x N] = A int8 [M x K] . B int8 [N x K]^T."""
     torch = _torch()
@@ -283,17 +320,27 @@ class Int8MixedLinear:
     for the outlier columns), an optional fp16 bias and an optional activation
     fused after it, and applies matmul_mixed."""
 
-    def __init__(self, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, bias=None, activation=None):
+    def __init__(self, CB, SCB, W_f16=None, threshold: float = DEFAULT_THRESHOLD, bias=None, activation=None,
+                 has_fp16_weights: bool = False):
         self.CB, self.SCB, self.W_f16, self.threshold = CB, SCB, W_f16, threshold
         self.bias, self.activation = bias, activation
+        # True: only W_f16 is kept and quantized on every call (Linear8bitLt's
+        # training mode); CB/SCB are then unused.
+        self.has_fp16_weights = has_fp16_weights
 
     @classmethod
     def from_fp16(cls, W, threshold: float = DEFAULT_THRESHOLD, keep_fp16_weights: bool = True, bias=None,
-                  activation=None):
-        """Quantize W fp16 [N x K] per output row (offline weight preparation)."""
+                  activation=None, has_fp16_weights: bool = False):
+        """Quantize W fp16 [N x K] per output row (offline weight preparation),
+        or, with has_fp16_weights, keep W in fp16 and quantize it per call."""
+        if has_fp16_weights:
+            return cls(None, None, W, threshold, bias, activation, has_fp16_weights=True)
         CB, SCB, _ = quantize_rowwise(W, 0.0)
         return cls(CB, SCB, W if keep_fp16_weights else None, threshold, bias, activation)
 
     def __call__(self, X, Y=None):
+        if self.has_fp16_weights:
+            return matmul_mixed_fp16w(X, self.W_f16, self.threshold, Y=Y, bias=self.bias,
+                                      activation=self.activation)
         return matmul_mixed(X, self.CB, self.SCB, self.W_f16, self.threshold, Y=Y, bias=self.bias,
                             activation=self.activation)

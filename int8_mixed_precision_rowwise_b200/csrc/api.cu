@@ -142,6 +142,13 @@ size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K)
     return carve(nullptr, M, K, true, decode_shape(M, N), nullptr);
 }
 
+size_t llmint8_workspace_size_fp16w(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return 0;
+    return align256(llmint8_workspace_size(M, N, K)) + align256((size_t)N * (size_t)K) + align256((size_t)N * 4);
+}
+
 llmint8_status llmint8_workspace_init(void *workspace, size_t ws_bytes, llmint8_stream_t stream)
 {
     if (!workspace || ws_bytes < 256)
@@ -322,6 +329,47 @@ llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, 
         return LLMINT8_ERR_CUDA;
 
     return copy_debug(dbg, ws, M, N, K, CB, SCB, X_f16, W_f16, true, dev, stream);
+}
+
+llmint8_status llmint8_matmul_mixed_fp16w(const void *X_f16, int64_t M, int64_t K, const void *W_f16, int64_t N,
+                                          float threshold, const void *bias_f16, int activation, void *Y_f16,
+                                          void *workspace, size_t ws_bytes, const llmint8_debug *dbg,
+                                          llmint8_stream_t stream)
+{
+    // The checks of llmint8_matmul_mixed_ex that matter before W is quantized.
+    if (M < 0 || N < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k(K);
+    if (st != LLMINT8_OK)
+        return st;
+    if (M > INT32_MAX || N > INT32_MAX || M * K > (int64_t)1 << 40 || N * K > (int64_t)1 << 40)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (!X_f16 || !W_f16 || !Y_f16 || !workspace)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (activation != LLMINT8_ACT_NONE && activation != LLMINT8_ACT_GELU_TANH)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X_f16) || !aligned16(W_f16) || !aligned16(Y_f16) || !aligned16(workspace) ||
+        (bias_f16 && !aligned16(bias_f16)))
+        return LLMINT8_ERR_ALIGNMENT;
+    if (ws_bytes < llmint8_workspace_size_fp16w(M, N, K))
+        return LLMINT8_ERR_WORKSPACE;
+    if (M == 0 || N == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    // W's codes and row absmax live after the linear's own workspace.
+    const size_t base = align256(llmint8_workspace_size(M, N, K));
+    char *w = static_cast<char *>(workspace);
+    int8_t *cb = reinterpret_cast<int8_t *>(w + base);
+    float *sb = reinterpret_cast<float *>(w + base + align256((size_t)N * (size_t)K));
+    Workspace ws;
+    carve(w, M, K, true, decode_shape(M, N), &ws);
+    if (launch_quantize(W_f16, N, K, 0.f, cb, sb, nullptr, ws.col_idx, ws.count, ws.sync, ws.status, dev,
+                        stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return llmint8_matmul_mixed_ex(X_f16, M, K, cb, sb, W_f16, N, threshold, bias_f16, activation, Y_f16, workspace,
+                                   base, dbg, stream);
 }
 
 llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B, int64_t N, int64_t K,

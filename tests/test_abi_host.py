@@ -102,6 +102,22 @@ def test_matmul_ex_argument_errors(lib):
     assert call(wsb=1024, bias=A, act=1) == lib.ERR_WORKSPACE
 
 
+def test_matmul_fp16w_argument_errors(lib):
+    f = lib._matmul_mixed_fp16w
+    M, N, K = 64, 64, 128
+    ws = lib.workspace_size_fp16w(M, N, K)
+    assert ws >= lib.workspace_size(M, N, K) + N * K + 4 * N
+
+    def call(W=A, wsb=ws, K=K, act=0):
+        return f(A, M, K, W, N, 6.0, None, act, A, A, wsb, None, None)
+
+    assert call(W=None) == lib.ERR_INVALID_ARG
+    assert call(W=A + 8) == lib.ERR_ALIGNMENT
+    assert call(wsb=lib.workspace_size(M, N, K)) == lib.ERR_WORKSPACE
+    assert call(K=100) == lib.ERR_UNSUPPORTED_SHAPE
+    assert call(act=3) == lib.ERR_INVALID_ARG
+
+
 def test_quantize_argument_errors(lib):
     q = lib._quantize_rowwise
     ws = lib.quantize_workspace_size(32, 64)

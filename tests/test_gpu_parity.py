@@ -360,6 +360,36 @@ def test_matmul_mixed_bias_activation(lib, dev, oracle_mod, M, N, K, act):
     assert not bad.any(), f"{bad.sum()} outside tolerance, worst {np.abs(y - r['Y']).max()}"
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 520, 1040), (4, 640, 1024), (64, 256, 4096)])
+def test_fp16_weights_mode(lib, dev, oracle_mod, M, N, K):
+    """llmint8_matmul_mixed_fp16w quantizes W on every call: its output is
+    bit-identical to quantizing W once and calling matmul_mixed_ex, and its
+    codes, outlier set and int32 products match the oracle exactly."""
+    lin = Linear("fw", M, N, K, 4, 60.0)
+    X16, _ = make_activations(lin, seed=M + N + K)
+    W16 = make_weight(lin, seed=7)
+    bias = np.random.default_rng(3).standard_normal(N).astype(np.float16)
+    X, W, b = to_dev(X16, dev), to_dev(W16, dev), to_dev(bias, dev)
+    dbg = dict(codes=torch.empty((M, K), dtype=torch.int8, device=dev),
+               row_absmax=torch.empty(M, dtype=torch.float32, device=dev),
+               col_idx=torch.empty(K, dtype=torch.int32, device=dev),
+               count=torch.empty(1, dtype=torch.int32, device=dev),
+               acc=torch.empty((M, N), dtype=torch.int32, device=dev))
+    Y1 = lib.matmul_mixed_fp16w(X, W, 6.0, bias=b, activation="gelu_tanh", debug=dbg)
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    Y2 = lib.matmul_mixed(X, CB, SCB, W, 6.0, bias=b, activation="gelu_tanh")
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    r = oracle_mod.matmul_mixed(X16, 6.0, W=W16, bias=bias, activation="gelu_tanh")
+    n = int(dbg["count"].item())
+    assert np.array_equal(dbg["col_idx"][:n].cpu().numpy(), r["O"])
+    assert np.array_equal(dbg["codes"].cpu().numpy(), r["CX"])
+    assert np.array_equal(dbg["acc"].cpu().numpy(), r["acc"])
+    y = Y1.cpu().numpy().astype(np.float64)
+    pre = r["Y_lin"] + bias.astype(np.float64)[None, :]
+    assert np.all(np.abs(y - r["Y"]) <= 1.13 * (1e-2 + 2e-3 * np.abs(pre)) + 5e-4 * np.abs(r["Y"]))
+
+
 def test_repeat_calls_identical(lib, dev):
     lin = Linear("t", 300, 600, 1024, 4, 60.0)
     X16, _ = make_activations(lin, seed=1)
