@@ -374,7 +374,6 @@ def measure_secondary(L, dev):
     out["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
                                   "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
     del bufs, fns
-    out["per_linear"] = per_linear_times(L, dev)
     for M in (1, 8, 32):
         lin = synthetic.decode_bloom(M).linears[0]
         X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
@@ -387,6 +386,8 @@ def measure_secondary(L, dev):
                                "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
         del layer, X, Y
     torch.cuda.empty_cache()
+    # Last: the per-linear GEMMs run the GPU at its power cap for seconds.
+    out["per_linear"] = per_linear_times(L, dev)
     return out
 
 

@@ -259,6 +259,15 @@ __device__ bool row_scales(const DParams &p, int et, uint32_t xloaded_bar, uint3
         s_hit[i] = 0u;
     if (et < 32)
         s_rmax[et] = 0u;
+    // This CTA's partial-ready flag and (CTA 0) the outlier-list flag are read
+    // only after the second grid barrier: clearing them here, before the
+    // first one, keeps whatever an earlier call (or other data) left there
+    // from ever matching this call's generation.
+    if (et == 0) {
+        p.pflags[c] = 0u;
+        if (c == 0)
+            p.sync[3] = 0u;
+    }
     named_barrier_sync(1, NHELP);
     // The first PC vectors of each thread stay in registers for the maxima.
     constexpr int PC = 4;
