@@ -197,14 +197,19 @@ llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t
     cudaError_t e = device_info(&dev);
     if (e != cudaSuccess)
         return LLMINT8_ERR_CUDA;
+    if (quantize_smem_fits(rows, cols, dev)) {
+        // X fits in shared memory: one kernel, nothing to clear first.
+        e = launch_quantize_smem(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.tagged, ws.col_idx,
+                                 ws.count, ws.sync, ws.status, dev, stream);
+        return cuda_status(e);
+    }
+    // The streaming quantizer ORs into the caller's bitmap: clear it. (Its
+    // other state clears itself; the barrier word keeps its generation.)
     const size_t nwords = (size_t)((cols + 31) / 32);
     if (outlier_bitmap) {
         if ((e = cudaMemsetAsync(outlier_bitmap, 0, nwords * 4, stream)) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
     }
-    // |O| and the kernel's sync words (header bytes 4..23); the status word stays.
-    if ((e = cudaMemsetAsync(ws.count, 0, 20, stream)) != cudaSuccess)
-        return LLMINT8_ERR_CUDA;
     e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.col_idx, ws.count, ws.sync,
                         ws.status, dev, stream);
     return cuda_status(e);
@@ -294,14 +299,20 @@ llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, 
         return copy_debug(dbg, ws, M, N, K, CB, SCB, X_f16, W_f16, false, dev, stream);
     }
 
-    // Clear |O| and the bitmap (one memset: they sit next to each other).
-    char *clear_from = reinterpret_cast<char *>(ws.count);
-    const size_t clear_bytes = (reinterpret_cast<char *>(ws.bitmap) - clear_from) + (size_t)((K + 31) / 32) * 4;
-    if ((e = cudaMemsetAsync(clear_from, 0, clear_bytes, stream)) != cudaSuccess)
-        return LLMINT8_ERR_CUDA;
-    if ((e = launch_quantize(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws.col_idx, ws.count, ws.sync, ws.status,
-                             dev, stream)) != cudaSuccess)
-        return LLMINT8_ERR_CUDA;
+    if (quantize_smem_fits(M, K, dev)) {
+        // X fits in shared memory: one kernel, nothing to clear first.
+        if ((e = launch_quantize_smem(X_f16, M, K, t, ws.cx, ws.sx, nullptr, ws.tagged, ws.col_idx, ws.count,
+                                      ws.sync, ws.status, dev, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    } else {
+        // The streaming quantizer ORs into the bitmap: clear it. (Its other
+        // state clears itself; the barrier word keeps its generation.)
+        if ((e = cudaMemsetAsync(ws.bitmap, 0, (size_t)((K + 31) / 32) * 4, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+        if ((e = launch_quantize(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws.col_idx, ws.count, ws.sync,
+                                 ws.status, dev, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    }
 
     GemmArgs g{};
     g.A = ws.cx;

@@ -18,9 +18,12 @@ constexpr int kHeaderBytes = 256;
 // Workspace layout (byte offsets; every region 256-byte aligned):
 //   [0]      uint32 status word (bits LLMINT8_DEV_*)
 //   [4]      int32  |O| (outlier column count)
-//   [8]      uint32 grid-barrier counter and generation, late-outlier flag,
-//            decode outlier-list flag
+//   [8]      uint64 grid barrier: arrival count (low half), generation (high
+//            half); never cleared by the library after workspace_init
+//   [16]     uint32 late-outlier flag, [20] decode outlier-list flag
 //   [256]    uint32 outlier bitmap [ceil(K/32)]
+//   ...      uint64 epoch-tagged outlier bitmap [ceil(K/32)] (upper half: the
+//            call's barrier generation; words of other calls count as empty)
 //   ...      int32  ascending outlier columns [K]
 //   ...      fp32   SX [M]
 //   ...      int8   CX [M x K]
@@ -35,6 +38,7 @@ struct Workspace {
     int32_t *count;
     uint32_t *sync;
     uint32_t *bitmap;
+    unsigned long long *tagged;
     int32_t *col_idx;
     float *sx;
     int8_t *cx;
@@ -63,6 +67,7 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
     char *hdr = take(kHeaderBytes);
     size_t nwords = (size_t)((K + 31) / 32);
     char *bm = take(nwords * 4);
+    char *tg = take(nwords * 8);
     char *ci = take((size_t)K * 4);
     char *sx = with_codes ? take((size_t)M * 4) : nullptr;
     char *cx = with_codes ? take((size_t)M * (size_t)K) : nullptr;
@@ -75,6 +80,7 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
         ws->count = hdr ? reinterpret_cast<int32_t *>(hdr + 4) : nullptr;
         ws->sync = hdr ? reinterpret_cast<uint32_t *>(hdr + 8) : nullptr;
         ws->bitmap = reinterpret_cast<uint32_t *>(bm);
+        ws->tagged = reinterpret_cast<unsigned long long *>(tg);
         ws->col_idx = reinterpret_cast<int32_t *>(ci);
         ws->sx = reinterpret_cast<float *>(sx);
         ws->cx = reinterpret_cast<int8_t *>(cx);
@@ -108,6 +114,15 @@ cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols, float t, 
 // The smallest fp16 value >= t, so that for fp16 x, |x| >= t exactly when
 // |x| >= threshold_fp16(t) (+inf when no finite value qualifies, 0 for t <= 0).
 __half threshold_fp16(float t);
+
+// The quantizer for an X whose rows fit in the shared memory of one CTA per
+// SM (one read of X, one grid barrier, nothing to clear before the call):
+// `tagged` is the workspace's epoch-tagged bitmap, bitmap_out (may be null)
+// receives the outlier bitmap, col_idx/count the ascending outlier columns.
+bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev);
+cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
+                                 uint32_t *bitmap_out, unsigned long long *tagged, int32_t *col_idx, int32_t *count,
+                                 uint32_t *sync, uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
 
 // Bitmap -> ascending column list and count (one CTA).
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

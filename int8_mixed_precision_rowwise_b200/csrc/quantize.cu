@@ -328,9 +328,17 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     uint4 v[V];
     griddep_release(); // the GEMM may start its weight stream now; it waits for this kernel's output
 
+    if constexpr (!THR) {
+        if (blockIdx.x == 0 && tid == 0 && count)
+            *count = 0; // no outlier columns
+    }
     if constexpr (THR) {
         for (int w = tid; w < nwords; w += 256)
             s_known[w] = 0u;
+        // The late-column flag is raised only after the first barrier: clear
+        // it here (before anyone can raise it) instead of before the launch.
+        if (blockIdx.x == 0 && tid == 0)
+            sync[2] = 0u;
         __syncthreads();
         // A row that fits in registers is read here once and for all: every
         // group seeds its first row and keeps it for the quantize step, so
@@ -526,6 +534,155 @@ cudaError_t launch_fused_v(const void *X, int64_t rows, int cols, float t, int8_
                                                      status, dev, stream);
 }
 
+// OR `bits` into the epoch-tagged bitmap word *w (epoch in the upper 32
+// bits, set bits in the lower 32): a word tagged with another epoch counts as
+// empty. Returns false if the compare-and-swap kept losing (bounded).
+__device__ bool tagged_or(unsigned long long *w, uint32_t epoch, uint32_t bits)
+{
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(w);
+    for (int n = 0; n < 100000; ++n) {
+        const unsigned long long want = ((uint32_t)(old >> 32) == epoch)
+                                            ? (old | bits)
+                                            : (((unsigned long long)epoch << 32) | bits);
+        if (want == old)
+            return true;
+        const unsigned long long prev = atomicCAS(w, old, want);
+        if (prev == old)
+            return true;
+        old = prev;
+    }
+    return false;
+}
+
+// The quantizer for an X that fits in the shared memory of one CTA per SM.
+// Each CTA holds its block of rows (contiguous in X) for the whole call:
+//   load    - one bulk copy of the block into shared memory;
+//   mark    - the block's outlier columns (|x| >= t16), published into a
+//             bitmap of 64-bit words tagged with this call's epoch (the grid
+//             barrier's generation at the start, the same in every CTA), so
+//             that no word needs clearing between calls;
+//   barrier - after it the words tagged with the epoch are the complete set;
+//   rows    - one warp per row: maximum over the non-outlier columns, codes
+//             (rint(x * 127 / absmax), outlier columns 0), absmax; CTA 0
+//             writes the output bitmap and the ascending outlier columns.
+// The set is complete before any row is quantized, so the result is the
+// definition's with no fix-up, after a single read of X from HBM.
+template <bool THR>
+__global__ void __launch_bounds__(256, 1)
+    k_quant_smem(const uint4 *__restrict__ X, int rows, int cols, __half t16, int8_t *__restrict__ codes,
+                 float *__restrict__ absmax, uint32_t *__restrict__ bitmap_out, unsigned long long *tagged,
+                 int32_t *__restrict__ col_idx, int32_t *__restrict__ count, uint32_t *sync,
+                 uint32_t *__restrict__ status)
+{
+    extern __shared__ __align__(1024) uint8_t q_smem[];
+    __shared__ uint64_t s_bar;
+    __shared__ int s_flag;
+    __shared__ uint32_t s_epoch;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nvec = cols >> 3, nwords = (cols + 31) >> 5;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int r0 = (int)((int64_t)c * rows / G), r1 = (int)((int64_t)(c + 1) * rows / G);
+    const int nr = r1 - r0;
+    const uint4 *sx = reinterpret_cast<const uint4 *>(q_smem);
+    const uint32_t xbytes = (uint32_t)nr * (uint32_t)cols * 2u;
+    uint32_t *s_bm = reinterpret_cast<uint32_t *>(q_smem + ((xbytes + 15u) & ~15u));
+    const uint32_t bar = smem_u32(&s_bar);
+    griddep_release();
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        unsigned long long w;
+        asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(w) : "l"(sync) : "memory");
+        s_epoch = (uint32_t)(w >> 32);
+        s_flag = 1;
+    }
+    for (int w = tid; w < nwords; w += 256)
+        s_bm[w] = 0u;
+    __syncthreads();
+    if (tid == 0 && nr > 0) {
+        mbar_arrive_expect_tx(bar, xbytes);
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(X + (int64_t)r0 * nvec);
+        for (uint32_t off = 0; off < xbytes; off += 32768u)
+            bulk_load(smem_u32(q_smem) + off, src + off, min(32768u, xbytes - off), bar);
+    }
+    const uint32_t epoch = s_epoch;
+    bool ok = true;
+    if (nr > 0)
+        ok = mbar_wait(bar, 0u);
+    if (THR && ok) {
+        for (int i = tid; i < nr * nvec; i += 256) {
+            const uint32_t h = hit_mask8(sx[i], t16);
+            if (h) {
+                const int vi = i % nvec;
+                atomicOr(&s_bm[vi >> 2], h << ((vi & 3) * 8));
+            }
+        }
+    }
+    __syncthreads();
+    if (THR && ok) {
+        for (int w = tid; w < nwords; w += 256) {
+            const uint32_t bits = s_bm[w];
+            if (bits && !tagged_or(tagged + w, epoch, bits))
+                ok = false;
+        }
+    }
+    if (!ok)
+        atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
+    __syncthreads();
+    if (tid == 0) {
+        s_flag = grid_barrier(sync, (uint32_t)G) ? 1 : 0;
+        if (!s_flag)
+            atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
+    }
+    __syncthreads();
+    if (!s_flag || !ok)
+        return;
+    if (THR) {
+        for (int w = tid; w < nwords; w += 256) {
+            const unsigned long long t = __ldcg(tagged + w);
+            s_bm[w] = ((uint32_t)(t >> 32) == epoch) ? (uint32_t)t : 0u;
+        }
+        __syncthreads();
+    }
+    for (int r = warp; r < nr; r += 8) {
+        const uint4 *xr = sx + (int64_t)r * nvec;
+        __half2 m2 = __float2half2_rn(0.f);
+        for (int vi = lane; vi < nvec; vi += 32) {
+            uint4 v = xr[vi];
+            const uint32_t kb = (s_bm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+            if (kb)
+                mask_known(v, kb);
+            __half2 a[4];
+            m2 = __hmax2(m2, vec_abs_max(v, a));
+        }
+        float amax = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float s = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+        int8_t *cr = codes + (int64_t)(r0 + r) * cols;
+        for (int vi = lane; vi < nvec; vi += 32) {
+            uint4 v = xr[vi];
+            const uint32_t kb = (s_bm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+            if (kb)
+                mask_known(v, kb);
+            *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) = codes8(v, s);
+        }
+        if (lane == 0)
+            absmax[r0 + r] = amax;
+    }
+    if (c == 0) {
+        if (bitmap_out)
+            for (int w = tid; w < nwords; w += 256)
+                bitmap_out[w] = s_bm[w];
+        if (THR)
+            compact_block<256>(s_bm, nwords, col_idx, count);
+        else if (tid == 0)
+            *count = 0;
+    }
+}
+
 } // namespace
 
 // The smallest fp16 value >= t, so that for fp16 x, |x| >= t exactly when
@@ -564,6 +721,58 @@ cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols64, float t
         return launch_fused_v<8, 32>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
                                      stream);
     return launch_fused_v<8, 8>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev, stream);
+}
+
+namespace {
+
+size_t quant_smem_bytes(int64_t rows, int64_t cols, int num_sms)
+{
+    const int64_t per = (rows + num_sms - 1) / num_sms;
+    return (size_t)((per * cols * 2 + 15) & ~15ll) + (size_t)((cols + 31) / 32) * 4;
+}
+
+} // namespace
+
+bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev)
+{
+    // Room for the block of rows and the bitmap, under the opt-in limit with
+    // a margin for the kernel's static shared memory.
+    return rows >= 1 && cols >= 8 && cols % 8 == 0 && rows <= INT32_MAX &&
+           quant_smem_bytes(rows, cols, dev.num_sms) + 2048 <= (size_t)dev.max_smem_optin;
+}
+
+cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
+                                 uint32_t *bitmap_out, unsigned long long *tagged, int32_t *col_idx, int32_t *count,
+                                 uint32_t *sync, uint32_t *status, const DeviceInfo &dev, cudaStream_t stream)
+{
+    const bool thr = t > 0.f;
+    auto kern = thr ? k_quant_smem<true> : k_quant_smem<false>;
+    const size_t smem = quant_smem_bytes(rows, cols, dev.num_sms);
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, size_t> configured; // (device, thr) -> bytes set
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        size_t &have = configured[std::make_pair(dev.device, thr ? 1 : 0)];
+        if (have < smem) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 dev.max_smem_optin - 1024);
+            if (e != cudaSuccess)
+                return e;
+            have = (size_t)dev.max_smem_optin - 1024;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)dev.num_sms);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative; // the grid barrier needs every CTA resident
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const uint4 *>(X), (int)rows, (int)cols,
+                              threshold_fp16(t), codes, absmax, bitmap_out, tagged, col_idx, count, sync, status);
 }
 
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

@@ -91,7 +91,9 @@ def check_full(lib, dev, oracle_mod, X16, W16, t, give_w16=True):
 # ------------------------------------------------------------------ quantizer
 
 @pytest.mark.parametrize("M,K,nout,scale", [(8, 64, 2, 20.0), (300, 1024, 5, 40.0), (513, 4096, 8, 40.0),
-                                            (64, 14336, 6, 60.0), (9, 57344, 29, 60.0), (3, 16, 1, 60.0)])
+                                            (64, 14336, 6, 60.0), (9, 57344, 29, 60.0), (3, 16, 1, 60.0),
+                                            # too large for shared memory: the streaming quantizer
+                                            (6000, 4096, 8, 40.0), (1500, 12288, 6, 40.0)])
 def test_quantize_rowwise_matches_oracle(lib, dev, oracle_mod, M, K, nout, scale):
     X16, _ = make_activations(Linear("q", M, 0, K, nout, scale), seed=M + K)
     codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
@@ -157,11 +159,13 @@ def test_quantize_edge_rows(lib, dev, oracle_mod):
 
 
 def test_quantize_late_outlier_column(lib, dev, oracle_mod):
-    """8192 rows: the outlier-column seed reads only the first rows, so a
-    column that crosses the threshold only in row 8100 is found late, while
-    rows 7000.. already took their maximum (5.5) in it. The result must still
-    be the definition's (every row re-quantized against the final set)."""
-    X = np.random.default_rng(8).standard_normal((8192, 2048)).astype(np.float32)
+    """8192 x 4096 (too large for the shared-memory quantizer, so the
+    streaming one with its seed runs): the seed reads each warp's first row
+    only, so a column that crosses the threshold only in row 8100 is found
+    late, while rows 7000.. already took their maximum (5.5) in it. The result
+    must still be the definition's (every row re-quantized against the final
+    set)."""
+    X = np.random.default_rng(8).standard_normal((8192, 4096)).astype(np.float32)
     X[:, 100] *= 0.1
     X[7000:, 100] = 5.5
     X[8100, 100] = 50.0
@@ -170,7 +174,7 @@ def test_quantize_late_outlier_column(lib, dev, oracle_mod):
     mask = oracle_mod.outlier_mask(X16, 6.0)
     assert mask[100]
     c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
-    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 2048), mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 4096), mask)
     assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
     assert np.array_equal(codes.cpu().numpy(), c_ref)
 
