@@ -79,7 +79,10 @@ LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t rows, int64_t cols);
 LLMINT8_API size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* Zero a workspace (a cudaMemsetAsync). A workspace must be zeroed once before
- * its first use; every call leaves it ready for the next one. */
+ * its first use; every call leaves it ready for the next one. Calls of any
+ * entry point and any shape may share one workspace; between calls it holds
+ * the library's state (a grid-barrier generation, epoch-tagged words), so the
+ * caller must not write into it. */
 LLMINT8_API llmint8_status llmint8_workspace_init(void *workspace, size_t ws_bytes, llmint8_stream_t stream);
 
 /* Synchronously read (and, if clear != 0, reset) the device status word of a

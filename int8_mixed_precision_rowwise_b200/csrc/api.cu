@@ -199,7 +199,7 @@ llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t
         return LLMINT8_ERR_CUDA;
     if (quantize_smem_fits(rows, cols, dev)) {
         // X fits in shared memory: one kernel, nothing to clear first.
-        e = launch_quantize_smem(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.tagged, ws.col_idx,
+        e = launch_quantize_smem(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.sets, ws.calls, ws.col_idx,
                                  ws.count, ws.sync, ws.status, dev, stream);
         return cuda_status(e);
     }
@@ -301,7 +301,7 @@ llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, 
 
     if (quantize_smem_fits(M, K, dev)) {
         // X fits in shared memory: one kernel, nothing to clear first.
-        if ((e = launch_quantize_smem(X_f16, M, K, t, ws.cx, ws.sx, nullptr, ws.tagged, ws.col_idx, ws.count,
+        if ((e = launch_quantize_smem(X_f16, M, K, t, ws.cx, ws.sx, nullptr, ws.sets, ws.calls, ws.col_idx, ws.count,
                                       ws.sync, ws.status, dev, stream)) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
     } else {

@@ -7,6 +7,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "llmint8.h"
+
 namespace llmint8 {
 
 // Decode (M <= kDecodeMaxM tokens) runs as one fused kernel with at most
@@ -14,6 +16,7 @@ namespace llmint8 {
 constexpr int kDecodeMaxM = 32;
 constexpr int kDecodeMaxCtas = 160;
 constexpr int kHeaderBytes = 256;
+constexpr size_t kSetWords = (LLMINT8_MAX_K + 31) / 32; // bitmap words of the widest X
 
 // Workspace layout (byte offsets; every region 256-byte aligned):
 //   [0]      uint32 status word (bits LLMINT8_DEV_*)
@@ -21,9 +24,13 @@ constexpr int kHeaderBytes = 256;
 //   [8]      uint64 grid barrier: arrival count (low half), generation (high
 //            half); never cleared by the library after workspace_init
 //   [16]     uint32 late-outlier flag, [20] decode outlier-list flag
-//   [256]    uint32 outlier bitmap [ceil(K/32)]
-//   ...      uint64 epoch-tagged outlier bitmap [ceil(K/32)] (upper half: the
-//            call's barrier generation; words of other calls count as empty)
+//   [24]     uint32 calls of the shared-memory quantizer so far
+//   [256]    uint32 two outlier bitmaps [2][kSetWords] of the shared-memory
+//            quantizer: call n ORs into set[n & 1] and clears set[(n+1) & 1]
+//            for the next call. Their place and size depend on no shape, so
+//            that whatever shapes share the workspace nothing else is
+//            written there.
+//   ...      uint32 outlier bitmap [ceil(K/32)]
 //   ...      int32  ascending outlier columns [K]
 //   ...      fp32   SX [M]
 //   ...      int8   CX [M x K]
@@ -38,7 +45,8 @@ struct Workspace {
     int32_t *count;
     uint32_t *sync;
     uint32_t *bitmap;
-    unsigned long long *tagged;
+    uint32_t *sets;   // [2][kSetWords]
+    uint32_t *calls;
     int32_t *col_idx;
     float *sx;
     int8_t *cx;
@@ -65,9 +73,9 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
         return base ? base + o : nullptr;
     };
     char *hdr = take(kHeaderBytes);
+    char *tg = take(kSetWords * 8);
     size_t nwords = (size_t)((K + 31) / 32);
     char *bm = take(nwords * 4);
-    char *tg = take(nwords * 8);
     char *ci = take((size_t)K * 4);
     char *sx = with_codes ? take((size_t)M * 4) : nullptr;
     char *cx = with_codes ? take((size_t)M * (size_t)K) : nullptr;
@@ -80,7 +88,8 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
         ws->count = hdr ? reinterpret_cast<int32_t *>(hdr + 4) : nullptr;
         ws->sync = hdr ? reinterpret_cast<uint32_t *>(hdr + 8) : nullptr;
         ws->bitmap = reinterpret_cast<uint32_t *>(bm);
-        ws->tagged = reinterpret_cast<unsigned long long *>(tg);
+        ws->sets = reinterpret_cast<uint32_t *>(tg);
+        ws->calls = hdr ? reinterpret_cast<uint32_t *>(hdr + 24) : nullptr;
         ws->col_idx = reinterpret_cast<int32_t *>(ci);
         ws->sx = reinterpret_cast<float *>(sx);
         ws->cx = reinterpret_cast<int8_t *>(cx);
@@ -117,12 +126,14 @@ __half threshold_fp16(float t);
 
 // The quantizer for an X whose rows fit in the shared memory of one CTA per
 // SM (one read of X, one grid barrier, nothing to clear before the call):
-// `tagged` is the workspace's epoch-tagged bitmap, bitmap_out (may be null)
-// receives the outlier bitmap, col_idx/count the ascending outlier columns.
+// `sets`/`calls` are the workspace's two bitmaps and call counter,
+// bitmap_out (may be null) receives the outlier bitmap, col_idx/count the
+// ascending outlier columns.
 bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev);
 cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
-                                 uint32_t *bitmap_out, unsigned long long *tagged, int32_t *col_idx, int32_t *count,
-                                 uint32_t *sync, uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
+                                 uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls, int32_t *col_idx,
+                                 int32_t *count, uint32_t *sync, uint32_t *status, const DeviceInfo &dev,
+                                 cudaStream_t stream);
 
 // Bitmap -> ascending column list and count (one CTA).
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

@@ -407,9 +407,16 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N)
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// bar.sync / bar.arrive / bar.red are the warp-aligned forms: every thread of
+// the warp must execute the same instruction together. The helpers below
+// reconverge the warp first (a branch on the lane just before them, such as
+// `if (lane == 0) { ... }`, may otherwise leave it split), so each must be
+// reached by all 32 lanes.
+
 // Named barrier over `nthreads` threads that also ORs a predicate across them.
 __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred)
 {
+    __syncwarp();
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -424,7 +431,15 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads)
 {
+    __syncwarp();
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Arrive at a named barrier without waiting (the producer side of bar.sync).
+__device__ __forceinline__ void named_barrier_arrive(int id, int nthreads)
+{
+    __syncwarp();
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 } // namespace llmint8

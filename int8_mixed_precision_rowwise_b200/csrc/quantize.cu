@@ -57,6 +57,7 @@ __device__ void compact_block(const uint32_t *s_bm, int nwords, int32_t *col_idx
     }
     if (lane == 31)
         s_warp[warp] = incl;
+    __syncwarp();
     __syncthreads();
     if (warp == 0) {
         int wv = lane < NT / 32 ? s_warp[lane] : 0;
@@ -72,6 +73,7 @@ __device__ void compact_block(const uint32_t *s_bm, int nwords, int32_t *col_idx
         if (lane == NT / 32 - 1)
             *count = wi;
     }
+    __syncwarp();
     __syncthreads();
     int pos = s_warp[warp] + incl - cnt;
     for (int w = w0; w < w1; ++w) {
@@ -534,150 +536,473 @@ cudaError_t launch_fused_v(const void *X, int64_t rows, int cols, float t, int8_
                                                      status, dev, stream);
 }
 
-// OR `bits` into the epoch-tagged bitmap word *w (epoch in the upper 32
-// bits, set bits in the lower 32): a word tagged with another epoch counts as
-// empty. Returns false if the compare-and-swap kept losing (bounded).
-__device__ bool tagged_or(unsigned long long *w, uint32_t epoch, uint32_t bits)
+// The quantizer for an X that fits in the shared memory of one CTA per SM.
+// Each CTA holds its block of rows (contiguous in X) for the whole call. The
+// block arrives as chunks of whole rows, each bulk-copied into shared memory
+// on an mbarrier of its own, and each of 15 worker warps takes rows
+// w, w + 15, ... as they land. Per row (threshold on):
+//   detect - the row's outlier columns (|x| >= t16) join the CTA's set s_bm;
+//            a column new to it is also ORed (fire and forget) into this
+//            call's global bitmap, and then counted in s_cnt;
+//   c      - the size of the CTA's set, read after the detection;
+//   row    - maximum over the columns outside the set, codes
+//            rint(x * 127 / absmax) (set columns 0) and absmax.
+// A control warp, once every row is detected, passes the grid barrier and
+// reads the complete set back. Sets only grow and every column counted in c
+// was in s_bm before the row read it, so a row whose c equals the size of
+// the complete set used exactly that set; the others (a column that only a
+// later row, or another CTA, saw) are quantized again from shared memory.
+// A short seed step (the first rows of the block detected before any row
+// goes on) makes that rare. The result is the definition's after a single
+// read of X from HBM, with the codes written while the block still arrives
+// and the grid barrier's latency behind the last rows.
+//
+// The global bitmap is one of two in the workspace: call n (the workspace's
+// call counter) ORs into set[n & 1], and CTA 0 clears set[(n + 1) & 1],
+// which no CTA of this call reads, for call n + 1.
+constexpr int kQsWorkers = 480;                 // 15 worker warps (16 warps in all: 128 registers a thread)
+constexpr int kQsWarps = kQsWorkers / 32;
+constexpr int kQsThreads = kQsWorkers + 32;     // + the control warp
+constexpr int kQsMaxChunks = 64;
+constexpr int kQsChunkBytes = 4096;
+constexpr int kQsSeedRows = 4;
+constexpr int kQsRegVec = 16;                   // rows of up to 32 * 16 vectors stay in registers
+
+// Rows of one CTA per chunk: at least kQsChunkBytes, at most kQsMaxChunks chunks.
+__host__ __device__ inline int qs_rows_per_chunk(int nr, int cols)
 {
-    unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(w);
-    for (int n = 0; n < 100000; ++n) {
-        const unsigned long long want = ((uint32_t)(old >> 32) == epoch)
-                                            ? (old | bits)
-                                            : (((unsigned long long)epoch << 32) | bits);
-        if (want == old)
-            return true;
-        const unsigned long long prev = atomicCAS(w, old, want);
-        if (prev == old)
-            return true;
-        old = prev;
-    }
-    return false;
+    const int by_size = (kQsChunkBytes + cols * 2 - 1) / (cols * 2);
+    return max(max(by_size, 1), (nr + kQsMaxChunks - 1) / kQsMaxChunks);
 }
 
-// The quantizer for an X that fits in the shared memory of one CTA per SM.
-// Each CTA holds its block of rows (contiguous in X) for the whole call:
-//   load    - one bulk copy of the block into shared memory;
-//   mark    - the block's outlier columns (|x| >= t16), published into a
-//             bitmap of 64-bit words tagged with this call's epoch (the grid
-//             barrier's generation at the start, the same in every CTA), so
-//             that no word needs clearing between calls;
-//   barrier - after it the words tagged with the epoch are the complete set;
-//   rows    - one warp per row: maximum over the non-outlier columns, codes
-//             (rint(x * 127 / absmax), outlier columns 0), absmax; CTA 0
-//             writes the output bitmap and the ascending outlier columns.
-// The set is complete before any row is quantized, so the result is the
-// definition's with no fix-up, after a single read of X from HBM.
+__device__ __forceinline__ uint32_t set_byte(const uint32_t *bm, int v)
+{
+    return (bm[v >> 2] >> ((v & 3) * 8)) & 0xFFu;
+}
+
+struct QsRow {
+    const uint4 *xr; // the row in shared memory
+    int nvec;
+    __half t16;
+    uint32_t *s_bm;  // the CTA's set (detection adds to it)
+    int *s_cnt;      // its size
+    uint32_t *gset;  // this call's global bitmap
+    int8_t *cr;      // the row's codes
+    float *am;       // the row's absmax
+    int lane;
+};
+
+// Add the outlier columns of vector v (x) to the CTA's set; columns new to
+// it are ORed into the global bitmap (no reply awaited), then counted.
+// Returns true if it added any. Out of line: it runs for the few vectors
+// holding an outlier, and inlined into every unrolled step it would crowd
+// the instruction cache that the common path runs from.
+__device__ __noinline__ bool qs_publish(uint4 x, int v, __half t16, uint32_t *s_bm, int *s_cnt, uint32_t *gset)
+{
+    const uint32_t bits = hit_mask8(x, t16) << ((v & 3) * 8);
+    const int w = v >> 2;
+    const uint32_t nb = bits & ~atomicOr(&s_bm[w], bits);
+    if (!nb)
+        return false;
+    atomicOr(gset + w, nb);
+    __threadfence_block(); // the bits are in s_bm before the count says so
+    atomicAdd(s_cnt, __popc(nb));
+    return true;
+}
+
+// |x| maximum of the vector; if it reaches t16, the vector's outlier
+// columns not among `known` (bits of the vector's columns already seen in
+// the CTA's set) are published (pub set when any was new to the CTA).
+__device__ __forceinline__ __half2 qs_detect_vec(const QsRow &q, int v, const uint4 &x, uint32_t known, bool &pub)
+{
+    __half2 a[4];
+    const __half2 m = vec_abs_max(x, a);
+    if (__hge(__hmax(__low2half(m), __high2half(m)), q.t16) && (hit_mask8(x, q.t16) & ~known))
+        pub |= qs_publish(x, v, q.t16, q.s_bm, q.s_cnt, q.gset);
+    return m;
+}
+
+// Size of the CTA's set, read by lane 0 after the warp's detection and
+// ordered before every later read of s_bm by the warp.
+__device__ __forceinline__ int qs_count(const QsRow &q)
+{
+    __syncwarp();
+    int c = 0;
+    if (q.lane == 0)
+        c = *reinterpret_cast<volatile int *>(q.s_cnt);
+    __threadfence_block();
+    c = __shfl_sync(0xffffffffu, c, 0);
+    __syncwarp();
+    return c;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float qs_scale(float amax) { return amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f; }
+
+// Set bytes of one lane's vectors (lane + 32 k), four to a word, and the
+// count c they were read after.
+struct QsSetCache {
+    uint32_t b[kQsRegVec / 4];
+    int count;
+};
+
+__device__ __forceinline__ void qs_load_set(QsSetCache &sc, const uint32_t *bm, int nvec, int lane, int count)
+{
+#pragma unroll
+    for (int j = 0; j < kQsRegVec / 4; ++j) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int v = lane + 32 * (4 * j + i);
+            if (v < nvec)
+                w |= set_byte(bm, v) << (8 * i);
+        }
+        sc.b[j] = w;
+    }
+    sc.count = count;
+}
+
+// Before the warp's last arrival at the detection barrier: the lanes that
+// ORed into the global bitmap wait for those operations to land.
+__device__ __forceinline__ void qs_arrive_detected(bool pub)
+{
+    if (pub)
+        __threadfence();
+    named_barrier_arrive(2, kQsThreads);
+}
+
+// One row held in registers (nvec <= 32 * kQsRegVec), against the CTA's set
+// through the lane's cache sc (or, fixed, against the set sc already holds:
+// no detection, no count). Known outlier columns are masked first; a vector
+// whose remaining maximum still reaches t16 holds a column the cache did not
+// have, and only then is the row's new part of the set published and the
+// maximum taken again against the set read afresh. Returns the count the
+// row's set was read after (0 when !THR or fixed).
+template <bool THR, bool FULL>
+__device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub, bool arrive)
+{
+    uint4 x[kQsRegVec];
+#pragma unroll
+    for (int k = 0; k < kQsRegVec; ++k) {
+        const int v = q.lane + 32 * k;
+        x[k] = (FULL || v < q.nvec) ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (THR && !fixed) { // the set grew since the cache was read: read it again
+        int now = 0;
+        if (q.lane == 0)
+            now = *reinterpret_cast<volatile int *>(q.s_cnt);
+        if (__shfl_sync(0xffffffffu, now, 0) != sc.count)
+            qs_load_set(sc, q.s_bm, q.nvec, q.lane, qs_count(q));
+    }
+    __half2 rm = __float2half2_rn(0.f);
+    bool fresh = false;
+#pragma unroll
+    for (int k = 0; k < kQsRegVec; ++k) {
+        if (THR) {
+            const uint32_t kb = (sc.b[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+            if (kb)
+                mask_known(x[k], kb);
+        }
+        __half2 a[4];
+        const __half2 mk = vec_abs_max(x[k], a);
+        if (THR && !fixed)
+            fresh |= __hge(__hmax(__low2half(mk), __high2half(mk)), q.t16);
+        rm = __hmax2(rm, mk);
+    }
+    if (THR && !fixed && __any_sync(0xffffffffu, fresh)) {
+        // columns new to this lane's cache: into the CTA's set, then the
+        // maximum again against the set read afresh
+#pragma unroll
+        for (int k = 0; k < kQsRegVec; ++k) {
+            __half2 a[4];
+            const __half2 mk = vec_abs_max(x[k], a);
+            if (__hge(__hmax(__low2half(mk), __high2half(mk)), q.t16))
+                pub |= qs_publish(x[k], q.lane + 32 * k, q.t16, q.s_bm, q.s_cnt, q.gset);
+        }
+        qs_load_set(sc, q.s_bm, q.nvec, q.lane, qs_count(q));
+        rm = __float2half2_rn(0.f);
+#pragma unroll
+        for (int k = 0; k < kQsRegVec; ++k) {
+            const uint32_t kb = (sc.b[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+            if (kb)
+                mask_known(x[k], kb);
+            __half2 a[4];
+            rm = __hmax2(rm, vec_abs_max(x[k], a));
+        }
+    }
+    if (THR && arrive)
+        qs_arrive_detected(pub);
+    const float amax = warp_max(fmaxf(__low2float(rm), __high2float(rm)));
+    const float s = qs_scale(amax);
+#pragma unroll
+    for (int k = 0; k < kQsRegVec; ++k) {
+        const int v = q.lane + 32 * k;
+        if (FULL || v < q.nvec)
+            *reinterpret_cast<uint2 *>(q.cr + (int64_t)v * 8) = codes8(x[k], s);
+    }
+    if (q.lane == 0)
+        *q.am = amax;
+    return (THR && !fixed) ? sc.count : 0;
+}
+
+// One longer row, read from shared memory in blocks of 8 vectors a lane
+// (three passes: detection, maximum, codes), the set read from bm directly.
 template <bool THR>
-__global__ void __launch_bounds__(256, 1)
+__device__ int qs_row_smem(const QsRow &q, bool detect, const uint32_t *bm, bool &pub, bool arrive)
+{
+    constexpr int U = 8;
+    int c = 0;
+    if (THR && detect) {
+        for (int b0 = 0; b0 < q.nvec; b0 += 32 * U) {
+            uint4 x[U];
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int v = b0 + q.lane + 32 * k;
+                x[k] = v < q.nvec ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int v = b0 + q.lane + 32 * k;
+                qs_detect_vec(q, v, x[k], v < q.nvec ? set_byte(q.s_bm, v) : 0xFFu, pub);
+            }
+        }
+    }
+    if (THR) {
+        c = qs_count(q);
+        if (arrive)
+            qs_arrive_detected(pub);
+    }
+    __half2 rm = __float2half2_rn(0.f);
+    for (int b0 = 0; b0 < q.nvec; b0 += 32 * U) {
+        uint4 x[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int v = b0 + q.lane + 32 * k;
+            x[k] = v < q.nvec ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int v = b0 + q.lane + 32 * k;
+            if (THR && v < q.nvec) {
+                const uint32_t sb = set_byte(bm, v);
+                if (sb)
+                    mask_known(x[k], sb);
+            }
+            __half2 a[4];
+            rm = __hmax2(rm, vec_abs_max(x[k], a));
+        }
+    }
+    const float amax = warp_max(fmaxf(__low2float(rm), __high2float(rm)));
+    const float s = qs_scale(amax);
+    for (int b0 = 0; b0 < q.nvec; b0 += 32 * U) {
+        uint4 x[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int v = b0 + q.lane + 32 * k;
+            x[k] = v < q.nvec ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int v = b0 + q.lane + 32 * k;
+            if (v < q.nvec) {
+                if (THR) {
+                    const uint32_t sb = set_byte(bm, v);
+                    if (sb)
+                        mask_known(x[k], sb);
+                }
+                *reinterpret_cast<uint2 *>(q.cr + (int64_t)v * 8) = codes8(x[k], s);
+            }
+        }
+    }
+    if (q.lane == 0)
+        *q.am = amax;
+    return c;
+}
+
+// REG: 0 the row is read from shared memory in blocks, 1 held in registers,
+// 2 held in registers and exactly 32 * kQsRegVec vectors long. reload: the
+// fixed final set bm (quantizing again after the grid barrier); detect:
+// run the detection step (the smem form; the register form always detects
+// unless reload).
+template <bool THR, int REG>
+__device__ __forceinline__ int qs_row(const QsRow &q, bool detect, const uint32_t *bm, QsSetCache &sc, bool reload,
+                                      bool &pub, bool arrive)
+{
+    if constexpr (REG == 2)
+        return qs_row_reg<THR, true>(q, sc, reload, pub, arrive);
+    else if constexpr (REG == 1)
+        return qs_row_reg<THR, false>(q, sc, reload, pub, arrive);
+    else
+        return qs_row_smem<THR>(q, detect, bm, pub, arrive);
+}
+
+template <bool THR, int REG>
+__global__ void __launch_bounds__(kQsThreads, 1)
     k_quant_smem(const uint4 *__restrict__ X, int rows, int cols, __half t16, int8_t *__restrict__ codes,
-                 float *__restrict__ absmax, uint32_t *__restrict__ bitmap_out, unsigned long long *tagged,
+                 float *__restrict__ absmax, uint32_t *__restrict__ bitmap_out, uint32_t *sets, uint32_t *calls,
                  int32_t *__restrict__ col_idx, int32_t *__restrict__ count, uint32_t *sync,
                  uint32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t q_smem[];
-    __shared__ uint64_t s_bar;
-    __shared__ int s_flag;
-    __shared__ uint32_t s_epoch;
+    __shared__ uint64_t s_bars[kQsMaxChunks];
+    __shared__ int s_cnt, s_gcount, s_fail, s_flag;
+    __shared__ uint32_t s_call;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nvec = cols >> 3, nwords = (cols + 31) >> 5;
     const int G = gridDim.x, c = blockIdx.x;
     const int r0 = (int)((int64_t)c * rows / G), r1 = (int)((int64_t)(c + 1) * rows / G);
     const int nr = r1 - r0;
+    const int rpc = qs_rows_per_chunk(max(nr, 1), cols);
+    const int nch = (nr + rpc - 1) / rpc;
     const uint4 *sx = reinterpret_cast<const uint4 *>(q_smem);
     const uint32_t xbytes = (uint32_t)nr * (uint32_t)cols * 2u;
-    uint32_t *s_bm = reinterpret_cast<uint32_t *>(q_smem + ((xbytes + 15u) & ~15u));
-    const uint32_t bar = smem_u32(&s_bar);
+    uint32_t *s_bm = reinterpret_cast<uint32_t *>(q_smem + ((xbytes + 15u) & ~15u)); // the CTA's set
+    uint32_t *s_gbm = s_bm + nwords;                                                  // the complete set
     griddep_release();
 
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        unsigned long long w;
-        asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(w) : "l"(sync) : "memory");
-        s_epoch = (uint32_t)(w >> 32);
-        s_flag = 1;
-    }
-    for (int w = tid; w < nwords; w += 256)
-        s_bm[w] = 0u;
-    __syncthreads();
-    if (tid == 0 && nr > 0) {
-        mbar_arrive_expect_tx(bar, xbytes);
-        const uint8_t *src = reinterpret_cast<const uint8_t *>(X + (int64_t)r0 * nvec);
-        for (uint32_t off = 0; off < xbytes; off += 32768u)
-            bulk_load(smem_u32(q_smem) + off, src + off, min(32768u, xbytes - off), bar);
-    }
-    const uint32_t epoch = s_epoch;
-    bool ok = true;
-    if (nr > 0)
-        ok = mbar_wait(bar, 0u);
-    if (THR && ok) {
-        for (int i = tid; i < nr * nvec; i += 256) {
-            const uint32_t h = hit_mask8(sx[i], t16);
-            if (h) {
-                const int vi = i % nvec;
-                atomicOr(&s_bm[vi >> 2], h << ((vi & 3) * 8));
+    if (warp == kQsWarps) {
+        // ------------------------------------------------ control warp
+        if (lane == 0) {
+            for (int j = 0; j < nch; ++j)
+                mbar_init(smem_u32(&s_bars[j]), 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            s_call = THR ? *reinterpret_cast<volatile uint32_t *>(calls) : 0u;
+            s_cnt = 0;
+            s_gcount = 0;
+            s_fail = 0;
+            s_flag = 1;
+        }
+        __syncwarp();
+        __syncthreads();
+        if (lane == 0) {
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(X + (int64_t)r0 * nvec);
+            for (int j = 0; j < nch; ++j) {
+                const uint32_t b0 = (uint32_t)(j * rpc) * (uint32_t)cols * 2u;
+                const uint32_t b1 = min(xbytes, (uint32_t)((j + 1) * rpc) * (uint32_t)cols * 2u);
+                const uint32_t bar = smem_u32(&s_bars[j]);
+                mbar_arrive_expect_tx(bar, b1 - b0);
+                for (uint32_t off = b0; off < b1; off += 32768u)
+                    bulk_load(smem_u32(q_smem) + off, src + off, min(32768u, b1 - off), bar);
             }
         }
-    }
-    __syncthreads();
-    if (THR && ok) {
-        for (int w = tid; w < nwords; w += 256) {
-            const uint32_t bits = s_bm[w];
-            if (bits && !tagged_or(tagged + w, epoch, bits))
-                ok = false;
-        }
-    }
-    if (!ok)
-        atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
-    __syncthreads();
-    if (tid == 0) {
-        s_flag = grid_barrier(sync, (uint32_t)G) ? 1 : 0;
-        if (!s_flag)
-            atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
-    }
-    __syncthreads();
-    if (!s_flag || !ok)
-        return;
-    if (THR) {
-        for (int w = tid; w < nwords; w += 256) {
-            const unsigned long long t = __ldcg(tagged + w);
-            s_bm[w] = ((uint32_t)(t >> 32) == epoch) ? (uint32_t)t : 0u;
-        }
-        __syncthreads();
-    }
-    for (int r = warp; r < nr; r += 8) {
-        const uint4 *xr = sx + (int64_t)r * nvec;
-        __half2 m2 = __float2half2_rn(0.f);
-        for (int vi = lane; vi < nvec; vi += 32) {
-            uint4 v = xr[vi];
-            const uint32_t kb = (s_bm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
-            if (kb)
-                mask_known(v, kb);
-            __half2 a[4];
-            m2 = __hmax2(m2, vec_abs_max(v, a));
-        }
-        float amax = fmaxf(__low2float(m2), __high2float(m2));
+        if (THR) {
+            named_barrier_sync(2, kQsThreads); // every row detected, its new columns in the global bitmap
+            bool passed = true;
+            if (lane == 0)
+                passed = grid_barrier(sync, (uint32_t)G);
+            passed = __shfl_sync(0xffffffffu, passed, 0);
+            const uint32_t *gset = sets + (s_call & 1u) * kSetWords;
+            int n = 0;
+            for (int w = lane; w < nwords; w += 32) {
+                const uint32_t g = __ldcg(gset + w);
+                s_gbm[w] = g;
+                n += __popc(g);
+            }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float s = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-        int8_t *cr = codes + (int64_t)(r0 + r) * cols;
-        for (int vi = lane; vi < nvec; vi += 32) {
-            uint4 v = xr[vi];
-            const uint32_t kb = (s_bm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
-            if (kb)
-                mask_known(v, kb);
-            *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) = codes8(v, s);
+            for (int o = 16; o > 0; o >>= 1)
+                n += __shfl_xor_sync(0xffffffffu, n, o);
+            if (lane == 0) {
+                s_gcount = n;
+                if (!passed)
+                    s_flag = 0;
+                if (c == 0) // every CTA read the counter before the barrier
+                    *reinterpret_cast<volatile uint32_t *>(calls) = s_call + 1u;
+            }
+            named_barrier_arrive(3, kQsThreads); // the complete set is in s_gbm
         }
-        if (lane == 0)
-            absmax[r0 + r] = amax;
+    } else {
+        // ------------------------------------------------ worker warps
+        for (int w = tid; w < nwords; w += kQsWorkers)
+            s_bm[w] = 0u;
+        __syncthreads();
+        if (THR && c == 0) { // the other bitmap, for the next call
+            uint32_t *next = sets + ((s_call + 1u) & 1u) * kSetWords;
+            for (int w = tid; w < (int)kSetWords; w += kQsWorkers)
+                next[w] = 0u;
+        }
+        QsRow q;
+        q.nvec = nvec;
+        q.t16 = t16;
+        q.s_bm = s_bm;
+        q.s_cnt = &s_cnt;
+        q.gset = sets + (s_call & 1u) * kSetWords;
+        q.lane = lane;
+        QsSetCache sc;
+        sc.count = -1;
+        bool ok = true, pub = false;
+        // seed: the first rows of the block, spread over every worker, are
+        // detected before any row is quantized
+        const int nseed = THR ? min(nr, kQsSeedRows) : 0;
+        if (THR) {
+            for (int j = 0; j * rpc < nseed; ++j)
+                if (!mbar_wait(smem_u32(&s_bars[j]), 0u))
+                    ok = false;
+            if (ok) {
+                const int n = nseed * nvec;
+                int i = tid, v = tid % nvec;
+                const int step = kQsWorkers % nvec;
+                for (; i < n; i += kQsWorkers) {
+                    qs_detect_vec(q, v, sx[i], set_byte(s_bm, v), pub);
+                    v += step;
+                    if (v >= nvec)
+                        v -= nvec;
+                }
+            }
+            named_barrier_sync(1, kQsWorkers);
+        }
+        int cmin = INT_MAX;
+        if (THR && warp >= nr)
+            qs_arrive_detected(pub); // no rows: nothing to detect
+        for (int r = warp; r < nr; r += kQsWarps) {
+            const bool last = r + kQsWarps >= nr;
+            if (!mbar_wait(smem_u32(&s_bars[r / rpc]), 0u)) {
+                ok = false;
+                if (THR && last)
+                    qs_arrive_detected(pub);
+                continue;
+            }
+            q.xr = sx + (int64_t)r * nvec;
+            q.cr = codes + (int64_t)(r0 + r) * cols;
+            q.am = absmax + r0 + r;
+            cmin = min(cmin, qs_row<THR, REG>(q, r >= nseed, s_bm, sc, false, pub, last));
+        }
+        if (THR) {
+            named_barrier_sync(3, kQsThreads);
+            if (s_flag && __all_sync(0xffffffffu, ok)) {
+                const int total = s_gcount;
+                if (cmin != INT_MAX && cmin != total) { // a row saw only part of the set: this warp's rows again
+                    if (REG)
+                        qs_load_set(sc, s_gbm, nvec, lane, total);
+                    for (int r = warp; r < nr; r += kQsWarps) {
+                        q.xr = sx + (int64_t)r * nvec;
+                        q.cr = codes + (int64_t)(r0 + r) * cols;
+                        q.am = absmax + r0 + r;
+                        qs_row<THR, REG>(q, false, s_gbm, sc, true, pub, false);
+                    }
+                }
+            }
+        }
+        if (!__all_sync(0xffffffffu, ok) && lane == 0)
+            s_fail = 1;
     }
+    __syncwarp();
+    __syncthreads();
+    if (tid == 0 && (s_fail || !s_flag))
+        atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
     if (c == 0) {
+        const uint32_t *fin = THR ? s_gbm : s_bm;
         if (bitmap_out)
-            for (int w = tid; w < nwords; w += 256)
-                bitmap_out[w] = s_bm[w];
+            for (int w = tid; w < nwords; w += kQsThreads)
+                bitmap_out[w] = fin[w];
         if (THR)
-            compact_block<256>(s_bm, nwords, col_idx, count);
+            compact_block<kQsThreads>(fin, nwords, col_idx, count);
         else if (tid == 0)
             *count = 0;
     }
@@ -727,8 +1052,9 @@ namespace {
 
 size_t quant_smem_bytes(int64_t rows, int64_t cols, int num_sms)
 {
+    // the block of rows, then the CTA's set and the complete set
     const int64_t per = (rows + num_sms - 1) / num_sms;
-    return (size_t)((per * cols * 2 + 15) & ~15ll) + (size_t)((cols + 31) / 32) * 4;
+    return (size_t)((per * cols * 2 + 15) & ~15ll) + (size_t)((cols + 31) / 32) * 8;
 }
 
 } // namespace
@@ -742,17 +1068,21 @@ bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev)
 }
 
 cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
-                                 uint32_t *bitmap_out, unsigned long long *tagged, int32_t *col_idx, int32_t *count,
-                                 uint32_t *sync, uint32_t *status, const DeviceInfo &dev, cudaStream_t stream)
+                                 uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls, int32_t *col_idx,
+                                 int32_t *count, uint32_t *sync, uint32_t *status, const DeviceInfo &dev,
+                                 cudaStream_t stream)
 {
     const bool thr = t > 0.f;
-    auto kern = thr ? k_quant_smem<true> : k_quant_smem<false>;
+    const int reg = cols / 8 == 32 * kQsRegVec ? 2 : cols / 8 < 32 * kQsRegVec ? 1 : 0;
+    auto kern = thr ? (reg == 2 ? k_quant_smem<true, 2> : reg == 1 ? k_quant_smem<true, 1> : k_quant_smem<true, 0>)
+                    : (reg == 2 ? k_quant_smem<false, 2>
+                                : reg == 1 ? k_quant_smem<false, 1> : k_quant_smem<false, 0>);
     const size_t smem = quant_smem_bytes(rows, cols, dev.num_sms);
     static std::mutex mu;
-    static std::map<std::pair<int, int>, size_t> configured; // (device, thr) -> bytes set
+    static std::map<std::pair<int, int>, size_t> configured; // (device, variant) -> bytes set
     {
         std::lock_guard<std::mutex> lock(mu);
-        size_t &have = configured[std::make_pair(dev.device, thr ? 1 : 0)];
+        size_t &have = configured[std::make_pair(dev.device, (thr ? 1 : 0) + 2 * reg)];
         if (have < smem) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  dev.max_smem_optin - 1024);
@@ -763,7 +1093,7 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)dev.num_sms);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(kQsThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -772,7 +1102,7 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const uint4 *>(X), (int)rows, (int)cols,
-                              threshold_fp16(t), codes, absmax, bitmap_out, tagged, col_idx, count, sync, status);
+                              threshold_fp16(t), codes, absmax, bitmap_out, sets, calls, col_idx, count, sync, status);
 }
 
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

@@ -179,6 +179,81 @@ def test_quantize_late_outlier_column(lib, dev, oracle_mod):
     assert np.array_equal(codes.cpu().numpy(), c_ref)
 
 
+@pytest.mark.parametrize("M,K,rows_hit", [
+    (4096, 4096, [4095]),        # only the last chunk of the last CTA sees it
+    (4096, 4096, [7 * 28 + 5]),  # mid-block of one CTA: its earlier chunks and every other CTA are stale
+    (1000, 2064, [0, 999]),      # ragged rows per CTA, a partial bitmap word
+    (150, 4096, [149]),          # about one row per CTA
+])
+def test_quantize_resident_stale_chunks(lib, dev, oracle_mod, M, K, rows_hit):
+    """Shapes that fit the shared-memory quantizer, with an outlier column
+    that only a few rows cross (the other rows take their maximum, 5.5, in
+    it). Chunks quantized before the column was known must be quantized again
+    against the complete set: the result is still the definition's."""
+    X = np.random.default_rng(11).standard_normal((M, K)).astype(np.float32)
+    X[:, 37] *= 0.1
+    X[:, 37] += 5.5 * (np.arange(M) % 3 == 0)
+    for r in rows_hit:
+        X[r, 37] = 40.0
+    X[:, 1000 % K] *= 30.0  # a column every chunk sees
+    X16 = X.astype(np.float16)
+    codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
+    mask = oracle_mod.outlier_mask(X16, 6.0)
+    assert mask[37]
+    c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+@pytest.mark.parametrize("M,K", [(5000, 16), (777, 32), (40, 48), (3, 57344), (148 * 13, 4112)])
+def test_quantize_resident_odd_shapes(lib, dev, oracle_mod, M, K):
+    """Narrow rows (a vector or two per row, many rows per chunk), a few very
+    long rows, and a ragged width, with and without the threshold."""
+    X16 = make_random((M, K), seed=M + K, scale=2.0)
+    X16[M // 2, K - 1] = 9.0
+    for t in (6.0, 0.0):
+        codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), t)
+        mask = oracle_mod.outlier_mask(X16, t) if t > 0 else np.zeros(K, np.uint8)
+        c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+        if t > 0:
+            assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
+        assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
+        assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_workspace_shared_across_shapes(lib, dev, oracle_mod):
+    """One workspace for calls of several shapes and entry points, in an order
+    that leaves other regions' data (codes, column lists) where a later shape
+    keeps its outlier bookkeeping: every result is still the definition's."""
+    shapes = [(64, 4096), (300, 1040), (2000, 256), (64, 4096), (1000, 2064), (4096, 4096), (64, 4096)]
+    nbytes = max(max(lib.workspace_size(M, 512, K), lib.quantize_workspace_size(M, K)) for M, K in shapes)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    lib.workspace_init(ws)
+    for i, (M, K) in enumerate(shapes):
+        lin = Linear("ws", M, 512, K, 3 + i % 3, 50.0)
+        X16, _ = make_activations(lin, seed=100 + i)
+        X = to_dev(X16, dev)
+        mask = oracle_mod.outlier_mask(X16, 6.0)
+        c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
+        codes, absmax, bm = lib.quantize_rowwise(X, 6.0, workspace=ws)
+        assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask), (M, K)
+        assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32)), (M, K)
+        assert np.array_equal(codes.cpu().numpy(), c_ref), (M, K)
+        if M <= 2000:  # and a matmul on the same workspace, its codes checked through the debug outputs
+            W16 = make_weight(lin, seed=i)
+            W = to_dev(W16, dev)
+            CB, SCB, _ = lib.quantize_rowwise(W, 0.0, workspace=ws)
+            dbg = dict(codes=torch.empty((M, K), dtype=torch.int8, device=dev),
+                       row_absmax=torch.empty(M, dtype=torch.float32, device=dev),
+                       col_idx=torch.empty(K, dtype=torch.int32, device=dev),
+                       count=torch.empty(1, dtype=torch.int32, device=dev))
+            lib.matmul_mixed(X, CB, SCB, W, 6.0, workspace=ws, debug=dbg)
+            n = int(dbg["count"].item())
+            assert np.array_equal(dbg["col_idx"][:n].cpu().numpy(), np.flatnonzero(mask)), (M, K)
+            assert np.array_equal(dbg["codes"].cpu().numpy(), c_ref), (M, K)
+
+
 def test_quantize_row_of_outliers(lib, dev, oracle_mod):
     """One row >= t everywhere makes every column an outlier: all codes 0,
     every absmax 0 (the int8 part is empty)."""
