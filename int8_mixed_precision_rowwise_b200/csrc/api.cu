@@ -199,8 +199,8 @@ llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t
         return LLMINT8_ERR_CUDA;
     if (quantize_smem_fits(rows, cols, dev)) {
         // X fits in shared memory: one kernel, nothing to clear first.
-        e = launch_quantize_smem(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.sets, ws.calls, ws.col_idx,
-                                 ws.count, ws.sync, ws.status, dev, stream);
+        e = launch_quantize_smem(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, ws.sets, ws.calls,
+                                 ws.arrivals, ws.col_idx, ws.count, ws.status, dev, stream);
         return cuda_status(e);
     }
     // The streaming quantizer ORs into the caller's bitmap: clear it. (Its
@@ -301,8 +301,8 @@ llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, 
 
     if (quantize_smem_fits(M, K, dev)) {
         // X fits in shared memory: one kernel, nothing to clear first.
-        if ((e = launch_quantize_smem(X_f16, M, K, t, ws.cx, ws.sx, nullptr, ws.sets, ws.calls, ws.col_idx, ws.count,
-                                      ws.sync, ws.status, dev, stream)) != cudaSuccess)
+        if ((e = launch_quantize_smem(X_f16, M, K, t, ws.cx, ws.sx, nullptr, ws.sets, ws.calls, ws.arrivals,
+                                      ws.col_idx, ws.count, ws.status, dev, stream)) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
     } else {
         // The streaming quantizer ORs into the bitmap: clear it. (Its other

@@ -25,6 +25,8 @@ constexpr size_t kSetWords = (LLMINT8_MAX_K + 31) / 32; // bitmap words of the w
 //            half); never cleared by the library after workspace_init
 //   [16]     uint32 late-outlier flag, [20] decode outlier-list flag
 //   [24]     uint32 calls of the shared-memory quantizer so far
+//   [32]     uint64 arrivals at the shared-memory quantizer's grid barrier so
+//            far (one per CTA per call: a multiple of the grid between calls)
 //   [256]    uint32 two outlier bitmaps [2][kSetWords] of the shared-memory
 //            quantizer: call n ORs into set[n & 1] and clears set[(n+1) & 1]
 //            for the next call. Their place and size depend on no shape, so
@@ -47,6 +49,7 @@ struct Workspace {
     uint32_t *bitmap;
     uint32_t *sets;   // [2][kSetWords]
     uint32_t *calls;
+    unsigned long long *arrivals;
     int32_t *col_idx;
     float *sx;
     int8_t *cx;
@@ -90,6 +93,7 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
         ws->bitmap = reinterpret_cast<uint32_t *>(bm);
         ws->sets = reinterpret_cast<uint32_t *>(tg);
         ws->calls = hdr ? reinterpret_cast<uint32_t *>(hdr + 24) : nullptr;
+        ws->arrivals = hdr ? reinterpret_cast<unsigned long long *>(hdr + 32) : nullptr;
         ws->col_idx = reinterpret_cast<int32_t *>(ci);
         ws->sx = reinterpret_cast<float *>(sx);
         ws->cx = reinterpret_cast<int8_t *>(cx);
@@ -126,14 +130,15 @@ __half threshold_fp16(float t);
 
 // The quantizer for an X whose rows fit in the shared memory of one CTA per
 // SM (one read of X, one grid barrier, nothing to clear before the call):
-// `sets`/`calls` are the workspace's two bitmaps and call counter,
+// `sets`/`calls`/`arrivals` are the workspace's two bitmaps, call counter and
+// barrier arrival counter,
 // bitmap_out (may be null) receives the outlier bitmap, col_idx/count the
 // ascending outlier columns.
 bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev);
 cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
-                                 uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls, int32_t *col_idx,
-                                 int32_t *count, uint32_t *sync, uint32_t *status, const DeviceInfo &dev,
-                                 cudaStream_t stream);
+                                 uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls,
+                                 unsigned long long *arrivals, int32_t *col_idx, int32_t *count,
+                                 uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
 
 // Bitmap -> ascending column list and count (one CTA).
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,

@@ -536,15 +536,19 @@ cudaError_t launch_fused_v(const void *X, int64_t rows, int cols, float t, int8_
                                                      status, dev, stream);
 }
 
-// The quantizer for an X that fits in the shared memory of one CTA per SM.
-// Each CTA holds its block of rows (contiguous in X) for the whole call. The
-// block arrives as chunks of whole rows, each bulk-copied into shared memory
-// on an mbarrier of its own, and each of 15 worker warps takes rows
-// w, w + 15, ... as they land. Per row (threshold on):
+// The quantizer for an X that fits in the shared memory of one CTA per SM,
+// with rows of up to 4096 columns. Each CTA holds its block of rows
+// (contiguous in X) for the whole call. The block arrives as chunks of whole
+// rows, each bulk-copied into shared memory on an mbarrier of its own (a few
+// chunks in flight at a time), and each of 15 worker warps takes rows
+// w, w + 15, ... as they land, a row in the warp's registers. Per row
+// (threshold on):
 //   detect - the row's outlier columns (|x| >= t16) join the CTA's set s_bm;
 //            a column new to it is also ORed (fire and forget) into this
 //            call's global bitmap, and then counted in s_cnt;
-//   c      - the size of the CTA's set, read after the detection;
+//   c      - the size of the set the row is quantized against: each lane
+//            caches the set bytes of its vectors, read after reading c, and
+//            reads them again when s_cnt has moved or the row added to it;
 //   row    - maximum over the columns outside the set, codes
 //            rint(x * 127 / absmax) (set columns 0) and absmax.
 // A control warp, once every row is detected, passes the grid barrier and
@@ -566,6 +570,7 @@ constexpr int kQsThreads = kQsWorkers + 32;     // + the control warp
 constexpr int kQsMaxChunks = 64;
 constexpr int kQsChunkBytes = 4096;
 constexpr int kQsSeedRows = 4;
+constexpr int kQsInFlight = 8;                  // chunks of one CTA requested ahead
 constexpr int kQsRegVec = 16;                   // rows of up to 32 * 16 vectors stay in registers
 
 // Rows of one CTA per chunk: at least kQsChunkBytes, at most kQsMaxChunks chunks.
@@ -604,9 +609,9 @@ __device__ __noinline__ bool qs_publish(uint4 x, int v, __half t16, uint32_t *s_
     const uint32_t nb = bits & ~atomicOr(&s_bm[w], bits);
     if (!nb)
         return false;
-    atomicOr(gset + w, nb);
     __threadfence_block(); // the bits are in s_bm before the count says so
     atomicAdd(s_cnt, __popc(nb));
+    atomicOr(gset + w, nb); // after the fence: it would wait for this one to land
     return true;
 }
 
@@ -702,7 +707,6 @@ __device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub,
             qs_load_set(sc, q.s_bm, q.nvec, q.lane, qs_count(q));
     }
     __half2 rm = __float2half2_rn(0.f);
-    bool fresh = false;
 #pragma unroll
     for (int k = 0; k < kQsRegVec; ++k) {
         if (THR) {
@@ -711,12 +715,11 @@ __device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub,
                 mask_known(x[k], kb);
         }
         __half2 a[4];
-        const __half2 mk = vec_abs_max(x[k], a);
-        if (THR && !fixed)
-            fresh |= __hge(__hmax(__low2half(mk), __high2half(mk)), q.t16);
-        rm = __hmax2(rm, mk);
+        rm = __hmax2(rm, vec_abs_max(x[k], a));
     }
-    if (THR && !fixed && __any_sync(0xffffffffu, fresh)) {
+    // The maximum over the columns left reaches t16 exactly when one of
+    // them is an outlier column the cache did not have.
+    if (THR && !fixed && __any_sync(0xffffffffu, __hge(__hmax(__low2half(rm), __high2half(rm)), q.t16))) {
         // columns new to this lane's cache: into the CTA's set, then the
         // maximum again against the set read afresh
 #pragma unroll
@@ -752,108 +755,18 @@ __device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub,
     return (THR && !fixed) ? sc.count : 0;
 }
 
-// One longer row, read from shared memory in blocks of 8 vectors a lane
-// (three passes: detection, maximum, codes), the set read from bm directly.
-template <bool THR>
-__device__ int qs_row_smem(const QsRow &q, bool detect, const uint32_t *bm, bool &pub, bool arrive)
-{
-    constexpr int U = 8;
-    int c = 0;
-    if (THR && detect) {
-        for (int b0 = 0; b0 < q.nvec; b0 += 32 * U) {
-            uint4 x[U];
-#pragma unroll
-            for (int k = 0; k < U; ++k) {
-                const int v = b0 + q.lane + 32 * k;
-                x[k] = v < q.nvec ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int k = 0; k < U; ++k) {
-                const int v = b0 + q.lane + 32 * k;
-                qs_detect_vec(q, v, x[k], v < q.nvec ? set_byte(q.s_bm, v) : 0xFFu, pub);
-            }
-        }
-    }
-    if (THR) {
-        c = qs_count(q);
-        if (arrive)
-            qs_arrive_detected(pub);
-    }
-    __half2 rm = __float2half2_rn(0.f);
-    for (int b0 = 0; b0 < q.nvec; b0 += 32 * U) {
-        uint4 x[U];
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const int v = b0 + q.lane + 32 * k;
-            x[k] = v < q.nvec ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const int v = b0 + q.lane + 32 * k;
-            if (THR && v < q.nvec) {
-                const uint32_t sb = set_byte(bm, v);
-                if (sb)
-                    mask_known(x[k], sb);
-            }
-            __half2 a[4];
-            rm = __hmax2(rm, vec_abs_max(x[k], a));
-        }
-    }
-    const float amax = warp_max(fmaxf(__low2float(rm), __high2float(rm)));
-    const float s = qs_scale(amax);
-    for (int b0 = 0; b0 < q.nvec; b0 += 32 * U) {
-        uint4 x[U];
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const int v = b0 + q.lane + 32 * k;
-            x[k] = v < q.nvec ? q.xr[v] : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const int v = b0 + q.lane + 32 * k;
-            if (v < q.nvec) {
-                if (THR) {
-                    const uint32_t sb = set_byte(bm, v);
-                    if (sb)
-                        mask_known(x[k], sb);
-                }
-                *reinterpret_cast<uint2 *>(q.cr + (int64_t)v * 8) = codes8(x[k], s);
-            }
-        }
-    }
-    if (q.lane == 0)
-        *q.am = amax;
-    return c;
-}
-
-// REG: 0 the row is read from shared memory in blocks, 1 held in registers,
-// 2 held in registers and exactly 32 * kQsRegVec vectors long. reload: the
-// fixed final set bm (quantizing again after the grid barrier); detect:
-// run the detection step (the smem form; the register form always detects
-// unless reload).
-template <bool THR, int REG>
-__device__ __forceinline__ int qs_row(const QsRow &q, bool detect, const uint32_t *bm, QsSetCache &sc, bool reload,
-                                      bool &pub, bool arrive)
-{
-    if constexpr (REG == 2)
-        return qs_row_reg<THR, true>(q, sc, reload, pub, arrive);
-    else if constexpr (REG == 1)
-        return qs_row_reg<THR, false>(q, sc, reload, pub, arrive);
-    else
-        return qs_row_smem<THR>(q, detect, bm, pub, arrive);
-}
-
-template <bool THR, int REG>
+template <bool THR, bool FULL>
 __global__ void __launch_bounds__(kQsThreads, 1)
     k_quant_smem(const uint4 *__restrict__ X, int rows, int cols, __half t16, int8_t *__restrict__ codes,
                  float *__restrict__ absmax, uint32_t *__restrict__ bitmap_out, uint32_t *sets, uint32_t *calls,
-                 int32_t *__restrict__ col_idx, int32_t *__restrict__ count, uint32_t *sync,
+                 unsigned long long *arrivals, int32_t *__restrict__ col_idx, int32_t *__restrict__ count,
                  uint32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t q_smem[];
     __shared__ uint64_t s_bars[kQsMaxChunks];
     __shared__ int s_cnt, s_gcount, s_fail, s_flag;
     __shared__ uint32_t s_call;
+    __shared__ unsigned long long s_target;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nvec = cols >> 3, nwords = (cols + 31) >> 5;
     const int G = gridDim.x, c = blockIdx.x;
@@ -874,6 +787,13 @@ __global__ void __launch_bounds__(kQsThreads, 1)
                 mbar_init(smem_u32(&s_bars[j]), 1);
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
             s_call = THR ? *reinterpret_cast<volatile uint32_t *>(calls) : 0u;
+            if (THR) {
+                // This call's barrier opens when the count reaches the next
+                // multiple of the grid (CTAs that arrived already are below it).
+                unsigned long long a;
+                asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(a) : "l"(arrivals) : "memory");
+                s_target = a - a % (unsigned long long)G + (unsigned long long)G;
+            }
             s_cnt = 0;
             s_gcount = 0;
             s_fail = 0;
@@ -882,21 +802,48 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         __syncwarp();
         __syncthreads();
         if (lane == 0) {
+            // At most kQsInFlight chunks of this CTA in flight: the next is
+            // requested when the oldest lands, so that every CTA's rows
+            // arrive as a steady stream from the start (with all of them
+            // requested at once, the order HBM serves them in left some
+            // CTAs without their first rows until most of X had arrived).
             const uint8_t *src = reinterpret_cast<const uint8_t *>(X + (int64_t)r0 * nvec);
-            for (int j = 0; j < nch; ++j) {
+            auto issue = [&](int j) {
                 const uint32_t b0 = (uint32_t)(j * rpc) * (uint32_t)cols * 2u;
                 const uint32_t b1 = min(xbytes, (uint32_t)((j + 1) * rpc) * (uint32_t)cols * 2u);
                 const uint32_t bar = smem_u32(&s_bars[j]);
                 mbar_arrive_expect_tx(bar, b1 - b0);
                 for (uint32_t off = b0; off < b1; off += 32768u)
                     bulk_load(smem_u32(q_smem) + off, src + off, min(32768u, b1 - off), bar);
+            };
+            for (int j = 0; j < min(nch, kQsInFlight); ++j)
+                issue(j);
+            for (int j = kQsInFlight; j < nch; ++j) {
+                if (!mbar_wait(smem_u32(&s_bars[j - kQsInFlight]), 0u))
+                    s_fail = 1; // the workers' wait on that chunk fails too
+                issue(j);
             }
         }
         if (THR) {
             named_barrier_sync(2, kQsThreads); // every row detected, its new columns in the global bitmap
             bool passed = true;
-            if (lane == 0)
-                passed = grid_barrier(sync, (uint32_t)G);
+            if (lane == 0) {
+                // Grid barrier: one posted add per CTA (release: the CTA's
+                // bits, made visible by its workers' fences, come first),
+                // then wait for the count to reach this call's target.
+                asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(arrivals) : "memory");
+                const uint64_t t0 = global_timer_ns();
+                for (;;) {
+                    unsigned long long a;
+                    asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(a) : "l"(arrivals) : "memory");
+                    if ((long long)(a - s_target) >= 0)
+                        break;
+                    if (global_timer_ns() - t0 > kWaitLimitNs) {
+                        passed = false;
+                        break;
+                    }
+                }
+            }
             passed = __shfl_sync(0xffffffffu, passed, 0);
             const uint32_t *gset = sets + (s_call & 1u) * kSetWords;
             int n = 0;
@@ -971,20 +918,19 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             q.xr = sx + (int64_t)r * nvec;
             q.cr = codes + (int64_t)(r0 + r) * cols;
             q.am = absmax + r0 + r;
-            cmin = min(cmin, qs_row<THR, REG>(q, r >= nseed, s_bm, sc, false, pub, last));
+            cmin = min(cmin, qs_row_reg<THR, FULL>(q, sc, false, pub, last));
         }
         if (THR) {
             named_barrier_sync(3, kQsThreads);
             if (s_flag && __all_sync(0xffffffffu, ok)) {
                 const int total = s_gcount;
                 if (cmin != INT_MAX && cmin != total) { // a row saw only part of the set: this warp's rows again
-                    if (REG)
-                        qs_load_set(sc, s_gbm, nvec, lane, total);
+                    qs_load_set(sc, s_gbm, nvec, lane, total);
                     for (int r = warp; r < nr; r += kQsWarps) {
                         q.xr = sx + (int64_t)r * nvec;
                         q.cr = codes + (int64_t)(r0 + r) * cols;
                         q.am = absmax + r0 + r;
-                        qs_row<THR, REG>(q, false, s_gbm, sc, true, pub, false);
+                        qs_row_reg<THR, FULL>(q, sc, true, pub, false);
                     }
                 }
             }
@@ -1061,28 +1007,29 @@ size_t quant_smem_bytes(int64_t rows, int64_t cols, int num_sms)
 
 bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev)
 {
-    // Room for the block of rows and the bitmap, under the opt-in limit with
-    // a margin for the kernel's static shared memory.
-    return rows >= 1 && cols >= 8 && cols % 8 == 0 && rows <= INT32_MAX &&
+    // Rows that a warp holds in registers, and room for the block of rows and
+    // the two bitmaps under the opt-in limit, with a margin for the kernel's
+    // static shared memory. (Longer rows go to the streaming quantizer, which
+    // keeps a row of up to 65536 columns in the registers of one CTA.)
+    return rows >= 1 && cols >= 8 && cols % 8 == 0 && cols <= 8 * 32 * kQsRegVec && rows <= INT32_MAX &&
            quant_smem_bytes(rows, cols, dev.num_sms) + 2048 <= (size_t)dev.max_smem_optin;
 }
 
 cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
-                                 uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls, int32_t *col_idx,
-                                 int32_t *count, uint32_t *sync, uint32_t *status, const DeviceInfo &dev,
-                                 cudaStream_t stream)
+                                 uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls,
+                                 unsigned long long *arrivals, int32_t *col_idx, int32_t *count,
+                                 uint32_t *status, const DeviceInfo &dev, cudaStream_t stream)
 {
     const bool thr = t > 0.f;
-    const int reg = cols / 8 == 32 * kQsRegVec ? 2 : cols / 8 < 32 * kQsRegVec ? 1 : 0;
-    auto kern = thr ? (reg == 2 ? k_quant_smem<true, 2> : reg == 1 ? k_quant_smem<true, 1> : k_quant_smem<true, 0>)
-                    : (reg == 2 ? k_quant_smem<false, 2>
-                                : reg == 1 ? k_quant_smem<false, 1> : k_quant_smem<false, 0>);
+    const bool full = cols / 8 == 32 * kQsRegVec;
+    auto kern = thr ? (full ? k_quant_smem<true, true> : k_quant_smem<true, false>)
+                    : (full ? k_quant_smem<false, true> : k_quant_smem<false, false>);
     const size_t smem = quant_smem_bytes(rows, cols, dev.num_sms);
     static std::mutex mu;
     static std::map<std::pair<int, int>, size_t> configured; // (device, variant) -> bytes set
     {
         std::lock_guard<std::mutex> lock(mu);
-        size_t &have = configured[std::make_pair(dev.device, (thr ? 1 : 0) + 2 * reg)];
+        size_t &have = configured[std::make_pair(dev.device, (thr ? 1 : 0) + (full ? 2 : 0))];
         if (have < smem) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  dev.max_smem_optin - 1024);
@@ -1102,7 +1049,7 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const uint4 *>(X), (int)rows, (int)cols,
-                              threshold_fp16(t), codes, absmax, bitmap_out, sets, calls, col_idx, count, sync, status);
+                              threshold_fp16(t), codes, absmax, bitmap_out, sets, calls, arrivals, col_idx, count, status);
 }
 
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,
