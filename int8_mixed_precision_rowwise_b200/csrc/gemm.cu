@@ -68,7 +68,8 @@ struct Smem {
     static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
     static constexpr int SIDE_OFF = B_OFF + STAGES * B_BYTES;          // float [OC][BN]
     static constexpr int SCALE_OFF = SIDE_OFF + OC * BN * 4;           // float [BN]
-    static constexpr int BAR_OFF = SCALE_OFF + BN * 4;                 // uint64 barriers
+    static constexpr int COLS_OFF = SCALE_OFF + BN * 4;                // int [OC] outlier columns
+    static constexpr int BAR_OFF = COLS_OFF + OC * 4;                  // uint64 barriers
     static constexpr int NBARS = 2 * STAGES + 5;                       // full, empty, tfull[2], tempty[2], drain
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;               // tmem base, abort flag
     static constexpr int BYTES = MISC_OFF + 16;
@@ -101,8 +102,65 @@ __device__ __forceinline__ void report(const KParams &p, volatile int *s_abort, 
 // issuer. Tiles are first_tile, first_tile + tile_step, ...; this CTA's
 // accumulator rows are a_row_off .. a_row_off + 127 of each a_tile_rows-row
 // A tile.
+// One tile's staging loads held in registers as they arrive (raw: no
+// arithmetic on them, so issuing them does not wait for them): the scales of
+// the thread's entries of s_scale, its row's SX and outlier values of X, and
+// up to 2 x 128 x 8 gathered outlier values of W (fp16 bits, or the int8
+// code and its row's SB).
+constexpr int kPipeCols = 8;   // outlier columns the pipelined staging covers
+constexpr int kPipeGather = 16; // gathers per thread it covers
+template <int BN>
+struct StageRegs {
+    float sc[(BN + 127) / 128];
+    float own_scale;
+    uint32_t own_side[kPipeCols]; // fp16 bits of X[i, col_k]
+    uint32_t g[kPipeGather];      // fp16 bits of W[r, col] or the int8 code of CB[r, col]
+    float gsb[kPipeGather];       // SB[r] (code form only)
+};
+
+template <int BN>
+__device__ __forceinline__ void stage_issue(const KParams &p, const int *s_cols, int cnt, int tile, int a_tile_rows,
+                                            int a_row_off, int r_in_tile, int et, StageRegs<BN> &st)
+{
+    const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
+    const int arow = mb * a_tile_rows + a_row_off + r_in_tile;
+    const int brow0 = nb * BN;
+#pragma unroll
+    for (int u = 0; u < (BN + 127) / 128; ++u) {
+        const int idx = et + u * 128, r = brow0 + idx;
+        st.sc[u] = (idx < BN && r < p.N) ? p.sb[r] : 0.f;
+    }
+    st.own_scale = arow < p.M ? p.sx[arow] : 0.f;
+    const unsigned short *x16 = reinterpret_cast<const unsigned short *>(p.X16);
+#pragma unroll
+    for (int k = 0; k < kPipeCols; ++k)
+        st.own_side[k] = (k < cnt && arow < p.M) ? x16[(int64_t)arow * p.K + s_cols[k]] : 0u;
+    const unsigned short *w16 = reinterpret_cast<const unsigned short *>(p.W16);
+#pragma unroll
+    for (int u = 0; u < kPipeGather; ++u) {
+        const int idx = u * 128 + et;
+        uint32_t v = 0u;
+        float sbv = 0.f;
+        if (idx < cnt * BN) {
+            const int k = idx / BN, r = brow0 + (idx - k * BN);
+            if (r < p.N) {
+                const int64_t off = (int64_t)r * p.K + s_cols[k];
+                if (p.W16) {
+                    v = w16[off];
+                } else {
+                    v = (uint32_t)(uint8_t)p.CB[off];
+                    sbv = p.sb[r];
+                }
+            }
+        }
+        st.g[u] = v;
+        st.gsb[u] = sbv;
+    }
+}
+
 template <int BN, bool SWAP, bool RAW, bool PAIR>
 __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lane, float *s_side, float *s_scale,
+                                             int *s_cols,
                                              uint32_t tfull0, uint32_t tempty0, volatile int *s_abort,
                                              uint32_t tmem_base, int first_tile, int tile_step, int num_tiles,
                                              int a_tile_rows, int a_row_off)
@@ -114,8 +172,21 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
     const int r_in_tile = q * 32 + lane;    // accumulator row (A-side row in the tile)
     const int cnt = RAW ? 0 : min(*p.count, p.K);
     const bool fast = cnt <= OC;
+    if (!RAW && fast) {
+        // The outlier columns, the same for every tile, once into shared memory.
+        for (int k = et; k < cnt; k += 128)
+            s_cols[k] = p.col_idx[k];
+        named_barrier_sync(1, 128);
+    }
     uint32_t tph[2] = {0u, 0u};
     int local = 0;
+    // Few outlier columns: the next tile's staging loads go out before this
+    // tile's epilogue and land while it runs (under the TMA stream a round of
+    // them takes several microseconds, longer than a K = 4096 tile's MMAs).
+    const bool pipe = !RAW && !SWAP && fast && cnt <= kPipeCols && cnt * BN <= kPipeGather * 128;
+    StageRegs<BN> nx;
+    if (pipe && first_tile < num_tiles)
+        stage_issue<BN>(p, s_cols, cnt, first_tile, a_tile_rows, a_row_off, r_in_tile, et, nx);
     for (int tile = first_tile; tile < num_tiles; tile += tile_step, ++local) {
         const int b = local & 1;
         const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
@@ -126,12 +197,63 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
 #pragma unroll
         for (int k = 0; k < OC; ++k)
             own_side[k] = 0.f;
-        if (!RAW) {
-            // Stage the outlier operands and scales while the MMAs run.
+        if (pipe) {
+            named_barrier_sync(1, 128); // the previous tile's readers are done with s_side / s_scale
+#pragma unroll
+            for (int u = 0; u < (BN + 127) / 128; ++u)
+                if (et + u * 128 < BN)
+                    s_scale[et + u * 128] = nx.sc[u];
+#pragma unroll
+            for (int u = 0; u < kPipeGather; ++u) {
+                const int idx = u * 128 + et;
+                if (idx < cnt * BN)
+                    s_side[idx] = p.W16 ? __half2float(__ushort_as_half((unsigned short)nx.g[u]))
+                                        : __fdiv_rn(__fmul_rn((float)(int8_t)(uint8_t)nx.g[u], nx.gsb[u]), 127.0f);
+            }
+            own_scale = nx.own_scale;
+#pragma unroll
+            for (int k = 0; k < kPipeCols; ++k)
+                own_side[k] = __half2float(__ushort_as_half((unsigned short)nx.own_side[k]));
             named_barrier_sync(1, 128);
-            for (int idx = et; idx < BN; idx += 128) {
-                const int r = brow0 + idx;
-                s_scale[idx] = SWAP ? (r < p.M ? p.sx[r] : 0.f) : (r < p.N ? p.sb[r] : 0.f);
+            if (tile + tile_step < num_tiles)
+                stage_issue<BN>(p, s_cols, cnt, tile + tile_step, a_tile_rows, a_row_off, r_in_tile, et, nx);
+        } else if (!RAW) {
+            // Stage the tile's scales and outlier operands while the MMAs run.
+            // Every load of the first round goes out before any is used (with
+            // the column list in shared memory, nothing here waits on a load
+            // to find its address): under the TMA stream each global round
+            // trip costs a microsecond or more, and at K = 4096 a tile's MMAs
+            // last only about 10 us.
+            named_barrier_sync(1, 128);
+            constexpr int NSC = (BN + 127) / 128;
+            float sc[NSC];
+#pragma unroll
+            for (int u = 0; u < NSC; ++u) {
+                const int idx = et + u * 128, r = brow0 + idx;
+                sc[u] = 0.f;
+                if (idx < BN)
+                    sc[u] = SWAP ? (r < p.M ? p.sx[r] : 0.f) : (r < p.N ? p.sb[r] : 0.f);
+            }
+            if (SWAP) {
+                if (arow < p.N) {
+                    own_scale = p.sb[arow];
+                    if (fast) {
+#pragma unroll
+                        for (int k = 0; k < OC; ++k)
+                            if (k < cnt)
+                                own_side[k] = wtilde(p, arow, s_cols[k]);
+                    }
+                }
+            } else {
+                if (arow < p.M) {
+                    own_scale = p.sx[arow];
+                    if (fast) {
+#pragma unroll
+                        for (int k = 0; k < OC; ++k)
+                            if (k < cnt)
+                                own_side[k] = __half2float(p.X16[(int64_t)arow * p.K + s_cols[k]]);
+                    }
+                }
             }
             if (fast) {
                 // Eight independent gathers in flight per thread, then the stores.
@@ -144,7 +266,7 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                         if (idx < cnt * BN) {
                             const int k = idx / BN, c = idx - k * BN;
                             const int r = brow0 + c;
-                            const int col = p.col_idx[k];
+                            const int col = s_cols[k];
                             if (SWAP) {
                                 if (r < p.M)
                                     v = __half2float(p.X16[(int64_t)r * p.K + col]);
@@ -163,27 +285,10 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                     }
                 }
             }
-            if (SWAP) {
-                if (arow < p.N) {
-                    own_scale = p.sb[arow];
-                    if (fast) {
 #pragma unroll
-                        for (int k = 0; k < OC; ++k)
-                            if (k < cnt)
-                                own_side[k] = wtilde(p, arow, p.col_idx[k]);
-                    }
-                }
-            } else {
-                if (arow < p.M) {
-                    own_scale = p.sx[arow];
-                    if (fast) {
-#pragma unroll
-                        for (int k = 0; k < OC; ++k)
-                            if (k < cnt)
-                                own_side[k] = __half2float(p.X16[(int64_t)arow * p.K + p.col_idx[k]]);
-                    }
-                }
-            }
+            for (int u = 0; u < NSC; ++u)
+                if (et + u * 128 < BN)
+                    s_scale[et + u * 128] = sc[u];
             named_barrier_sync(1, 128);
         }
 
@@ -383,6 +488,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float *s_side = reinterpret_cast<float *>(smem + L::SIDE_OFF);
     float *s_scale = reinterpret_cast<float *>(smem + L::SCALE_OFF);
+    int *s_cols = reinterpret_cast<int *>(smem + L::COLS_OFF);
     const uint32_t bar0 = sbase + L::BAR_OFF;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -536,7 +642,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
-        run_epilogue<BN, SWAP, RAW, false>(p, warp, lane, s_side, s_scale, tfull_bar(0), tempty_bar(0), s_abort,
+        run_epilogue<BN, SWAP, RAW, false>(p, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
+                                           s_abort,
                                            tmem_base, blockIdx.x, gridDim.x, num_tiles, BM, 0);
     }
 
@@ -561,7 +668,8 @@ struct SmemPair {
     static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
     static constexpr int SIDE_OFF = B_OFF + STAGES * B_BYTES;
     static constexpr int SCALE_OFF = SIDE_OFF + OC * BN * 4;
-    static constexpr int BAR_OFF = SCALE_OFF + BN * 4;
+    static constexpr int COLS_OFF = SCALE_OFF + BN * 4;
+    static constexpr int BAR_OFF = COLS_OFF + OC * 4;
     static constexpr int NBARS = 2 * STAGES + 5;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int BYTES = MISC_OFF + 16;
@@ -599,6 +707,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const bool leader = rank == 0;
     float *s_side = reinterpret_cast<float *>(smem + L::SIDE_OFF);
     float *s_scale = reinterpret_cast<float *>(smem + L::SCALE_OFF);
+    int *s_cols = reinterpret_cast<int *>(smem + L::COLS_OFF);
     const uint32_t bar0 = sbase + L::BAR_OFF;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -754,7 +863,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
-        run_epilogue<BN, false, RAW, true>(p, warp, lane, s_side, s_scale, tfull_bar(0), tempty_bar(0), s_abort,
+        run_epilogue<BN, false, RAW, true>(p, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
+                                           s_abort,
                                            tmem_base, pair_id, num_pairs, num_tiles, 2 * BM, (int)rank * BM);
     }
 
