@@ -183,6 +183,8 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
     // Few outlier columns: the next tile's staging loads go out before this
     // tile's epilogue and land while it runs (under the TMA stream a round of
     // them takes several microseconds, longer than a K = 4096 tile's MMAs).
+    static_assert(RAW || SWAP || OC * BN >= (kPipeGather + kPipeCols) * 128,
+                  "the pipelined staging keeps W's values and X's values in s_side");
     const bool pipe = !RAW && !SWAP && fast && cnt <= kPipeCols && cnt * BN <= kPipeGather * 128;
     StageRegs<BN> nx;
     if (pipe && first_tile < num_tiles)
@@ -211,9 +213,15 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                                         : __fdiv_rn(__fmul_rn((float)(int8_t)(uint8_t)nx.g[u], nx.gsb[u]), 127.0f);
             }
             own_scale = nx.own_scale;
+            // The row's outlier values of X go to this thread's slots after
+            // the staged W values (s_side holds OC * BN floats, the pipelined
+            // case fills at most kPipeCols * BN + kPipeCols * 128 of them),
+            // so that the outlier loop below can run over the actual count.
+            float *s_own = s_side + cnt * BN;
 #pragma unroll
             for (int k = 0; k < kPipeCols; ++k)
-                own_side[k] = __half2float(__ushort_as_half((unsigned short)nx.own_side[k]));
+                if (k < cnt)
+                    s_own[k * 128 + et] = __half2float(__ushort_as_half((unsigned short)nx.own_side[k]));
             named_barrier_sync(1, 128);
             if (tile + tile_step < num_tiles)
                 stage_issue<BN>(p, s_cols, cnt, tile + tile_step, a_tile_rows, a_row_off, r_in_tile, et, nx);
@@ -332,7 +340,25 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
                     y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
-                if (fast) {
+                if (pipe) {
+                    // A loop over the actual columns: the form unrolled over
+                    // OC below is about 1300 instructions per chunk, more
+                    // than the instruction cache keeps next to the rest.
+                    const float *s_own = s_side + cnt * BN;
+#pragma unroll 1
+                    for (int k = 0; k < cnt; ++k) {
+                        const float xv = s_own[k * 128 + et];
+                        const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 w = wrow[c4];
+                            y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                            y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                            y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                            y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                        }
+                    }
+                } else if (fast) {
 #pragma unroll
                     for (int k = 0; k < OC; ++k) {
                         if (k < cnt) {
