@@ -325,7 +325,11 @@ def test_tiny_workload(lib, dev, oracle_mod):
 @pytest.mark.parametrize("M,N,K,nout,give_w16", [
     (333, 777, 1024, 5, True), (333, 777, 1024, 5, False), (129, 300, 2048, 40, True),
     (1, 640, 1024, 6, False), (8, 640, 1024, 6, True), (16, 200, 512, 3, False), (17, 640, 1024, 6, True),
-    (32, 640, 1024, 6, False), (256, 512, 256, 0, True), (200, 384, 80, 2, True)])
+    (32, 640, 1024, 6, False), (256, 512, 256, 0, True), (200, 384, 80, 2, True),
+    # the epilogue's pipelined staging: at its column limit, one past it, both W sources,
+    # the single-CTA form, and more tiles than CTA pairs (each pair prefetches its next tile)
+    (300, 1000, 1024, 8, True), (300, 1000, 1024, 8, False), (300, 1000, 1024, 9, False),
+    (100, 700, 1024, 8, False), (1024, 8192, 256, 6, True), (1024, 8192, 256, 6, False)])
 def test_matmul_mixed_matches_oracle(lib, dev, oracle_mod, M, N, K, nout, give_w16):
     lin = Linear("t", M, N, K, nout, 60.0)
     X16, cols = make_activations(lin, seed=M + N)
