@@ -786,14 +786,7 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             for (int j = 0; j < nch; ++j)
                 mbar_init(smem_u32(&s_bars[j]), 1);
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            s_call = THR ? *reinterpret_cast<volatile uint32_t *>(calls) : 0u;
-            if (THR) {
-                // This call's barrier opens when the count reaches the next
-                // multiple of the grid (CTAs that arrived already are below it).
-                unsigned long long a;
-                asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(a) : "l"(arrivals) : "memory");
-                s_target = a - a % (unsigned long long)G + (unsigned long long)G;
-            }
+            s_call = 0u;
             s_cnt = 0;
             s_gcount = 0;
             s_fail = 0;
@@ -801,23 +794,38 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         }
         __syncwarp();
         __syncthreads();
+        // At most kQsInFlight chunks of this CTA in flight: the next is
+        // requested when the oldest lands, so that every CTA's rows arrive as
+        // a steady stream from the start (with all of them requested at once,
+        // the order HBM serves them in left some CTAs without their first
+        // rows until most of X had arrived). Lane 0 issues.
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(X + (int64_t)r0 * nvec);
+        auto issue = [&](int j) {
+            const uint32_t b0 = (uint32_t)(j * rpc) * (uint32_t)cols * 2u;
+            const uint32_t b1 = min(xbytes, (uint32_t)((j + 1) * rpc) * (uint32_t)cols * 2u);
+            const uint32_t bar = smem_u32(&s_bars[j]);
+            mbar_arrive_expect_tx(bar, b1 - b0);
+            for (uint32_t off = b0; off < b1; off += 32768u)
+                bulk_load(smem_u32(q_smem) + off, src + off, min(32768u, b1 - off), bar);
+        };
         if (lane == 0) {
-            // At most kQsInFlight chunks of this CTA in flight: the next is
-            // requested when the oldest lands, so that every CTA's rows
-            // arrive as a steady stream from the start (with all of them
-            // requested at once, the order HBM serves them in left some
-            // CTAs without their first rows until most of X had arrived).
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(X + (int64_t)r0 * nvec);
-            auto issue = [&](int j) {
-                const uint32_t b0 = (uint32_t)(j * rpc) * (uint32_t)cols * 2u;
-                const uint32_t b1 = min(xbytes, (uint32_t)((j + 1) * rpc) * (uint32_t)cols * 2u);
-                const uint32_t bar = smem_u32(&s_bars[j]);
-                mbar_arrive_expect_tx(bar, b1 - b0);
-                for (uint32_t off = b0; off < b1; off += 32768u)
-                    bulk_load(smem_u32(q_smem) + off, src + off, min(32768u, b1 - off), bar);
-            };
             for (int j = 0; j < min(nch, kQsInFlight); ++j)
                 issue(j);
+            if (THR) {
+                // The counters only after the first copies are on their way
+                // (each read is a global round trip): which global bitmap this
+                // call uses, and the arrival count its barrier opens at (the
+                // next multiple of the grid; CTAs that arrived already are
+                // below it).
+                s_call = *reinterpret_cast<volatile uint32_t *>(calls);
+                unsigned long long a;
+                asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(a) : "l"(arrivals) : "memory");
+                s_target = a - a % (unsigned long long)G + (unsigned long long)G;
+            }
+        }
+        if (THR)
+            named_barrier_arrive(4, kQsThreads); // s_call and s_target are set
+        if (lane == 0) {
             for (int j = kQsInFlight; j < nch; ++j) {
                 if (!mbar_wait(smem_u32(&s_bars[j - kQsInFlight]), 0u))
                     s_fail = 1; // the workers' wait on that chunk fails too
@@ -869,6 +877,8 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         for (int w = tid; w < nwords; w += kQsWorkers)
             s_bm[w] = 0u;
         __syncthreads();
+        if (THR)
+            named_barrier_sync(4, kQsThreads); // the control warp has read the counters
         if (THR && c == 0) { // the other bitmap, for the next call
             uint32_t *next = sets + ((s_call + 1u) & 1u) * kSetWords;
             for (int w = tid; w < (int)kSetWords; w += kQsWorkers)
