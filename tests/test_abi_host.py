@@ -67,6 +67,17 @@ def _mm(lib, X=A, M=64, K=128, CB=A, SCB=A, W=None, N=64, t=6.0, Y=A, ws=A, wsb=
     return lib._matmul_mixed(X, M, K, CB, SCB, W, N, t, Y, ws, wsb, None, None)
 
 
+def test_workspace_holds_the_fixed_regions(lib):
+    """Every workspace, whatever its shape, has the header and the resident
+    quantizer's two outlier bitmaps (sized for the widest X) at the front, so
+    that calls of any shapes can share it."""
+    fixed = 256 + 2 * 4 * ((133143 + 31) // 32)
+    for rows, cols in [(1, 16), (8, 64), (4096, 4096), (2048, 57344)]:
+        assert lib.quantize_workspace_size(rows, cols) >= fixed + (cols + 31) // 32 * 4 + cols * 4
+    for M, N, K in [(1, 16, 16), (32, 14336, 14336), (2048, 16384, 4096)]:
+        assert lib.workspace_size(M, N, K) >= fixed + M * K + 4 * M
+
+
 def test_matmul_argument_errors(lib):
     assert _mm(lib, K=100) == lib.ERR_UNSUPPORTED_SHAPE     # K % 16
     assert _mm(lib, K=0) == lib.ERR_UNSUPPORTED_SHAPE
