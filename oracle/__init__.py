@@ -59,6 +59,12 @@ def _load():
         lib.oracle_bias_act.restype = None
         lib.oracle_bias_act.argtypes = [P, I64, I64, P, ctypes.c_int]
         lib.oracle_mixed_output.restype = None
+        lib.oracle_quantize_rows_asym.argtypes = [P, I64, I64, P, P, P, P]
+        lib.oracle_quantize_rows_asym.restype = I64
+        lib.oracle_code_row_sums.argtypes = [P, I64, I64, P]
+        lib.oracle_code_row_sums.restype = None
+        lib.oracle_mixed_output_asym.argtypes = [P, P, P, P, P, I64, I64, P, I64, P, I64, P, P]
+        lib.oracle_mixed_output_asym.restype = None
         _lib = lib
     return _lib
 
@@ -192,3 +198,79 @@ def matmul_mixed(X, threshold: float, W=None, CB=None, SB=None, use_fp16_weight_
     Y_lin = mixed_output(acc, SX, SB, x, O, Wt)
     Y = Y_lin if (bias is None and not ACTIVATIONS[activation]) else bias_act(Y_lin, bias, activation)
     return dict(O=O, CX=CX, SX=SX, CB=CB, SB=SB, acc=acc, Wt=Wt, Y_lin=Y_lin, Y=Y)
+
+
+# ---- the zero-point (unsigned int8) variant: section "模型量化简介" ----------------
+
+def _mask(outlier, cols):
+    if outlier is None:
+        return None
+    outlier = np.asarray(outlier)
+    if outlier.dtype == np.uint8 and outlier.shape == (cols,):
+        return np.ascontiguousarray(outlier)
+    mask = np.zeros(cols, dtype=np.uint8)
+    mask[outlier.astype(np.int64)] = 1
+    return mask
+
+
+def quantize_rowwise_asym(X, outlier: np.ndarray | None = None):
+    """(codes int8 [M x K] = q - 128, scale fp32 [M], zero int32 [M]) of the
+    zero-point quantization over the non-outlier columns: range
+    [min(0, min x), max(0, max x)], s = 255 / range, z = rint(-lo * s),
+    q = clamp(rint(x * s) + z, 0, 255); outlier columns get q = z."""
+    x = _f32(X)
+    rows, cols = x.shape
+    mask = _mask(outlier, cols)
+    codes = np.empty((rows, cols), dtype=np.int8)
+    scale = np.empty(rows, dtype=np.float32)
+    zero = np.empty(rows, dtype=np.int32)
+    clamped = _load().oracle_quantize_rows_asym(_ptr(x), rows, cols, _ptr(mask), _ptr(codes), _ptr(scale),
+                                                _ptr(zero))
+    if clamped:
+        raise AssertionError(f"oracle clamped {clamped} zero-point codes")
+    return codes, scale, zero
+
+
+def code_row_sums(CB) -> np.ndarray:
+    """int64 [N]: sum over K of each row of the int8 weight codes."""
+    cb = np.ascontiguousarray(CB, dtype=np.int8)
+    N, K = cb.shape
+    R = np.empty(N, dtype=np.int64)
+    _load().oracle_code_row_sums(_ptr(cb), N, K, _ptr(R))
+    return R
+
+
+def mixed_output_asym(acc, scale, zero, R, SB, X, cols, Wt) -> np.ndarray:
+    """fp64 [M x N] = (acc + (128 - z_i) R_j) SB_j / (127 s_i) + X[:, cols] . Wt^T."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    M, N = acc.shape
+    x = _f32(X)
+    K = x.shape[1]
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    Wt = np.ascontiguousarray(Wt, dtype=np.float32)
+    sc = np.ascontiguousarray(scale, dtype=np.float32)
+    z = np.ascontiguousarray(zero, dtype=np.int32)
+    r = np.ascontiguousarray(R, dtype=np.int64)
+    sb = np.ascontiguousarray(SB, dtype=np.float32)
+    Y = np.empty((M, N), dtype=np.float64)
+    _load().oracle_mixed_output_asym(_ptr(acc), _ptr(sc), _ptr(z), _ptr(r), _ptr(sb), M, N, _ptr(x), K,
+                                     _ptr(cols), cols.size, _ptr(Wt), _ptr(Y))
+    return Y
+
+
+def matmul_mixed_asym(X, threshold: float, W=None, CB=None, SB=None, use_fp16_weight_cols: bool = True):
+    """The LLM.int8() linear with zero-point codes for X (the weight keeps its
+    absmax codes). Returns a dict with O, CX, SXs (scales), ZX (zero points),
+    CB, SB, R (code row sums), acc (int8 product of the stored codes), Wt and
+    Y (fp64)."""
+    x = _f32(X)
+    if CB is None:
+        CB, SB = quantize_weight(W)
+    N, K = CB.shape
+    O = outlier_cols(x, threshold)
+    CX, SXs, ZX = quantize_rowwise_asym(x, O)
+    acc = int8_matmul(CX, CB)
+    R = code_row_sums(CB)
+    Wt = outlier_weight(O, N, K, W=W if (W is not None and use_fp16_weight_cols) else None, CB=CB, SB=SB)
+    Y = mixed_output_asym(acc, SXs, ZX, R, SB, x, O, Wt)
+    return dict(O=O, CX=CX, SXs=SXs, ZX=ZX, CB=CB, SB=SB, R=R, acc=acc, Wt=Wt, Y=Y)

@@ -184,3 +184,85 @@ void oracle_bias_act(double *Y, int64_t M, int64_t N, const float *bias, int act
         }
     }
 }
+
+/* The unsigned-int8 / zero-point alternative to absmax quantization (section
+ * "模型量化简介": subtract the minimum and scale by the range, close to
+ * zero-point quantization, which keeps 0 exactly representable), applied row
+ * by row to the non-outlier part. Reading taken: the range of row i is
+ * [lo, hi] = [min(0, min x), max(0, max x)] over its non-outlier columns, so
+ * that 0 is inside it; s = 255 / (hi - lo) in fp32 (0 for an all-zero or
+ * empty row); zero point z = rint(-lo * s) in [0, 255]; code
+ * q = clamp(rint(x * s) + z, 0, 255), stored as the int8 value q - 128.
+ * Outlier columns get q = z (they then contribute nothing after z is taken
+ * off). Dequantization: x ~ (q - z) / s. Returns the number of codes clamped
+ * (0 when the arithmetic is right: hi * s <= 255 - z up to rounding). */
+int64_t oracle_quantize_rows_asym(const float *X, int64_t rows, int64_t cols, const uint8_t *is_outlier,
+                                  int8_t *codes, float *scale, int32_t *zero)
+{
+    int64_t clamped = 0;
+    for (int64_t i = 0; i < rows; ++i) {
+        const float *x = X + i * cols;
+        float lo = 0.0f, hi = 0.0f;
+        for (int64_t c = 0; c < cols; ++c) {
+            if (is_outlier && is_outlier[c])
+                continue;
+            if (x[c] < lo)
+                lo = x[c];
+            if (x[c] > hi)
+                hi = x[c];
+        }
+        const float range = hi - lo;
+        const float s = range > 0.0f ? 255.0f / range : 0.0f;
+        const int32_t z = (int32_t)rintf(-lo * s);
+        scale[i] = s;
+        zero[i] = z;
+        for (int64_t c = 0; c < cols; ++c) {
+            int32_t q = z;
+            if (!(is_outlier && is_outlier[c])) {
+                const float v = x[c] * s;
+                q = (int32_t)rintf(v) + z;
+            }
+            if (q < 0 || q > 255) {
+                ++clamped;
+                q = q < 0 ? 0 : 255;
+            }
+            codes[i * cols + c] = (int8_t)(q - 128);
+        }
+    }
+    return clamped;
+}
+
+/* Row sums of the int8 weight codes, R[j] = sum_c CB[j,c] (exact). */
+void oracle_code_row_sums(const int8_t *CB, int64_t N, int64_t K, int64_t *R)
+{
+    for (int64_t j = 0; j < N; ++j) {
+        int64_t s = 0;
+        for (int64_t c = 0; c < K; ++c)
+            s += CB[j * K + c];
+        R[j] = s;
+    }
+}
+
+/* Steps 2-3 with zero-point codes for X, in fp64: with c = q - 128,
+ *   sum_k (q - z_i) CB[j,k] = acc[i,j] + (128 - z_i) * R[j],
+ * dequantized by 1 / s_i on the X side and SB[j] / 127 on the weight side:
+ *   Y[i,j] = (acc[i,j] + (128 - z_i) R[j]) * SB[j] / (127 s_i)   (0 if s_i = 0)
+ *          + sum_k X[i, cols[k]] * Wt[j,k]. */
+void oracle_mixed_output_asym(const int32_t *acc, const float *SXs, const int32_t *ZX, const int64_t *R,
+                              const float *SB, int64_t M, int64_t N, const float *X, int64_t K,
+                              const int64_t *cols, int64_t n_out, const float *Wt, double *Y)
+{
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t j = 0; j < N; ++j) {
+            double y = 0.0;
+            if (SXs[i] > 0.0f) {
+                const double t = (double)acc[i * N + j] + (double)(128 - ZX[i]) * (double)R[j];
+                y = t * (double)SB[j] / (127.0 * (double)SXs[i]);
+            }
+            double o = 0.0;
+            for (int64_t k = 0; k < n_out; ++k)
+                o += (double)X[i * K + cols[k]] * (double)Wt[j * n_out + k];
+            Y[i * N + j] = y + o;
+        }
+    }
+}

@@ -331,3 +331,82 @@ def test_bias_is_added_per_output_feature(oracle_mod):
     assert np.allclose(diff, np.broadcast_to(bias.astype(np.float64), diff.shape), rtol=0, atol=1e-12)
     # a per-row (token) bias would be a different matrix
     assert not np.allclose(diff, bias[:6].astype(np.float64)[:, None], atol=1e-3)
+
+
+# ---- zero-point (unsigned int8) variant: section "模型量化简介" of the page
+# "Hugging Face 将 LLM.int8() 8-bit 量化集成进 transformers 与 accelerate" --------
+
+def test_asym_worked_vector_uses_the_full_unsigned_range(oracle_mod):
+    """The absmax example vector under zero-point quantization: its minimum
+    maps to q = 0 and its maximum to q = 255, and every value comes back
+    within half a step (1 / (2 s)) of itself."""
+    x = np.array([[1.2, -0.5, -4.3, 1.2, -3.1, 0.8, 2.4, 5.4]], dtype=np.float32)
+    c, s, z = oracle_mod.quantize_rowwise_asym(x)
+    q = c.astype(np.int32) + 128
+    assert q[0, 2] == 0 and q[0, 7] == 255
+    back = (q - z[:, None]) / s[:, None].astype(np.float64)
+    assert np.all(np.abs(back - x) <= 0.5 / s[0] * (1 + 1e-6))
+
+
+def test_asym_zero_is_exact_and_ranges_include_zero(oracle_mod):
+    """0 is represented exactly (q = z dequantizes to 0) whatever the signs of
+    the row, including all-positive and all-negative rows."""
+    rows = np.array([[0.0, 1.5, 3.0, 0.25], [-2.0, -1.0, 0.0, -0.5], [0.0, -3.0, 7.0, 1.0]], dtype=np.float32)
+    c, s, z = oracle_mod.quantize_rowwise_asym(rows)
+    q = c.astype(np.int32) + 128
+    for i in range(3):
+        zero_cols = np.flatnonzero(rows[i] == 0)
+        assert np.all(q[i, zero_cols] == z[i])
+    assert z[0] == 0 and q[0].max() == 255          # non-negative row: lo = 0
+    assert z[1] == 255 and q[1].min() == 0          # non-positive row: hi = 0
+
+
+def test_asym_all_zero_row_and_outlier_columns(oracle_mod):
+    """An all-zero row has scale 0; outlier columns carry q = z, so that they
+    drop out once the zero point is taken off."""
+    x = np.zeros((2, 16), dtype=np.float32)
+    x[1] = np.linspace(-1, 2, 16)
+    x[1, 5] = 40.0
+    c, s, z = oracle_mod.quantize_rowwise_asym(x, outlier=[5])
+    assert s[0] == 0 and z[0] == 0
+    q = c.astype(np.int32) + 128
+    assert q[1, 5] == z[1]
+    # the outlier column did not set the range
+    assert abs(255.0 / s[1] - 3.0) < 1e-5
+
+
+def test_asym_linear_equals_the_dequantized_product(oracle_mod):
+    """The oracle's asymmetric output, which goes through acc + (128 - z) R,
+    equals the fp64 product of the dequantized operands formed directly from
+    the codes (x~ = (q - z) / s, w~ = CB * SB / 127) plus the outlier part:
+    a dropped or sign-flipped correction term fails here."""
+    rng = np.random.default_rng(5)
+    X = (rng.standard_normal((9, 48)) + 0.7).astype(np.float16)
+    X[:, 11] *= 30
+    W = (0.02 * rng.standard_normal((13, 48))).astype(np.float16)
+    r = oracle_mod.matmul_mixed_asym(X, 6.0, W=W)
+    O = r["O"]
+    assert 11 in O
+    q = r["CX"].astype(np.float64) + 128
+    xt = (q - r["ZX"][:, None]) / r["SXs"].astype(np.float64)[:, None]
+    wt = r["CB"].astype(np.float64) * r["SB"].astype(np.float64)[:, None] / 127.0
+    keep = np.ones(48, bool)
+    keep[O] = False
+    ref = xt[:, keep] @ wt[:, keep].T + X.astype(np.float64)[:, O] @ W.astype(np.float64)[:, O].T
+    assert np.allclose(r["Y"], ref, rtol=1e-9, atol=1e-9)
+
+
+def test_asym_error_bound_against_exact_product(oracle_mod):
+    """|Y - X W^T| is within the quantization steps of the two operands:
+    sum_k |x| * SB / 254 + |w~| / (2 s) per output (plus fp32 slack)."""
+    rng = np.random.default_rng(6)
+    X = rng.standard_normal((7, 64)).astype(np.float16)
+    W = (0.05 * rng.standard_normal((5, 64))).astype(np.float16)
+    r = oracle_mod.matmul_mixed_asym(X, 0.0, W=W)
+    x = X.astype(np.float64)
+    w = W.astype(np.float64)
+    wt = r["CB"].astype(np.float64) * r["SB"].astype(np.float64)[:, None] / 127.0
+    bound = (np.abs(x) @ (r["SB"].astype(np.float64)[:, None] / 254.0 * np.ones((5, 64))).T
+             + (0.5 / r["SXs"].astype(np.float64))[:, None] * np.abs(wt).sum(1)[None, :])
+    err = np.abs(r["Y"] - x @ w.T)
+    assert np.all(err <= bound * (1 + 1e-4) + 1e-6)
