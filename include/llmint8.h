@@ -229,6 +229,54 @@ LLMINT8_API llmint8_status llmint8_matmul_mixed_fp16w(const void *X_f16, int64_t
                                           const llmint8_debug *dbg, llmint8_stream_t stream);
 
 /*
+ * Zero-point (unsigned int8) variant of the activation quantization: the
+ * alternative to absmax in section "模型量化简介" of the page "Hugging Face 将
+ * LLM.int8() 8-bit 量化集成进 transformers 与 accelerate" (subtract the minimum,
+ * scale by the range, 0 exactly representable). Per row of X, over the
+ * non-outlier columns: range [lo, hi] = [min(0, min x), max(0, max x)],
+ * s = 255 / (hi - lo) in fp32 (0 for an all-zero row), zero point
+ * z = rint(-lo * s), code q = clamp(rint(x * s) + z, 0, 255) stored as the
+ * int8 value q - 128 (rint: round half to even); outlier columns get q = z.
+ * The weight keeps its absmax codes (CB, SCB). With c = q - 128,
+ *   sum_k (q - z_i) CB[j,k] = acc[i,j] + (128 - z_i) * R[j],  R[j] = sum_k CB[j,k],
+ * so the int8 product is the same tensor-core GEMM and the epilogue adds
+ * (128 - z_i) R[j] before dequantizing by SB[j] / (127 s_i). K is limited to
+ * LLMINT8_MAX_K_ASYM so that these int8 sums fit in int32 (|c| <= 128).
+ */
+#define LLMINT8_MAX_K_ASYM 132104
+
+/* Zero-point codes of X [rows x cols] (fp16, device): codes int8 [rows x cols]
+ * out, scale fp32 [rows] out (s), zero int32 [rows] out (z). threshold and
+ * outlier_bitmap as in llmint8_quantize_rowwise (the bitmap is written; the
+ * outlier columns are found first, then the rows are coded against them).
+ * workspace: at least llmint8_quantize_workspace_size(rows, cols) bytes,
+ * zeroed once. Device pointers 16-byte aligned. Errors as
+ * llmint8_quantize_rowwise, with cols > LLMINT8_MAX_K_ASYM unsupported. */
+LLMINT8_API llmint8_status llmint8_quantize_rowwise_asym(const void *X_f16, int64_t rows, int64_t cols,
+                                             float threshold, int8_t *codes, float *scale, int32_t *zero,
+                                             uint32_t *outlier_bitmap, void *workspace, size_t ws_bytes,
+                                             llmint8_stream_t stream);
+
+/* R[j] = sum over K of CB[j, :] (int8 [N x K], device, 16-byte aligned) into
+ * row_sums int32 [N] (device, 4-byte aligned): the weight-side term of the
+ * zero-point product, computed once per weight like SCB. */
+LLMINT8_API llmint8_status llmint8_code_row_sums(const int8_t *CB, int64_t N, int64_t K, int32_t *row_sums,
+                                     llmint8_stream_t stream);
+
+/* Bytes of workspace needed by llmint8_matmul_mixed_asym. */
+LLMINT8_API size_t llmint8_workspace_size_asym(int64_t M, int64_t N, int64_t K);
+
+/* The LLM.int8() linear with zero-point codes for X: as llmint8_matmul_mixed,
+ * plus CB_row_sums (int32 [N], from llmint8_code_row_sums). Always runs the
+ * GEMM path (no fused decode kernel). dbg->row_absmax receives the scales s,
+ * dbg->codes the int8 codes q - 128, dbg->acc the int32 product of the stored
+ * codes. workspace >= llmint8_workspace_size_asym(M, N, K) bytes, zeroed once. */
+LLMINT8_API llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
+                                         const float *SCB, const int32_t *CB_row_sums, const void *W_f16,
+                                         int64_t N, float threshold, void *Y_f16, void *workspace,
+                                         size_t ws_bytes, const llmint8_debug *dbg, llmint8_stream_t stream);
+
+/*
  * Plain int8 GEMM with int32 output: acc[i,j] = sum_k A[i,k] * B[j,k]
  * (the int8 product of vector-wise quantization, [Q]).
  *   A (device) int8 [M x K], B (device) int8 [N x K], acc (device) int32 [M x N].

@@ -19,11 +19,13 @@ __all__ = [
     "LIB_PATH", "LLMInt8Error", "status_string", "quantize_workspace_size", "workspace_size",
     "workspace_init", "read_status", "quantize_rowwise", "find_outlier_cols", "matmul_mixed",
     "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc", "matmul_mixed_fp16w",
-    "workspace_size_fp16w", "ACTIVATIONS",
+    "workspace_size_fp16w", "ACTIVATIONS", "quantize_rowwise_asym", "code_row_sums", "workspace_size_asym",
+    "matmul_mixed_asym", "MAX_K_ASYM",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
 DEFAULT_THRESHOLD = 6.0
+MAX_K_ASYM = 132104  # LLMINT8_MAX_K_ASYM
 
 OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(7)
 
@@ -54,6 +56,12 @@ _SIGNATURES = {
                                          ctypes.c_size_t, ctypes.POINTER(_Debug), _P]),
     "llmint8_gemm_s8s8s32": (_ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
     "llmint8_quantize_rowwise_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
+    "llmint8_quantize_rowwise_asym": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                            _P]),
+    "llmint8_code_row_sums": (_ST, [_P, _I64, _I64, _P, _P]),
+    "llmint8_workspace_size_asym": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "llmint8_matmul_mixed_asym": (_ST, [_P, _I64, _I64, _P, _P, _P, _P, _I64, ctypes.c_float, _P, _P,
+                                        ctypes.c_size_t, ctypes.POINTER(_Debug), _P]),
 }
 EXPORTED = tuple(_SIGNATURES)
 NOALLOC_MAX_ROWS = NOALLOC_MAX_COLS = 65536
@@ -344,3 +352,74 @@ class Int8MixedLinear:
                                       activation=self.activation)
         return matmul_mixed(X, self.CB, self.SCB, self.W_f16, self.threshold, Y=Y, bias=self.bias,
                             activation=self.activation)
+
+
+# ---- zero-point (unsigned int8) codes for X ------------------------------------------
+
+def quantize_rowwise_asym(X, threshold: float = 0.0, codes=None, scale=None, zero=None, outlier_bitmap=None,
+                          workspace=None):
+    """(codes int8 = q - 128, scale fp32 [rows], zero int32 [rows], outlier_bitmap or None) of
+    fp16 X [rows x cols]: zero-point quantization over the non-outlier columns
+    (llmint8_quantize_rowwise_asym)."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    rows, cols = X.shape
+    dev = X.device
+    if codes is None:
+        codes = torch.empty((rows, cols), dtype=torch.int8, device=dev)
+    if scale is None:
+        scale = torch.empty(rows, dtype=torch.float32, device=dev)
+    if zero is None:
+        zero = torch.empty(rows, dtype=torch.int32, device=dev)
+    if outlier_bitmap is None and threshold > 0:
+        outlier_bitmap = torch.empty((cols + 31) // 32, dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else get_workspace(quantize_workspace_size(rows, cols), dev)
+    _check(load()["_quantize_rowwise_asym"](X.data_ptr(), rows, cols, float(threshold), codes.data_ptr(),
+                                            scale.data_ptr(), zero.data_ptr(), _ptr(outlier_bitmap), ws.data_ptr(),
+                                            ws.numel(), _stream_ptr(dev)), "llmint8_quantize_rowwise_asym")
+    return codes, scale, zero, outlier_bitmap
+
+
+def code_row_sums(CB, out=None):
+    """int32 [N]: the sum of each row of the int8 weight codes CB [N x K]."""
+    torch = _torch()
+    _need_cuda(CB, "CB", torch.int8)
+    N, K = CB.shape
+    if out is None:
+        out = torch.empty(N, dtype=torch.int32, device=CB.device)
+    _check(load()["_code_row_sums"](CB.data_ptr(), N, K, out.data_ptr(), _stream_ptr(CB.device)),
+           "llmint8_code_row_sums")
+    return out
+
+
+def workspace_size_asym(M: int, N: int, K: int) -> int:
+    return int(load()["_workspace_size_asym"](M, N, K))
+
+
+def matmul_mixed_asym(X, CB, SCB, CB_row_sums, W_f16=None, threshold: float = DEFAULT_THRESHOLD, Y=None,
+                      workspace=None, debug: dict | None = None):
+    """Y fp16 [M x N] = the LLM.int8() linear with zero-point codes for X
+    (llmint8_matmul_mixed_asym). ``CB_row_sums`` from code_row_sums(CB).
+    ``debug`` as for matmul_mixed (row_absmax receives the scales s)."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    _need_cuda(CB, "CB", torch.int8)
+    _need_cuda(SCB, "SCB", torch.float32)
+    _need_cuda(CB_row_sums, "CB_row_sums", torch.int32)
+    if W_f16 is not None:
+        _need_cuda(W_f16, "W_f16", torch.float16)
+    M, K = X.shape
+    N = CB.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    ws = workspace if workspace is not None else get_workspace(workspace_size_asym(M, N, K), dev)
+    dbg = None
+    if debug:
+        dbg = _Debug(*(_ptr(debug.get(k)) for k in ("codes", "row_absmax", "col_idx", "count", "acc")),
+                     *(_event(debug.get(k)) for k in ("gemm_begin", "gemm_end")))
+    _check(load()["_matmul_mixed_asym"](X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(), CB_row_sums.data_ptr(),
+                                        _ptr(W_f16), N, float(threshold), Y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                        ctypes.byref(dbg) if dbg else None, _stream_ptr(dev)),
+           "llmint8_matmul_mixed_asym")
+    return Y

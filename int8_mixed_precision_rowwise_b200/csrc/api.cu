@@ -419,3 +419,172 @@ llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B,
 }
 
 } // extern "C"
+
+// ---------------------------------------------------------------- zero-point variant
+
+namespace {
+
+llmint8_status check_k_asym(int64_t K)
+{
+    if (K <= 0 || K % 16 != 0 || K > LLMINT8_MAX_K_ASYM)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    return LLMINT8_OK;
+}
+
+// Outlier detection for the zero-point path: the absmax quantizer's bitmap
+// and column list (its codes and row maxima go to the given scratch and are
+// overwritten by the zero-point codes right after).
+cudaError_t detect_outliers(const void *X_f16, int64_t rows, int64_t cols, float t, int8_t *codes_scratch,
+                            float *rowmax_scratch, uint32_t *bitmap, const Workspace &ws, const DeviceInfo &dev,
+                            cudaStream_t stream)
+{
+    if (quantize_smem_fits(rows, cols, dev))
+        return launch_quantize_smem(X_f16, rows, cols, t, codes_scratch, rowmax_scratch, bitmap, ws.sets, ws.calls,
+                                    ws.arrivals, ws.col_idx, ws.count, ws.status, dev, stream);
+    cudaError_t e = cudaMemsetAsync(bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream);
+    if (e != cudaSuccess)
+        return e;
+    return launch_quantize(X_f16, rows, cols, t, codes_scratch, rowmax_scratch, bitmap, ws.col_idx, ws.count,
+                           ws.sync, ws.status, dev, stream);
+}
+
+} // namespace
+
+size_t llmint8_workspace_size_asym(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return 0;
+    (void)N;
+    return align256(carve(nullptr, M, K, true, false, nullptr)) + align256((size_t)M * 4);
+}
+
+llmint8_status llmint8_quantize_rowwise_asym(const void *X_f16, int64_t rows, int64_t cols, float threshold,
+                                             int8_t *codes, float *scale, int32_t *zero, uint32_t *outlier_bitmap,
+                                             void *workspace, size_t ws_bytes, llmint8_stream_t stream)
+{
+    if (rows < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k_asym(cols);
+    if (st != LLMINT8_OK)
+        return st;
+    if (rows > INT32_MAX || rows * cols > (int64_t)1 << 40)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    const float t = effective_threshold(threshold);
+    if (!X_f16 || !codes || !scale || !zero || !workspace || (t > 0.f && !outlier_bitmap))
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X_f16) || !aligned16(codes) || !aligned16(scale) || !aligned16(zero) || !aligned16(workspace) ||
+        (outlier_bitmap && !aligned16(outlier_bitmap)))
+        return LLMINT8_ERR_ALIGNMENT;
+    Workspace ws;
+    const size_t need = carve(static_cast<char *>(workspace), rows, cols, false, false, &ws);
+    if (ws_bytes < need)
+        return LLMINT8_ERR_WORKSPACE;
+    if (rows == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    cudaError_t e = cudaSuccess;
+    if (t > 0.f) {
+        if ((e = detect_outliers(X_f16, rows, cols, t, codes, scale, outlier_bitmap, ws, dev, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    } else if (outlier_bitmap &&
+               (e = cudaMemsetAsync(outlier_bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream)) != cudaSuccess) {
+        return LLMINT8_ERR_CUDA;
+    }
+    e = launch_quantize_asym(X_f16, rows, cols, t > 0.f ? outlier_bitmap : nullptr, codes, scale, zero, dev, stream);
+    return cuda_status(e);
+}
+
+llmint8_status llmint8_code_row_sums(const int8_t *CB, int64_t N, int64_t K, int32_t *row_sums,
+                                     llmint8_stream_t stream)
+{
+    if (N < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k_asym(K);
+    if (st != LLMINT8_OK)
+        return st;
+    if (N > INT32_MAX || N * K > (int64_t)1 << 40)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (!CB || !row_sums)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(CB) || (reinterpret_cast<uintptr_t>(row_sums) & 3u))
+        return LLMINT8_ERR_ALIGNMENT;
+    if (N == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return cuda_status(launch_code_row_sums(CB, N, K, row_sums, dev, stream));
+}
+
+llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
+                                         const float *SCB, const int32_t *CB_row_sums, const void *W_f16,
+                                         int64_t N, float threshold, void *Y_f16, void *workspace, size_t ws_bytes,
+                                         const llmint8_debug *dbg, llmint8_stream_t stream)
+{
+    if (M < 0 || N < 0)
+        return LLMINT8_ERR_INVALID_ARG;
+    llmint8_status st = check_k_asym(K);
+    if (st != LLMINT8_OK)
+        return st;
+    if (M > INT32_MAX || N > INT32_MAX || M * K > (int64_t)1 << 40 || N * K > (int64_t)1 << 40)
+        return LLMINT8_ERR_UNSUPPORTED_SHAPE;
+    if (!X_f16 || !CB || !SCB || !CB_row_sums || !Y_f16 || !workspace)
+        return LLMINT8_ERR_INVALID_ARG;
+    if (!aligned16(X_f16) || !aligned16(CB) || !aligned16(SCB) || !aligned16(Y_f16) || !aligned16(workspace) ||
+        (W_f16 && !aligned16(W_f16)) || (reinterpret_cast<uintptr_t>(CB_row_sums) & 3u))
+        return LLMINT8_ERR_ALIGNMENT;
+    if (dbg) {
+        if ((dbg->codes && !aligned16(dbg->codes)) || (dbg->row_absmax && !aligned16(dbg->row_absmax)) ||
+            (dbg->col_idx && !aligned16(dbg->col_idx)) || (dbg->acc && !aligned16(dbg->acc)) ||
+            (dbg->count && (reinterpret_cast<uintptr_t>(dbg->count) & 3u)))
+            return LLMINT8_ERR_ALIGNMENT;
+    }
+    Workspace ws;
+    const size_t base = align256(carve(static_cast<char *>(workspace), M, K, true, false, &ws));
+    if (ws_bytes < base + align256((size_t)M * 4))
+        return LLMINT8_ERR_WORKSPACE;
+    int32_t *zx = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + base);
+    if (M == 0 || N == 0)
+        return LLMINT8_OK;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    const float t = effective_threshold(threshold);
+    cudaError_t e = cudaSuccess;
+    if (t > 0.f) {
+        if ((e = detect_outliers(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws, dev, stream)) != cudaSuccess)
+            return LLMINT8_ERR_CUDA;
+    } else if ((e = cudaMemsetAsync(ws.count, 0, sizeof(int32_t), stream)) != cudaSuccess) {
+        return LLMINT8_ERR_CUDA;
+    }
+    if ((e = launch_quantize_asym(X_f16, M, K, t > 0.f ? ws.bitmap : nullptr, ws.cx, ws.sx, zx, dev, stream)) !=
+        cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    GemmArgs g{};
+    g.A = ws.cx;
+    g.B = CB;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.sx = ws.sx;
+    g.sb = SCB;
+    g.X16 = X_f16;
+    g.W16 = W_f16;
+    g.col_idx = ws.col_idx;
+    g.count = ws.count;
+    g.status = ws.status;
+    g.epi = Epilogue::MixedFp16;
+    g.Y = Y_f16;
+    g.zx = zx;
+    g.rsum = CB_row_sums;
+    if (dbg && dbg->gemm_begin &&
+        cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if ((e = launch_gemm(g, dev, stream)) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    if (dbg && dbg->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return copy_debug(dbg, ws, M, N, K, CB, SCB, X_f16, W_f16, true, dev, stream);
+}

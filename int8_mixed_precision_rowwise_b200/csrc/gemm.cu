@@ -58,6 +58,9 @@ struct KParams {
     int act;                   // LLMINT8_ACT_*
     void *Y;
     uint32_t *status;
+    // Zero-point codes of X (null: absmax codes): sx holds the scale s per
+    // row, zx the zero point, rsum the code row sums of W.
+    const int32_t *zx, *rsum;
 };
 
 template <int BN, int STAGES>
@@ -195,6 +198,7 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
         const int arow = mb * a_tile_rows + a_row_off + r_in_tile; // A-operand row of this thread
         const int brow0 = nb * BN;               // first B-operand row of the tile
         float own_scale = 0.f;
+        const int own_z = (!RAW && !SWAP && p.zx && arow < p.M) ? __ldg(p.zx + arow) : 128;
         float own_side[OC];
 #pragma unroll
         for (int k = 0; k < OC; ++k)
@@ -337,9 +341,22 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                     continue;
                 }
                 float y[32];
+                if (p.zx) {
+                    // Zero-point codes: sum_k (q - z_i) CB[j,k] = acc + (128 - z_i) R[j],
+                    // dequantized by SB[j] / (127 s_i) (s_i = 0: an all-zero row).
+                    const float zc = (float)(128 - own_z);
+                    const float inv = own_scale > 0.f ? __frcp_rn(127.0f * own_scale) : 0.f;
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
+                    for (int c = 0; c < 32; ++c) {
+                        const int j = j0 + c;
+                        const float rj = j < p.N ? (float)__ldg(p.rsum + j) : 0.f;
+                        y[c] = fmaf(zc, rj, (float)(int32_t)acc[c]) * (s_scale[g * 32 + c] * inv);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
+                }
                 if (pipe) {
                     // A loop over the actual columns: the form unrolled over
                     // OC below is about 1300 instructions per chunk, more
@@ -443,9 +460,22 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                 }
             } else {
                 float y[BN];
+                if (p.zx) {
+                    // Zero-point codes (see the other form): token c = brow0 + c.
+                    const float rj = j < p.N ? (float)__ldg(p.rsum + j) : 0.f;
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
-                    y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
+                    for (int c = 0; c < BN; ++c) {
+                        const int r = brow0 + c;
+                        const float zc = r < p.M ? (float)(128 - __ldg(p.zx + r)) : 0.f;
+                        const float sc = s_scale[c];
+                        const float inv = sc > 0.f ? __frcp_rn(127.0f * sc) : 0.f;
+                        y[c] = fmaf(zc, rj, (float)(int32_t)acc[c]) * (own_scale * inv);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
+                }
                 if (fast) {
 #pragma unroll
                     for (int k = 0; k < OC; ++k) {
@@ -1039,6 +1069,8 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     p.act = a.act;
     p.Y = a.Y;
     p.status = a.status;
+    p.zx = a.zx;
+    p.rsum = a.rsum;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int grid = std::min(tiles, dev.num_sms);
     return launch_dependent(kern, grid, L::ALLOC, stream, ta, tb, p);
@@ -1080,6 +1112,8 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.act = a.act;
     p.Y = a.Y;
     p.status = a.status;
+    p.zx = a.zx;
+    p.rsum = a.rsum;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int pairs = std::min(tiles, dev.num_sms / 2);
     return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, p);

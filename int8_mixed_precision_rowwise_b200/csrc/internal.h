@@ -140,6 +140,14 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
                                  unsigned long long *arrivals, int32_t *col_idx, int32_t *count,
                                  uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
 
+// Zero-point codes of X's rows against a complete outlier bitmap (null: no
+// outliers): codes int8 (q - 128), scale s and zero point z per row.
+cudaError_t launch_quantize_asym(const void *X, int64_t rows, int64_t cols, const uint32_t *bitmap, int8_t *codes,
+                                 float *scale, int32_t *zero, const DeviceInfo &dev, cudaStream_t stream);
+// R[j] = sum of the int8 codes of row j of CB [N x K] (K a multiple of 16).
+cudaError_t launch_code_row_sums(const int8_t *CB, int64_t N, int64_t K, int32_t *R, const DeviceInfo &dev,
+                                 cudaStream_t stream);
+
 // Bitmap -> ascending column list and count (one CTA).
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,
                            cudaStream_t stream);
@@ -162,6 +170,10 @@ struct GemmArgs {
     int act;             // LLMINT8_ACT_* applied after the bias
     void *Y;             // fp16 [M x N]  (MixedFp16) or int32 [M x N] (RawInt32)
     uint32_t *status;
+    // Zero-point codes of X (null: absmax codes): sx then holds the scale s
+    // per row, zx the zero point per row, rsum the code row sums of B.
+    const int32_t *zx;
+    const int32_t *rsum;
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, const DeviceInfo &dev, cudaStream_t stream);

@@ -1062,6 +1062,131 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
                               threshold_fp16(t), codes, absmax, bitmap_out, sets, calls, arrivals, col_idx, count, status);
 }
 
+namespace {
+
+// Zero-point quantization of the rows: the unsigned-int8 alternative to
+// absmax (page "Hugging Face 将 LLM.int8() 8-bit 量化集成进 transformers 与
+// accelerate", section "模型量化简介": subtract the minimum, scale by the
+// range, with 0 exactly representable), one warp per row. Over the columns
+// not in `bitmap` (null: every column): range [lo, hi] = [min(0, min x),
+// max(0, max x)], s = 255 / (hi - lo) in fp32 (0 for an all-zero row), zero
+// point z = rint(-lo * s), code q = clamp(rint(x * s) + z, 0, 255) stored as
+// the int8 value q - 128; columns in `bitmap` get q = z, so that they drop
+// out once z is taken off. Outlier columns are zeroed before the range is
+// taken (0 lies inside it anyway).
+__global__ void __launch_bounds__(256) k_quant_asym(const uint4 *__restrict__ X, int64_t rows, int cols,
+                                                    const uint32_t *__restrict__ bitmap, int8_t *__restrict__ codes,
+                                                    float *__restrict__ scale, int32_t *__restrict__ zero)
+{
+    extern __shared__ uint32_t s_abm[];
+    const int nvec = cols >> 3, nwords = (cols + 31) >> 5;
+    for (int w = threadIdx.x; w < nwords; w += blockDim.x)
+        s_abm[w] = bitmap ? bitmap[w] : 0u;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+        const uint4 *xr = X + r * nvec;
+        __half2 lo2 = __float2half2_rn(0.f), hi2 = __float2half2_rn(0.f);
+        for (int vi = lane; vi < nvec; vi += 32) {
+            uint4 v = __ldg(xr + vi);
+            const uint32_t kb = (s_abm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+            if (kb)
+                mask_known(v, kb);
+            const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                lo2 = __hmin2(lo2, h[i]);
+                hi2 = __hmax2(hi2, h[i]);
+            }
+        }
+        float lo = fminf(__low2float(lo2), __high2float(lo2));
+        float hi = fmaxf(__low2float(hi2), __high2float(hi2));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        const float range = __fsub_rn(hi, lo);
+        const float sc = range > 0.f ? __fdiv_rn(255.0f, range) : 0.f;
+        const int z = __float2int_rn(__fmul_rn(-lo, sc));
+        int8_t *cr = codes + r * (int64_t)cols;
+        for (int vi = lane; vi < nvec; vi += 32) {
+            const uint4 v = __ldg(xr + vi);
+            const uint32_t kb = (s_abm[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+            const __half *h = reinterpret_cast<const __half *>(&v);
+            uint32_t b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                int q = z;
+                if (!((kb >> e) & 1u))
+                    q = __float2int_rn(__fmul_rn(__half2float(h[e]), sc)) + z;
+                q = min(max(q, 0), 255);
+                b[e] = (uint32_t)(q - 128) & 0xFFu;
+            }
+            *reinterpret_cast<uint2 *>(cr + (int64_t)vi * 8) =
+                make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                           b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+        }
+        if (lane == 0) {
+            scale[r] = sc;
+            zero[r] = z;
+        }
+    }
+}
+
+// R[j] = sum over K of the int8 codes of row j (one warp per row, four codes
+// per __dp4a).
+__global__ void __launch_bounds__(256) k_code_row_sums(const uint4 *__restrict__ CB, int64_t N, int K,
+                                                       int32_t *__restrict__ R)
+{
+    const int lane = threadIdx.x & 31;
+    const int nv = K >> 4;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); j < N; j += nwarps) {
+        const uint4 *row = CB + j * nv;
+        int acc = 0;
+        for (int vi = lane; vi < nv; vi += 32) {
+            const uint4 v = __ldg(row + vi);
+            acc = __dp4a((int)v.x, 0x01010101, acc);
+            acc = __dp4a((int)v.y, 0x01010101, acc);
+            acc = __dp4a((int)v.z, 0x01010101, acc);
+            acc = __dp4a((int)v.w, 0x01010101, acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0)
+            R[j] = acc;
+    }
+}
+
+} // namespace
+
+cudaError_t launch_quantize_asym(const void *X, int64_t rows, int64_t cols, const uint32_t *bitmap, int8_t *codes,
+                                 float *scale, int32_t *zero, const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (rows <= 0)
+        return cudaSuccess;
+    const size_t smem = (size_t)((cols + 31) / 32) * 4;
+    const int64_t want = (rows + 7) / 8;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)dev.num_sms * 8);
+    k_quant_asym<<<grid, 256, smem, stream>>>(reinterpret_cast<const uint4 *>(X), rows, (int)cols, bitmap, codes,
+                                              scale, zero);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_code_row_sums(const int8_t *CB, int64_t N, int64_t K, int32_t *R, const DeviceInfo &dev,
+                                 cudaStream_t stream)
+{
+    if (N <= 0)
+        return cudaSuccess;
+    const int64_t want = (N + 7) / 8;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)dev.num_sms * 8);
+    k_code_row_sums<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(CB), N, (int)K, R);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_compact(const uint32_t *bitmap, int64_t cols, int32_t *col_idx, int32_t *count,
                            cudaStream_t stream)
 {

@@ -224,10 +224,9 @@ def quantize_rowwise_asym(X, outlier: np.ndarray | None = None):
     codes = np.empty((rows, cols), dtype=np.int8)
     scale = np.empty(rows, dtype=np.float32)
     zero = np.empty(rows, dtype=np.int32)
-    clamped = _load().oracle_quantize_rows_asym(_ptr(x), rows, cols, _ptr(mask), _ptr(codes), _ptr(scale),
-                                                _ptr(zero))
-    if clamped:
-        raise AssertionError(f"oracle clamped {clamped} zero-point codes")
+    # The clamp is part of the reading: rint(x s) and rint(-lo s) round
+    # separately, so the row's extreme values can land one step past [0, 255].
+    _load().oracle_quantize_rows_asym(_ptr(x), rows, cols, _ptr(mask), _ptr(codes), _ptr(scale), _ptr(zero))
     return codes, scale, zero
 
 

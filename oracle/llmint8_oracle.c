@@ -195,7 +195,8 @@ void oracle_bias_act(double *Y, int64_t M, int64_t N, const float *bias, int act
  * q = clamp(rint(x * s) + z, 0, 255), stored as the int8 value q - 128.
  * Outlier columns get q = z (they then contribute nothing after z is taken
  * off). Dequantization: x ~ (q - z) / s. Returns the number of codes clamped
- * (0 when the arithmetic is right: hi * s <= 255 - z up to rounding). */
+ * (rint(x * s) and rint(-lo * s) round separately, so the row's extreme
+ * values can land one step past [0, 255]; the clamp keeps them in range). */
 int64_t oracle_quantize_rows_asym(const float *X, int64_t rows, int64_t cols, const uint8_t *is_outlier,
                                   int8_t *codes, float *scale, int32_t *zero)
 {

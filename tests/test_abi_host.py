@@ -129,6 +129,38 @@ def test_matmul_fp16w_argument_errors(lib):
     assert call(act=3) == lib.ERR_INVALID_ARG
 
 
+def test_asym_argument_errors(lib):
+    """The zero-point entry points check their arguments before queuing work;
+    K is limited to LLMINT8_MAX_K_ASYM (int32 sums of codes up to 128 in size)."""
+    q = lib._quantize_rowwise_asym
+    ws = lib.quantize_workspace_size(32, 64)
+    assert q(A, 32, 64, 6.0, A, A, A, None, A, ws, None) == lib.ERR_INVALID_ARG      # bitmap needed when t > 0
+    assert q(A, 32, 64, 0.0, A, A, None, None, A, ws, None) == lib.ERR_INVALID_ARG   # zero points
+    assert q(A, 32, 60, 0.0, A, A, A, None, A, ws, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert q(A, 32, lib.MAX_K_ASYM + 16, 0.0, A, A, A, None, A, 1 << 30, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert q(A, 32, 64, 0.0, A, A + 4, A, None, A, ws, None) == lib.ERR_ALIGNMENT
+    assert q(A, 32, 64, 0.0, A, A, A, None, A, 16, None) == lib.ERR_WORKSPACE
+    assert q(A, 0, 64, 0.0, A, A, A, None, A, ws, None) == lib.OK
+    r = lib._code_row_sums
+    assert r(A, 8, 64, None, None) == lib.ERR_INVALID_ARG
+    assert r(A, 8, 60, A, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert r(A + 8, 8, 64, A, None) == lib.ERR_ALIGNMENT
+    assert r(A, 0, 64, A, None) == lib.OK
+    m = lib._matmul_mixed_asym
+    M, N, K = 64, 64, 128
+    wsa = lib.workspace_size_asym(M, N, K)
+    assert wsa >= lib.workspace_size(M, 1, K) + 4 * M
+
+    def call(R=A, wsb=wsa, K=K, X=A):
+        return m(X, M, K, A, A, R, None, N, 6.0, A, A, wsb, None, None)
+
+    assert call(R=None) == lib.ERR_INVALID_ARG
+    assert call(R=A + 2) == lib.ERR_ALIGNMENT
+    assert call(X=A + 8) == lib.ERR_ALIGNMENT
+    assert call(wsb=wsa - 256) == lib.ERR_WORKSPACE
+    assert call(K=lib.MAX_K_ASYM + 16) == lib.ERR_UNSUPPORTED_SHAPE
+
+
 def test_quantize_argument_errors(lib):
     q = lib._quantize_rowwise
     ws = lib.quantize_workspace_size(32, 64)

@@ -1,0 +1,106 @@
+"""GPU parity of the zero-point (unsigned int8) variant: codes, scales, zero
+points, outlier bitmaps and int32 products bit-exact against the oracle; the
+fp16 output within 1e-2 + 2e-3 |y|."""
+import numpy as np
+import pytest
+import torch
+
+from synthetic import Linear, make_activations, make_random, make_weight
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 1e-2, 2e-3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import int8_mixed_precision_rowwise_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def dev(lib):
+    return torch.device("cuda", 0)
+
+
+def to_dev(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def bitmap_to_mask(words: np.ndarray, cols: int) -> np.ndarray:
+    bits = np.unpackbits(words.astype("<u4").view(np.uint8), bitorder="little")
+    return bits[:cols].astype(np.uint8)
+
+
+@pytest.mark.parametrize("M,K,nout,t", [(8, 64, 2, 6.0), (300, 1024, 5, 6.0), (300, 1024, 5, 0.0),
+                                        (4096, 4096, 8, 6.0), (2048, 14336, 7, 6.0), (3, 16, 1, 6.0)])
+def test_quantize_asym_matches_oracle(lib, dev, oracle_mod, M, K, nout, t):
+    lin = Linear("a", M, 1, K, nout, 40.0)
+    X16, _ = make_activations(lin, seed=M + K)
+    X16[M // 2] += np.float16(0.75)  # a row whose range is not symmetric about 0
+    if M > 3:
+        X16[1] = 0                   # an all-zero row
+    codes, scale, zero, bm = lib.quantize_rowwise_asym(to_dev(X16, dev), t)
+    mask = oracle_mod.outlier_mask(X16, t) if t > 0 else np.zeros(K, np.uint8)
+    c_ref, s_ref, z_ref = oracle_mod.quantize_rowwise_asym(X16, mask)
+    if t > 0:
+        assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(zero.cpu().numpy(), z_ref)
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
+def test_code_row_sums_exact(lib, dev, oracle_mod):
+    rng = np.random.default_rng(2)
+    CB = rng.integers(-127, 128, size=(1000, 4096), dtype=np.int8)
+    CB[3] = 127
+    CB[4] = -127
+    R = lib.code_row_sums(to_dev(CB, dev)).cpu().numpy()
+    assert np.array_equal(R.astype(np.int64), oracle_mod.code_row_sums(CB))
+
+
+@pytest.mark.parametrize("M,N,K,nout,give_w16", [
+    (333, 777, 1024, 5, True), (333, 777, 1024, 5, False), (100, 700, 1024, 8, False),
+    (16, 640, 1024, 6, True), (32, 300, 512, 3, False), (1024, 8192, 256, 6, True), (200, 384, 80, 2, True)])
+def test_matmul_asym_matches_oracle(lib, dev, oracle_mod, M, N, K, nout, give_w16):
+    lin = Linear("a", M, N, K, nout, 60.0)
+    X16, _ = make_activations(lin, seed=M + N)
+    X16[0] += np.float16(1.5)  # asymmetric range
+    W16 = make_weight(lin, seed=K)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    R = lib.code_row_sums(CB)
+    dbg = dict(codes=torch.empty((M, K), dtype=torch.int8, device=dev),
+               row_absmax=torch.empty(M, dtype=torch.float32, device=dev),
+               col_idx=torch.empty(K, dtype=torch.int32, device=dev),
+               count=torch.empty(1, dtype=torch.int32, device=dev),
+               acc=torch.empty((M, N), dtype=torch.int32, device=dev))
+    Y = lib.matmul_mixed_asym(X, CB, SCB, R, W if give_w16 else None, 6.0, debug=dbg)
+    torch.cuda.synchronize()
+    r = oracle_mod.matmul_mixed_asym(X16, 6.0, W=W16, use_fp16_weight_cols=give_w16)
+    n = int(dbg["count"].item())
+    assert np.array_equal(dbg["col_idx"][:n].cpu().numpy(), r["O"])
+    assert np.array_equal(CB.cpu().numpy(), r["CB"])
+    assert np.array_equal(dbg["codes"].cpu().numpy(), r["CX"])
+    assert np.array_equal(dbg["row_absmax"].cpu().numpy().view(np.uint32), r["SXs"].view(np.uint32))
+    assert np.array_equal(dbg["acc"].cpu().numpy(), r["acc"])
+    y = Y.cpu().numpy().astype(np.float64)
+    err = np.abs(y - r["Y"])
+    assert np.all(err <= ATOL + RTOL * np.abs(r["Y"])), f"worst {err.max():.4g}"
+
+
+def test_matmul_asym_without_threshold_and_zero_rows(lib, dev, oracle_mod):
+    X16 = make_random((300, 512), seed=9)
+    X16[7] = 0
+    X16[8] = np.abs(X16[8])
+    W16 = make_random((256, 512), seed=10, scale=0.02)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    Y = lib.matmul_mixed_asym(X, CB, SCB, lib.code_row_sums(CB), None, 0.0)
+    torch.cuda.synchronize()
+    r = oracle_mod.matmul_mixed_asym(X16, 0.0, W=W16, use_fp16_weight_cols=False)
+    y = Y.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(y - r["Y"]) <= ATOL + RTOL * np.abs(r["Y"]))
+    assert not y[7].any()
