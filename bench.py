@@ -386,9 +386,45 @@ def measure_secondary(L, dev):
                                "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
         del layer, X, Y
     torch.cuda.empty_cache()
+    out["zero_point"] = zero_point_times(L, dev, hbm)
     # Last: the per-linear GEMMs run the GPU at its power cap for seconds.
     out["per_linear"] = per_linear_times(L, dev)
     return out
+
+
+def zero_point_times(L, dev, hbm):
+    """The zero-point variant: its quantizer on 4096 x 4096 (GB/s of the same
+    algorithmic bytes plus the zero points) and the whole linear on the
+    2048 x 16384 x 4096 prefill shape (TOPS), both CUDA-graph timed."""
+    import torch
+
+    res = {}
+    lin = synthetic.QUANT_4096.linears[0]
+    bufs = []
+    for k in range(8):
+        X, _, _ = synthetic.torch_device_problem(
+            synthetic.Linear("q", lin.M, 1, lin.K, lin.n_outlier_cols, lin.outlier_scale), k, dev)
+        bufs.append((X, torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
+                     torch.empty(lin.M, dtype=torch.float32, device=dev),
+                     torch.empty(lin.M, dtype=torch.int32, device=dev),
+                     torch.empty((lin.K + 31) // 32, dtype=torch.int32, device=dev)))
+    fns = [lambda b=b: L.quantize_rowwise_asym(b[0], 6.0, b[1], b[2], b[3], b[4]) for b in bufs]
+    ms = graph_time_ms(fns, reps=4)
+    byts = 2 * lin.M * lin.K + lin.M * lin.K + 8 * lin.M + lin.K // 8
+    res["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
+                                  "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+    del bufs, fns
+    lin = synthetic.Linear("prefill", 2048, 16384, 4096, 4, 60.0)
+    X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
+    CB, SCB, _ = L.quantize_rowwise(W, 0.0)
+    R = L.code_row_sums(CB)
+    Y = torch.empty((lin.M, lin.N), dtype=torch.float16, device=dev)
+    ms = graph_time_ms([lambda: L.matmul_mixed_asym(X, CB, SCB, R, W, 6.0, Y=Y)], reps=10)
+    res["prefill_2048x16384x4096"] = {"call_us": round(ms * 1e3, 1),
+                                      "call_tops": round(ops_of(lin) / (ms * 1e-3) / 1e12, 1)}
+    del X, W, CB, SCB, R, Y
+    torch.cuda.empty_cache()
+    return res
 
 
 # --------------------------------------------------------------------------- CPU oracle arm
