@@ -161,6 +161,23 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- GPU arm
 
+def max_over_ranks(values, world, device):
+    """Each timing's maximum over the ranks (the slowest replica sets the
+    job's time); unchanged with one rank."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tops(world, ops_per_step, steps, ms_total):
+    """Whole-job throughput: every replica's work over the slowest replica's time."""
+    return world * ops_per_step * steps / (ms_total * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -243,14 +260,11 @@ def run_ours(args, rank, world, local_rank):
 
     secondary = measure_secondary(L, dev) if rank == 0 else None
 
-    t = torch.tensor([ms_total, gemm_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, gemm_ms, e2e_ms = t.tolist()
+    ms_total, gemm_ms, e2e_ms = max_over_ranks([ms_total, gemm_ms, e2e_ms], world, dev)
     if rank != 0:
         return None
     ms_step = ms_total / args.steps
-    value = world * step_ops * args.steps / (ms_total * 1e-3) / 1e12
+    value = whole_job_tops(world, step_ops, args.steps, ms_total)
     gemm_launches = args.steps * nlin
     achieved = step_ops * args.steps / (gemm_ms * 1e-3) / 1e12
     peak = int8_peak_sustained
