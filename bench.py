@@ -154,7 +154,9 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+            why = ("no clock sample during the timed region (shorter than nvidia-smi's first sample)"
+                   if self.proc is not None else "nvidia-smi unavailable")
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [why], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
 
