@@ -121,6 +121,12 @@ class ClockSampler:
                  "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # the region starts once nvidia-smi delivers samples (it takes a
+            # moment to start), so that short regions are covered too
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 3.0 and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.skip = len(self.lines)
         except OSError:
             self.proc = None
         return self
@@ -141,7 +147,7 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for line in self.lines[getattr(self, "skip", 0):]:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -231,9 +237,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     ms_total = t0.elapsed_time(t1)
     gemm_ms = sum(ev_b[k][i].elapsed_time(ev_e[k][i]) for k in range(args.steps) for i in range(nlin))
-    status = L.read_status(L._workspaces[local_rank], clear=False)
-    if status:
-        raise RuntimeError(f"device status word {status:#x}: a kernel gave up on a bounded wait")
+    for ws in L.workspaces(local_rank):
+        status = L.read_status(ws, clear=False)
+        if status:
+            raise RuntimeError(f"device status word {status:#x}: a kernel gave up on a bounded wait")
 
     # e2e: the same step through the public API with host buffers: X from pinned
     # host memory to the device, the layer, Y back to pinned host memory.
@@ -260,7 +267,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
 
-    secondary = measure_secondary(L, dev) if rank == 0 else None
+    int8_measured = measure_int8_peak(dev, local_rank) if rank == 0 else None
+    secondary = measure_secondary(L, dev, local_rank) if rank == 0 else None
 
     ms_total, gemm_ms, e2e_ms = max_over_ranks([ms_total, gemm_ms, e2e_ms], world, dev)
     if rank != 0:
@@ -269,9 +277,10 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_tops(world, step_ops, args.steps, ms_total)
     gemm_launches = args.steps * nlin
     achieved = step_ops * args.steps / (gemm_ms * 1e-3) / 1e12
-    peak = int8_peak_sustained
     traffic = recorded_traffic()
     clk = clocks.summary()
+    peak, peak_choice = pick_int8_peak(int8_peak_burst, int8_peak_sustained, clk, ms_total * 1e-3,
+                                       peaks.get("sm_max_mhz"))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
@@ -281,10 +290,14 @@ def run_ours(args, rank, world, local_rank):
             "bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TOPS",
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "kernel": "k_gemm_i8_pair (CTA-pair tcgen05 int8 GEMM, fused dequant + outlier epilogue)",
-            "peak_source": f"2 x bf16 sustained of {peak_kind} ({peaks.get('bf16_tflops_sustained')} TF/s), "
-                           f"nominal int8:bf16 = 4.5:2.25; burst equivalent {round(int8_peak_burst, 1)}, "
-                           "spec 4500",
+            "peak_source": f"2 x bf16 {peak_choice['kind']} of {peak_kind} (bf16 {peaks.get('bf16_tflops')} burst / "
+                           f"{peaks.get('bf16_tflops_sustained')} sustained TF/s), nominal int8:bf16 = 4.5:2.25",
+            "peak_choice": peak_choice["why"],
+            "peak_burst": round(int8_peak_burst, 1), "peak_sustained": round(int8_peak_sustained, 1),
             "frac_of_spec_4500": round(achieved / 4500.0, 4),
+            "int8_measured": int8_measured,
+            "frac_of_int8_measured": (round(achieved / int8_measured["tops"], 4)
+                                      if int8_measured and int8_measured.get("tops") else None),
         },
         "gemm_share_of_step": round(gemm_ms / ms_total, 4),
         "cpu_baseline": cpu_baseline(args) if world == 1 else None,
@@ -296,6 +309,67 @@ def run_ours(args, rank, world, local_rank):
         "secondary": secondary,
     }
     return line
+
+
+def pick_int8_peak(burst, sustained, clk, timed_s, sm_max):
+    """The int8 denominator that matches the clocks the timed region ran at:
+    the burst figure when the median SM clock sat at (within 5% of) its
+    maximum, the sustained one when it sat below (the power cap pulled it
+    down), and, with no clock sample, burst for a region under a second (too
+    short for the cap to act) and sustained otherwise."""
+    sm = clk.get("sm_mhz")
+    mx = clk.get("sm_max_mhz") or sm_max
+    if sm is not None and mx:
+        if sm >= 0.95 * mx:
+            return burst, {"kind": "burst", "why": f"median SM clock {sm:.0f} MHz at its maximum {mx:.0f} MHz"}
+        return sustained, {"kind": "sustained",
+                           "why": f"median SM clock {sm:.0f} MHz below its maximum {mx:.0f} MHz (power cap)"}
+    if timed_s < 1.0:
+        return burst, {"kind": "burst", "why": f"no clock sample; timed region {timed_s:.3f} s, under 1 s"}
+    return sustained, {"kind": "sustained", "why": f"no clock sample; timed region {timed_s:.1f} s"}
+
+
+def measure_int8_peak(dev, index, reps=10):
+    """A measured int8 tensor-core rate on this GPU: cuBLAS's int8 GEMM
+    (torch._int_mm, int32 out) on the fc1 shape 2048 x 57344 x 14336, timed
+    alone with CUDA events, best of `reps`, for the weight operand both
+    column-major (a transposed view) and row-major; the faster layout counts."""
+    import torch
+
+    lin = {l.name: l for l in WORKLOAD.linears}["fc1"]
+    M, N, K = lin.M, lin.N, lin.K
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    A = torch.randint(-127, 128, (M, K), generator=g, device=dev, dtype=torch.int8)
+    B = torch.randint(-127, 128, (N, K), generator=g, device=dev, dtype=torch.int8)
+    out = {"routine": "torch._int_mm (cuBLAS int8, int32 out)", "shape": [M, N, K]}
+    best = None
+    with ClockSampler(index) as clocks:
+        for layout, b in (("B column-major", B.t()), ("B row-major", B.t().contiguous())):
+            try:
+                for _ in range(2):
+                    torch._int_mm(A, b)
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(reps):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    torch._int_mm(A, b)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    ts.append(e0.elapsed_time(e1))
+                tops = 2 * M * N * K / (min(ts) * 1e-3) / 1e12
+                out[layout] = round(tops, 1)
+                if best is None or tops > best:
+                    best = tops
+            except RuntimeError as e:
+                out[layout] = f"failed: {str(e).splitlines()[0][:120]}"
+            del b
+    del A, B
+    torch.cuda.empty_cache()
+    out["tops"] = round(best, 1) if best else None
+    out["clocks"] = clocks.summary()
+    return out
 
 
 def per_linear_times(L, dev, reps=10):
@@ -334,10 +408,12 @@ def per_linear_times(L, dev, reps=10):
     return res
 
 
-def graph_time_ms(fns, reps):
+def graph_time_ms(fns, reps, min_s=0.3):
     """Average device time per call of `fns` (called in turn, `reps` times),
     captured into one CUDA graph so host launch overhead is excluded; the
-    calls rotate over inputs larger than L2 together."""
+    calls rotate over inputs larger than L2 together. The graph is replayed
+    for at least `min_s` seconds (so that the clock sampler sees the load);
+    the median replay counts."""
     import torch
 
     s = torch.cuda.Stream()
@@ -355,7 +431,8 @@ def graph_time_ms(fns, reps):
     g.replay()
     torch.cuda.synchronize()
     ts = []
-    for _ in range(3):
+    t_start = time.time()
+    while len(ts) < 3 or (time.time() - t_start < min_s and len(ts) < 5000):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         g.replay()
@@ -366,16 +443,18 @@ def graph_time_ms(fns, reps):
     return statistics.median(ts)
 
 
-def measure_secondary(L, dev):
+def measure_secondary(L, dev, index):
     """The quantizer (4096 x 4096, 8 columns x40) and the decode path (BLOOM
     width, M = 1, 8, 32) in HBM GB/s of algorithmic bytes. Each is timed as a
     CUDA graph of back-to-back calls; the quantizer rotates over 8 inputs
-    (256 MB, twice L2), the decode weights (205 MB) exceed L2 by themselves."""
+    (256 MB, twice L2), the decode weights (205 MB) exceed L2 by themselves.
+    Every leg carries the SM clocks sampled while it ran."""
     import torch
 
     peaks, _ = load_peaks()
     hbm = peaks["hbm_gbs"]
-    out = {"timing": "CUDA graph of back-to-back calls; inputs larger than L2", "hbm_peak_gbs": hbm}
+    out = {"timing": "CUDA graph of back-to-back calls, replayed >= 0.3 s, median replay; inputs larger than L2",
+           "hbm_peak_gbs": hbm}
     lin = synthetic.QUANT_4096.linears[0]
     bufs = []
     for k in range(8):
@@ -385,10 +464,11 @@ def measure_secondary(L, dev):
                      torch.empty(lin.M, dtype=torch.float32, device=dev),
                      torch.empty((lin.K + 31) // 32, dtype=torch.int32, device=dev)))
     fns = [lambda b=b: L.quantize_rowwise(b[0], 6.0, b[1], b[2], b[3]) for b in bufs]
-    ms = graph_time_ms(fns, reps=4)
+    with ClockSampler(index) as clk:
+        ms = graph_time_ms(fns, reps=4)
     byts = 2 * lin.M * lin.K + lin.M * lin.K + 4 * lin.M + lin.K // 8
     out["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
-                                  "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+                                  "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3), "clocks": clk.summary()}
     del bufs, fns
     for M in (1, 8, 32):
         lin = synthetic.decode_bloom(M).linears[0]
@@ -396,19 +476,22 @@ def measure_secondary(L, dev):
         layer = L.Int8MixedLinear.from_fp16(W, keep_fp16_weights=False)
         del W
         Y = torch.empty((M, lin.N), dtype=torch.float16, device=dev)
-        ms = graph_time_ms([lambda: layer(X, Y)], reps=20)
+        with ClockSampler(index) as clk:
+            ms = graph_time_ms([lambda: layer(X, Y)], reps=20)
         byts = lin.N * lin.K + 4 * lin.N + 2 * M * lin.K + 2 * M * lin.N
         out[f"decode_M{M}"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
-                               "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+                               "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3), "clocks": clk.summary()}
         del layer, X, Y
     torch.cuda.empty_cache()
-    out["zero_point"] = zero_point_times(L, dev, hbm)
+    out["zero_point"] = zero_point_times(L, dev, hbm, index)
     # Last: the per-linear GEMMs run the GPU at its power cap for seconds.
-    out["per_linear"] = per_linear_times(L, dev)
+    with ClockSampler(index) as clk:
+        out["per_linear"] = per_linear_times(L, dev)
+    out["per_linear"]["clocks"] = clk.summary()
     return out
 
 
-def zero_point_times(L, dev, hbm):
+def zero_point_times(L, dev, hbm, index):
     """The zero-point variant: its quantizer on 4096 x 4096 (GB/s of the same
     algorithmic bytes plus the zero points) and the whole linear on the
     2048 x 16384 x 4096 prefill shape (TOPS), both CUDA-graph timed."""
@@ -425,19 +508,22 @@ def zero_point_times(L, dev, hbm):
                      torch.empty(lin.M, dtype=torch.int32, device=dev),
                      torch.empty((lin.K + 31) // 32, dtype=torch.int32, device=dev)))
     fns = [lambda b=b: L.quantize_rowwise_asym(b[0], 6.0, b[1], b[2], b[3], b[4]) for b in bufs]
-    ms = graph_time_ms(fns, reps=4)
+    with ClockSampler(index) as clk:
+        ms = graph_time_ms(fns, reps=4)
     byts = 2 * lin.M * lin.K + lin.M * lin.K + 8 * lin.M + lin.K // 8
     res["quantizer_4096x4096"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
-                                  "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3)}
+                                  "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3), "clocks": clk.summary()}
     del bufs, fns
     lin = synthetic.Linear("prefill", 2048, 16384, 4096, 4, 60.0)
     X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
     CB, SCB, _ = L.quantize_rowwise(W, 0.0)
     R = L.code_row_sums(CB)
     Y = torch.empty((lin.M, lin.N), dtype=torch.float16, device=dev)
-    ms = graph_time_ms([lambda: L.matmul_mixed_asym(X, CB, SCB, R, W, 6.0, Y=Y)], reps=10)
+    with ClockSampler(index) as clk:
+        ms = graph_time_ms([lambda: L.matmul_mixed_asym(X, CB, SCB, R, W, 6.0, Y=Y)], reps=10)
     res["prefill_2048x16384x4096"] = {"call_us": round(ms * 1e3, 1),
-                                      "call_tops": round(ops_of(lin) / (ms * 1e-3) / 1e12, 1)}
+                                      "call_tops": round(ops_of(lin) / (ms * 1e-3) / 1e12, 1),
+                                      "clocks": clk.summary()}
     del X, W, CB, SCB, R, Y
     torch.cuda.empty_cache()
     return res
@@ -457,6 +543,62 @@ def oracle_sample_step(oracle, lin, li):
     return 2 * lin.M * SAMPLE_COLS * lin.K
 
 
+def host_info():
+    """The host the oracle runs on: logical CPUs the process may use, the CPU
+    model, and the threads the oracle uses (it is single-threaded C)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count()
+    return {"nproc": usable, "cpu_count": os.cpu_count(), "cpu_model": model, "oracle_threads": 1}
+
+
+def oracle_full_configs(oracle):
+    """The oracle timed on whole workloads that it finishes in seconds: the
+    tiny linear (8 x 64 -> 128), the 4096 x 4096 quantizer and the decode
+    linears at BLOOM width (M = 1, 8, 32 against a 14336 x 14336 int8
+    weight), each in the metric the GPU lines report (us, GB/s of the same
+    algorithmic bytes). Weight preparation (quantizing W) is not timed."""
+    res = {}
+    lin = synthetic.TINY.linears[0]
+    X16, W16, _ = synthetic.make_problem(lin, seed=0)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < 0.5:
+        oracle.matmul_mixed(X16, synthetic.TINY.threshold, W=W16)
+        n += 1
+    res["tiny_8x64x128"] = {"us": round((time.perf_counter() - t0) / n * 1e6, 1), "calls": n}
+    lin = synthetic.QUANT_4096.linears[0]
+    X16, _ = synthetic.make_activations(lin, seed=0)
+    t0 = time.perf_counter()
+    O = oracle.outlier_cols(X16, 6.0)
+    oracle.quantize_rowwise(X16, O)
+    sec = time.perf_counter() - t0
+    byts = 2 * lin.M * lin.K + lin.M * lin.K + 4 * lin.M + lin.K // 8
+    res["quantizer_4096x4096"] = {"ms": round(sec * 1e3, 1), "GBs": round(byts / sec / 1e9, 3)}
+    dlin = synthetic.decode_bloom(1).linears[0]
+    W16 = synthetic.make_weight(dlin, seed=0)
+    CB, SB = oracle.quantize_weight(W16)
+    del W16
+    for M in (1, 8, 32):
+        lin = synthetic.decode_bloom(M).linears[0]
+        X16, _ = synthetic.make_activations(lin, seed=M)
+        t0 = time.perf_counter()
+        oracle.matmul_mixed(X16, 6.0, CB=CB, SB=SB)
+        sec = time.perf_counter() - t0
+        byts = lin.N * lin.K + 4 * lin.N + 2 * M * lin.K + 2 * M * lin.N
+        res[f"decode_M{M}"] = {"ms": round(sec * 1e3, 1), "GBs": round(byts / sec / 1e9, 3)}
+    return res
+
+
 def cpu_baseline(args, steps=1):
     import oracle
 
@@ -470,10 +612,12 @@ def cpu_baseline(args, steps=1):
             oracle.matmul_mixed(X, WORKLOAD.threshold, W=W)
             secs += time.perf_counter() - t0
             ops += 2 * lin.M * SAMPLE_COLS * lin.K
+    host = host_info()
     return {"value": round(ops / secs / 1e12, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"all {WORKLOAD.linears[0].M} tokens x {SAMPLE_COLS} output rows of each of the four "
                       f"linears (full outlier detection and quantization of X), single-threaded C, "
-                      f"{secs:.1f} s"}
+                      f"{secs:.1f} s",
+            "host": host, "full_configs": oracle_full_configs(oracle)}
 
 
 def run_reference(args, rank, world):
@@ -501,7 +645,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": workload_config({"parallelism": "single"}),
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                         "host": host_info()},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -558,7 +703,7 @@ def run_profile_case(args):
             layer(xs[i], ys[i])
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
-    assert L.read_status(L._workspaces[0], clear=False) == 0
+    assert all(L.read_status(ws, clear=False) == 0 for ws in L.workspaces(0))
 
 
 def main():

@@ -30,7 +30,10 @@
  *     stream) and returns without waiting, except where stated.
  *   - Argument errors are returned before anything is queued. A failed launch
  *     returns LLMINT8_ERR_CUDA. Kernels never trap: a bounded wait that runs
- *     out sets a bit in the workspace status word (llmint8_read_status).
+ *     out sets a bit in the workspace status word. Compute calls only queue
+ *     work, so they return LLMINT8_OK before any kernel has run and never
+ *     report such a failure themselves; llmint8_read_status (after the
+ *     stream has finished) is the one place it shows, as LLMINT8_ERR_DEVICE.
  *   - fp16 inputs must be finite; NaN or Inf inputs are outside the contract.
  *   - M (rows) == 0 or N == 0 is a no-op that returns LLMINT8_OK.
  */
@@ -86,8 +89,12 @@ LLMINT8_API size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K);
 LLMINT8_API llmint8_status llmint8_workspace_init(void *workspace, size_t ws_bytes, llmint8_stream_t stream);
 
 /* Synchronously read (and, if clear != 0, reset) the device status word of a
- * workspace after the stream has finished. *out == 0 means no kernel reported
- * a failure. Waits for the whole device (cudaDeviceSynchronize). */
+ * workspace after the stream has finished. Waits for the whole device
+ * (cudaDeviceSynchronize). *out receives the word (LLMINT8_DEV_* bits). Returns
+ * LLMINT8_OK when it is 0, LLMINT8_ERR_DEVICE when a kernel reported a
+ * failure (its outputs are then incomplete; re-zero the workspace with
+ * llmint8_workspace_init before its next use), LLMINT8_ERR_CUDA if the
+ * synchronisation or the copy failed. */
 LLMINT8_API llmint8_status llmint8_read_status(void *workspace, size_t ws_bytes, int clear, uint32_t *out);
 
 /*
@@ -307,12 +314,25 @@ LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, cons
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents. Calls ordered on one stream are safe; calls whose work
  *     overlaps on the GPU (unordered streams) race and give wrong results.
+ *   - The address lookup is cached for the life of the process: after a
+ *     cudaDeviceReset of that device this entry point must not be called.
+ *   - A kernel that gives up on a bounded wait sets a bit in the array's own
+ *     status word (the outputs are then incomplete). The word keeps its bits
+ *     across calls until llmint8_noalloc_read_status reads and clears it.
  */
 #define LLMINT8_NOALLOC_MAX_ROWS 65536
 #define LLMINT8_NOALLOC_MAX_COLS 65536
 LLMINT8_API llmint8_status llmint8_quantize_rowwise_noalloc(const void *X_f16, int64_t rows, int64_t cols,
                                                 float threshold, int8_t *codes, float *row_absmax,
                                                 uint32_t *outlier_bitmap, llmint8_stream_t stream);
+
+/* Status word of llmint8_quantize_rowwise_noalloc's fixed array on the current
+ * device: waits for the device (cudaDeviceSynchronize), copies the word to
+ * *out (LLMINT8_DEV_* bits, 0 if no call since the last clear gave up on a
+ * wait) and, if clear != 0, resets it. Returns LLMINT8_OK when the word is 0,
+ * LLMINT8_ERR_DEVICE when it is not, LLMINT8_ERR_CUDA if a CUDA call failed,
+ * LLMINT8_ERR_INVALID_ARG for a NULL out. Allocates nothing. */
+LLMINT8_API llmint8_status llmint8_noalloc_read_status(int clear, uint32_t *out);
 
 #ifdef __cplusplus
 }

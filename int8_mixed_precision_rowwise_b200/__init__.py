@@ -18,7 +18,8 @@ import os
 __all__ = [
     "LIB_PATH", "LLMInt8Error", "status_string", "quantize_workspace_size", "workspace_size",
     "workspace_init", "read_status", "quantize_rowwise", "find_outlier_cols", "matmul_mixed",
-    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc", "matmul_mixed_fp16w",
+    "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc", "noalloc_read_status",
+    "matmul_mixed_fp16w",
     "workspace_size_fp16w", "ACTIVATIONS", "quantize_rowwise_asym", "code_row_sums", "workspace_size_asym",
     "matmul_mixed_asym", "MAX_K_ASYM",
 ]
@@ -56,6 +57,7 @@ _SIGNATURES = {
                                          ctypes.c_size_t, ctypes.POINTER(_Debug), _P]),
     "llmint8_gemm_s8s8s32": (_ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
     "llmint8_quantize_rowwise_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
+    "llmint8_noalloc_read_status": (_ST, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]),
     "llmint8_quantize_rowwise_asym": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                             _P]),
     "llmint8_code_row_sums": (_ST, [_P, _I64, _I64, _P, _P]),
@@ -151,18 +153,31 @@ def _need_cuda(t, name, dtype=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+# Cached workspaces, one per (device index, raw stream handle): calls that
+# share a workspace must be ordered, which calls queued on one stream are, so
+# two streams never share one.
 _workspaces: dict = {}
 
 
 def get_workspace(nbytes: int, device):
-    """A zeroed, cached workspace of at least nbytes on `device` (grown on demand)."""
+    """A zeroed, cached workspace of at least nbytes for `device` and its
+    current stream (grown on demand)."""
     torch = _torch()
-    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    d = torch.device(device)
+    index = d.index if d.index is not None else torch.cuda.current_device()
+    key = (index, _stream_ptr(torch.device("cuda", index)))
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
+        # The old buffer may still be in use by queued work on that stream:
+        # torch's allocator keeps it alive until the stream reaches this point.
+        ws = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=d)
         _workspaces[key] = ws
     return ws
+
+
+def workspaces(device=None) -> list:
+    """The cached workspaces (of one device index, or all)."""
+    return [ws for (idx, _), ws in _workspaces.items() if device is None or idx == device]
 
 
 def workspace_init(ws) -> None:
@@ -170,8 +185,22 @@ def workspace_init(ws) -> None:
 
 
 def read_status(ws, clear: bool = True) -> int:
+    """The workspace's device status word (0: no kernel gave up on a wait)."""
     out = ctypes.c_uint32(0)
-    _check(load()["_read_status"](ws.data_ptr(), ws.numel(), int(clear), ctypes.byref(out)), "llmint8_read_status")
+    st = load()["_read_status"](ws.data_ptr(), ws.numel(), int(clear), ctypes.byref(out))
+    if st != ERR_DEVICE:
+        _check(st, "llmint8_read_status")
+    return int(out.value)
+
+
+def noalloc_read_status(clear: bool = True) -> int:
+    """The status word of the allocation-free quantizer's fixed array on the
+    current device (0: none of its calls since the last clear gave up on a
+    wait)."""
+    out = ctypes.c_uint32(0)
+    st = load()["_noalloc_read_status"](int(clear), ctypes.byref(out))
+    if st != ERR_DEVICE:
+        _check(st, "llmint8_noalloc_read_status")
     return int(out.value)
 
 

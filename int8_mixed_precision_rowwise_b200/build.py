@@ -23,9 +23,10 @@ NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-Xcompiler", "-fPIC,-fvisibility=hidden",
-    "-shared", "-cudart", "static",
     "--expt-relaxed-constexpr",
 ]
+LINK_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static"]
+OBJ_DIR = os.path.join(HERE, "_build")
 
 
 def _nvcc() -> str:
@@ -44,10 +45,24 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile every source to an object in parallel (one nvcc per file), then
+    link the shared library with the CUDA runtime linked in statically."""
     if not force and not _stale():
         return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", LIB + ".tmp",
-           *[os.path.join(CSRC, f) for f in SOURCES]]
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    procs = []
+    objs = []
+    for f in SOURCES:
+        obj = os.path.join(OBJ_DIR, f + ".o")
+        objs.append(obj)
+        cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", "-o", obj, os.path.join(CSRC, f)]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        procs.append((f, subprocess.Popen(cmd)))
+    failed = [f for f, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(failed)})")
+    cmd = [_nvcc(), *LINK_FLAGS, "-o", LIB + ".tmp", *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)

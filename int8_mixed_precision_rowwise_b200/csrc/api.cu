@@ -167,7 +167,9 @@ llmint8_status llmint8_read_status(void *workspace, size_t ws_bytes, int clear, 
         e = cudaMemcpy(out, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && clear)
         e = cudaMemset(workspace, 0, sizeof(uint32_t));
-    return cuda_status(e);
+    if (e != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return *out ? LLMINT8_ERR_DEVICE : LLMINT8_OK;
 }
 
 llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t cols, float threshold,

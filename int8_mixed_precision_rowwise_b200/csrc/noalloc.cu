@@ -15,6 +15,10 @@
 // All calls on a device share it and it keeps the last call's contents, so
 // two calls whose work overlaps on the GPU (different streams, no ordering
 // between them) race on it; calls ordered on one stream are safe.
+//
+// Its status word keeps the bits of every call since it was last cleared
+// (a kernel that gave up on a bounded wait sets one and leaves its outputs
+// incomplete); llmint8_noalloc_read_status reads and clears it.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -29,9 +33,15 @@ namespace {
 
 constexpr int64_t kMaxRows = LLMINT8_NOALLOC_MAX_ROWS;
 constexpr int64_t kMaxCols = LLMINT8_NOALLOC_MAX_COLS;
-constexpr size_t kHeaderBytes = 256; // int32 |O| at 0, uint32 status at 4, grid-barrier words at 8
-constexpr size_t kColIdxOff = kHeaderBytes;
-constexpr size_t kScratchBytes = kColIdxOff + (size_t)kMaxCols * 4;
+// The array's header uses the first words of a workspace header (carve() in
+// internal.h): uint32 status at 0, int32 |O| at 4, the grid barrier's 64-bit
+// word at 8, the late-outlier flag at 16. Change the two together.
+constexpr size_t kNoallocHeaderBytes = 256;
+constexpr size_t kNoallocStatusOff = 0;
+constexpr size_t kNoallocCountOff = 4;
+constexpr size_t kNoallocSyncOff = 8;
+constexpr size_t kNoallocColIdxOff = kNoallocHeaderBytes;
+constexpr size_t kScratchBytes = kNoallocColIdxOff + (size_t)kMaxCols * 4;
 
 // The scratch. In host code this name is only a stand-in: the device address
 // comes from cudaGetSymbolAddress below, once per device.
@@ -41,7 +51,9 @@ std::mutex g_mu;
 void *g_scratch_addr[64] = {};
 
 // Device address of g_scratch on the current device `dev`, looked up on the
-// first call for that device and cached.
+// first call for that device and cached for the life of the process (a
+// cudaDeviceReset on that device invalidates it; this entry point must not be
+// used after one).
 cudaError_t scratch_address(int dev, void **out)
 {
     if (dev < 0 || dev >= 64)
@@ -90,13 +102,15 @@ extern "C" llmint8_status llmint8_quantize_rowwise_noalloc(const void *X_f16, in
     if (scratch_address(dev.device, &base) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     char *s = static_cast<char *>(base);
-    int32_t *count = reinterpret_cast<int32_t *>(s);
-    uint32_t *status = reinterpret_cast<uint32_t *>(s + 4);
-    uint32_t *sync = reinterpret_cast<uint32_t *>(s + 8);
-    int32_t *col_idx = reinterpret_cast<int32_t *>(s + kColIdxOff);
-    // The array keeps the previous call's contents: clear the count, status
-    // and grid-barrier words, and the caller's bitmap, which the kernels OR into.
-    if (cudaMemsetAsync(count, 0, 24, stream) != cudaSuccess)
+    uint32_t *status = reinterpret_cast<uint32_t *>(s + kNoallocStatusOff);
+    int32_t *count = reinterpret_cast<int32_t *>(s + kNoallocCountOff);
+    uint32_t *sync = reinterpret_cast<uint32_t *>(s + kNoallocSyncOff);
+    int32_t *col_idx = reinterpret_cast<int32_t *>(s + kNoallocColIdxOff);
+    // The array keeps the previous call's contents: clear the count, the
+    // grid-barrier word and the late-outlier flag (bytes 4..19, not the status
+    // word, which accumulates until read), and the caller's bitmap, which the
+    // kernels OR into.
+    if (cudaMemsetAsync(count, 0, 16, stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     if (outlier_bitmap &&
         cudaMemsetAsync(outlier_bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream) != cudaSuccess)
@@ -104,4 +118,25 @@ extern "C" llmint8_status llmint8_quantize_rowwise_noalloc(const void *X_f16, in
     cudaError_t e = launch_quantize(X_f16, rows, cols, t, codes, row_absmax, outlier_bitmap, col_idx, count, sync,
                                     status, dev, stream);
     return e == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+extern "C" llmint8_status llmint8_noalloc_read_status(int clear, uint32_t *out)
+{
+    if (!out)
+        return LLMINT8_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    void *base = nullptr;
+    if (scratch_address(dev.device, &base) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    uint32_t *status = reinterpret_cast<uint32_t *>(static_cast<char *>(base) + kNoallocStatusOff);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(out, status, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear)
+        e = cudaMemset(status, 0, sizeof(uint32_t));
+    if (e != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    return *out ? LLMINT8_ERR_DEVICE : LLMINT8_OK;
 }

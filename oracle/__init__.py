@@ -213,11 +213,12 @@ def _mask(outlier, cols):
     return mask
 
 
-def quantize_rowwise_asym(X, outlier: np.ndarray | None = None):
+def quantize_rowwise_asym(X, outlier: np.ndarray | None = None, return_clamped: bool = False):
     """(codes int8 [M x K] = q - 128, scale fp32 [M], zero int32 [M]) of the
     zero-point quantization over the non-outlier columns: range
     [min(0, min x), max(0, max x)], s = 255 / range, z = rint(-lo * s),
-    q = clamp(rint(x * s) + z, 0, 255); outlier columns get q = z."""
+    q = clamp(rint(x * s) + z, 0, 255); outlier columns get q = z. With
+    ``return_clamped`` a fourth item: how many codes the clamp moved."""
     x = _f32(X)
     rows, cols = x.shape
     mask = _mask(outlier, cols)
@@ -226,7 +227,10 @@ def quantize_rowwise_asym(X, outlier: np.ndarray | None = None):
     zero = np.empty(rows, dtype=np.int32)
     # The clamp is part of the reading: rint(x s) and rint(-lo s) round
     # separately, so the row's extreme values can land one step past [0, 255].
-    _load().oracle_quantize_rows_asym(_ptr(x), rows, cols, _ptr(mask), _ptr(codes), _ptr(scale), _ptr(zero))
+    clamped = _load().oracle_quantize_rows_asym(_ptr(x), rows, cols, _ptr(mask), _ptr(codes), _ptr(scale),
+                                                _ptr(zero))
+    if return_clamped:
+        return codes, scale, zero, int(clamped)
     return codes, scale, zero
 
 

@@ -42,9 +42,18 @@ def test_quantize_asym_matches_oracle(lib, dev, oracle_mod, M, K, nout, t):
     X16[M // 2] += np.float16(0.75)  # a row whose range is not symmetric about 0
     if M > 3:
         X16[1] = 0                   # an all-zero row
-    codes, scale, zero, bm = lib.quantize_rowwise_asym(to_dev(X16, dev), t)
+    # A row on [-1, 1] reaching both ends: s = 127.5, z = 128 and the code of
+    # 1.0 lands on 256 before the clamp (the oracle counts it below).
+    # (Its values stay below t, so the outlier columns do not change; its two
+    # ends go to columns outside them.)
+    crow = M - 1
+    X16[crow] = np.clip(X16[crow], -1, 1)
     mask = oracle_mod.outlier_mask(X16, t) if t > 0 else np.zeros(K, np.uint8)
-    c_ref, s_ref, z_ref = oracle_mod.quantize_rowwise_asym(X16, mask)
+    c_lo, c_hi = np.flatnonzero(mask == 0)[[0, -1]]
+    X16[crow, c_lo], X16[crow, c_hi] = -1.0, 1.0
+    codes, scale, zero, bm = lib.quantize_rowwise_asym(to_dev(X16, dev), t)
+    c_ref, s_ref, z_ref, clamped = oracle_mod.quantize_rowwise_asym(X16, mask, return_clamped=True)
+    assert clamped >= 1 and c_ref[crow, c_hi] == 127 and z_ref[crow] == 128
     if t > 0:
         assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
     assert np.array_equal(scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))

@@ -6,8 +6,12 @@ fp16 output satisfies |y - y_ref| <= 1e-2 + 2e-3 |y_ref| elementwise, with
 y_ref the oracle's fp64 value.
 
 Sizes here span several 128x256 output tiles with ragged edges in M, N and
-K, so the oracle finishes in seconds; the full-size workloads are compared on
-sampled rows and columns the oracle computes one by one.
+K, so the oracle finishes in seconds. The full-size workloads (prefill,
+decode and the four BLOOM block linears) are compared in full too: codes,
+row absmax, outlier set and weight codes against the oracle, the int32
+accumulators against the oracle's product (decode; prefill under the `slow`
+mark) or cuBLAS's on the oracle's codes, and every fp16 output against the
+oracle's output step on those accumulators.
 """
 import numpy as np
 import pytest
@@ -506,12 +510,18 @@ def test_cuda_graph_capture(lib, dev):
     assert torch.equal(Y, ref)
 
 
-# ------------------------------------------------------------------ full-size workloads, sampled
+# ------------------------------------------------------------------ full-size workloads, in full
 
-def sampled_check(lib, dev, oracle_mod, X, W, t, give_w16, rows, cols):
-    """Run the layer on device tensors X [M x K] and W [N x K]; compare the
-    outlier set and SX in full, CX / acc / Y on the sampled rows x columns,
-    and CB / SB on the sampled weight rows, against the oracle on host copies."""
+def full_check(lib, dev, oracle_mod, X, W, t, give_w16, rows, cols, acc_ref="int_mm"):
+    """Run the layer on device tensors X [M x K] and W [N x K] and compare it
+    with the oracle on host copies, every element:
+      - the outlier set, SX (fp32 bits), CX, CB and SB, against the oracle;
+      - the int32 accumulators: acc_ref="oracle" against the oracle's own
+        int8 product; acc_ref="int_mm" against torch._int_mm (cuBLAS, an
+        independent library routine) applied to the ORACLE's CX and CB, with
+        the oracle's own product checked on the sampled rows x columns;
+      - Y against the oracle's output step (dequantization plus the outlier
+        product, fp64) evaluated on that exact accumulator."""
     M, K = X.shape
     N = W.shape[0]
     CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
@@ -525,20 +535,37 @@ def sampled_check(lib, dev, oracle_mod, X, W, t, give_w16, rows, cols):
     Xh = X.cpu().numpy()
     O = oracle_mod.outlier_cols(Xh, t)
     n = int(dbg["count"].item())
-    assert np.array_equal(dbg["col_idx"][:n].cpu().numpy(), O)
-    cx_ref, sx_ref = oracle_mod.quantize_rowwise(Xh[rows], O)
-    assert np.array_equal(dbg["row_absmax"].cpu().numpy()[rows].view(np.uint32), sx_ref.view(np.uint32))
-    assert np.array_equal(dbg["codes"][rows].cpu().numpy(), cx_ref)
-    Wh = W[cols].cpu().numpy()
+    assert np.array_equal(dbg["col_idx"][:n].cpu().numpy(), O), "outlier columns"
+    cx_ref, sx_ref = oracle_mod.quantize_rowwise(Xh, O)
+    assert np.array_equal(dbg["row_absmax"].cpu().numpy().view(np.uint32), sx_ref.view(np.uint32)), "SX bits"
+    assert np.array_equal(dbg["codes"].cpu().numpy(), cx_ref), "activation codes"
+    del dbg["codes"]
+    Wh = W.cpu().numpy()
     cb_ref, sb_ref = oracle_mod.quantize_weight(Wh)
-    assert np.array_equal(CB[cols].cpu().numpy(), cb_ref)
-    assert np.array_equal(SCB[cols].cpu().numpy().view(np.uint32), sb_ref.view(np.uint32))
-    acc_ref = oracle_mod.int8_matmul(cx_ref, cb_ref)
-    acc = dbg["acc"][rows][:, cols].cpu().numpy()
-    assert np.array_equal(acc, acc_ref)
-    wt = oracle_mod.outlier_weight(O, len(cols), K, W=Wh if give_w16 else None, CB=cb_ref, SB=sb_ref)
-    y_ref = oracle_mod.mixed_output(acc_ref, sx_ref, sb_ref, Xh[rows], O, wt)
-    assert_y_close(Y[rows][:, cols].cpu().numpy(), y_ref, "Y sampled")
+    assert np.array_equal(CB.cpu().numpy(), cb_ref), "weight codes"
+    assert np.array_equal(SCB.cpu().numpy().view(np.uint32), sb_ref.view(np.uint32)), "weight absmax bits"
+    acc = dbg["acc"].cpu().numpy()
+    del dbg["acc"]
+    if acc_ref == "oracle":
+        acc_full = oracle_mod.int8_matmul(cx_ref, cb_ref)
+    else:
+        assert oracle_mod.int8_matmul(cx_ref[rows], cb_ref[cols]).tolist() == acc[rows][:, cols].tolist(), \
+            "int32 accumulators (oracle, sampled)"
+        a_dev = torch.from_numpy(cx_ref).to(dev)
+        b_dev = torch.from_numpy(cb_ref).to(dev).t().contiguous()
+        acc_full = torch._int_mm(a_dev, b_dev).cpu().numpy()
+        del a_dev, b_dev
+    assert np.array_equal(acc, acc_full), "int32 accumulators"
+    # W's outlier columns through the oracle, handed only those columns (a
+    # gather, no arithmetic) so that it does not widen the whole weight again
+    sel = np.arange(O.size, dtype=np.int64)
+    wt = oracle_mod.outlier_weight(sel, N, O.size, W=np.ascontiguousarray(Wh[:, O]) if give_w16 else None,
+                                   CB=np.ascontiguousarray(cb_ref[:, O]), SB=sb_ref)
+    del Wh
+    y_ref = oracle_mod.mixed_output(acc_full, sx_ref, sb_ref, Xh, O, wt)
+    assert_y_close(Y.cpu().numpy(), y_ref, "Y")
+    del CB, SCB, Y, dbg
+    torch.cuda.empty_cache()
     return O
 
 
@@ -549,36 +576,56 @@ def _samples(M, N, seed, nrows=8, ncols=96):
     return rows, cols
 
 
-def test_prefill_workload_sampled(lib, dev, oracle_mod):
-    """Prefill, 7B-class: X [2048 x 4096] with 4 columns x60, W [16384 x 4096]."""
+def test_prefill_workload_full(lib, dev, oracle_mod):
+    """Prefill, 7B-class: X [2048 x 4096] with 4 columns x60, W [16384 x 4096],
+    every output element; the accumulators against cuBLAS on the oracle's codes."""
     lin = synthetic.PREFILL_7B.linears[0]
     X16, cols = make_activations(lin, seed=0)
     W16 = make_weight(lin, seed=0)
     X, W = to_dev(X16, dev), to_dev(W16, dev)
     rows, jcols = _samples(lin.M, lin.N, 3)
-    O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols)
+    O = full_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols)
     assert set(cols.tolist()) <= set(O.tolist())
 
 
+@pytest.mark.slow
+def test_prefill_workload_full_oracle_product(lib, dev, oracle_mod):
+    """The same prefill workload with the int32 accumulators compared in full
+    against the oracle's own int8 product (137 G multiply-adds of plain C:
+    about a minute)."""
+    lin = synthetic.PREFILL_7B.linears[0]
+    X16, _ = make_activations(lin, seed=0)
+    W16 = make_weight(lin, seed=0)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    rows, jcols = _samples(lin.M, lin.N, 3)
+    full_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols, acc_ref="oracle")
+
+
 @pytest.mark.parametrize("M", [1, 8, 32])
-def test_decode_workload_sampled(lib, dev, oracle_mod, M):
+def test_decode_workload_full(lib, dev, oracle_mod, M):
     """Decode at BLOOM width: X [M x 14336], W int8-prequantized [14336 x 14336]
-    (outlier columns of W recovered as CB * SCB / 127)."""
+    (outlier columns of W recovered as CB * SCB / 127), every output against
+    the oracle's own int8 product."""
     lin = synthetic.decode_bloom(M).linears[0]
     X, W, cols = synthetic.torch_device_problem(lin, seed=M, device=dev)
     rows, jcols = _samples(lin.M, lin.N, M, ncols=160)
-    O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, False, rows, jcols)
+    O = full_check(lib, dev, oracle_mod, X, W, 6.0, False, rows, jcols, acc_ref="oracle")
     if M >= 16:
         assert set(cols.tolist()) <= set(O.tolist())
+    del X, W
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name", ["qkv", "attn_out", "fc1", "fc2"])
-def test_bloom_block_linear_sampled(lib, dev, oracle_mod, name):
+def test_bloom_block_linear_full(lib, dev, oracle_mod, name):
+    """The four BLOOM-176B block linears at 2048 tokens, every element; the
+    accumulators against cuBLAS on the oracle's codes, and against the
+    oracle's own product on sampled rows x columns."""
     lin = {l.name: l for l in synthetic.BLOOM_BLOCK_2048.linears}[name]
     seed = {"qkv": 11, "attn_out": 12, "fc1": 13, "fc2": 14}[name]
     X, W, cols = synthetic.torch_device_problem(lin, seed=seed, device=dev)
     rows, jcols = _samples(lin.M, lin.N, 7, nrows=6, ncols=64)
-    O = sampled_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols)
+    O = full_check(lib, dev, oracle_mod, X, W, 6.0, True, rows, jcols)
     assert set(cols.tolist()) <= set(O.tolist())
     del X, W
     torch.cuda.empty_cache()
@@ -586,6 +633,5 @@ def test_bloom_block_linear_sampled(lib, dev, oracle_mod, name):
 
 def test_status_word_clean(lib, dev):
     """No kernel reported a timed-out wait during this module."""
-    from int8_mixed_precision_rowwise_b200 import _workspaces
-    for ws in _workspaces.values():
+    for ws in lib.workspaces():
         assert lib.read_status(ws, clear=False) == 0

@@ -348,6 +348,23 @@ def test_asym_worked_vector_uses_the_full_unsigned_range(oracle_mod):
     assert np.all(np.abs(back - x) <= 0.5 / s[0] * (1 + 1e-6))
 
 
+def test_asym_clamp_catches_the_code_one_past_the_range(oracle_mod):
+    """The two separate roundings of the zero-point reading can step past
+    [0, 255]: for the row [-1, 1] the range is 2, s = 127.5 exactly,
+    z = rint(127.5) = 128 (half to even) and rint(1 * 127.5) = 128, so the
+    maximum lands on 128 + 128 = 256 before the clamp. The oracle must count
+    exactly that one clamp and store q = 255; the minimum lands on
+    rint(-127.5) + 128 = 0 with no clamp. The absmax worked vector needs none."""
+    x = np.array([[-1.0, 1.0, 0.0, 0.5]], dtype=np.float32)
+    c, s, z, clamped = oracle_mod.quantize_rowwise_asym(x, return_clamped=True)
+    q = c.astype(np.int32) + 128
+    assert s[0] == np.float32(127.5) and z[0] == 128
+    assert clamped == 1
+    assert q[0].tolist() == [0, 255, 128, 192]     # 0.5 * 127.5 = 63.75 -> 64, + 128
+    w = np.array([[1.2, -0.5, -4.3, 1.2, -3.1, 0.8, 2.4, 5.4]], dtype=np.float32)
+    assert oracle_mod.quantize_rowwise_asym(w, return_clamped=True)[3] == 0
+
+
 def test_asym_zero_is_exact_and_ranges_include_zero(oracle_mod):
     """0 is represented exactly (q = z dequantizes to 0) whatever the signs of
     the row, including all-positive and all-negative rows."""
