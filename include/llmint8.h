@@ -295,6 +295,92 @@ LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, cons
                                     llmint8_stream_t stream);
 
 /*
+ * Tensor parallelism: the pieces a linear split over several GPUs needs (page
+ * "优化故事：Bloom 推理", section "支持 TP": every GPU owns a part of the
+ * weights; the parts are combined with NCCL all-reduces, section "唾手可得的
+ * 优化"). The collectives themselves are the caller's (NCCL); these calls
+ * are the per-GPU steps around them. Each split reproduces the one-GPU
+ * result of [S]/[M]: the same outlier set, row absmax and codes.
+ *   - Column split (rows of W across GPUs): llmint8_matmul_mixed on the full X
+ *     and this GPU's rows of CB/SCB/W; outputs are column blocks, put back in
+ *     place by llmint8_gather_column_blocks after an all-gather.
+ *   - Row split (K across GPUs; CB/SCB quantized over the FULL rows of W):
+ *     llmint8_quantize_rowwise on this GPU's columns of X gives its outlier
+ *     bitmap and the row absmax over its other columns; a max all-reduce of
+ *     that absmax gives the full one; llmint8_quantize_rowwise_given codes the
+ *     columns with it; llmint8_find_outlier_cols lists the outlier columns;
+ *     llmint8_matmul_codes writes an fp32 partial product; a sum all-reduce
+ *     adds the partials and llmint8_bias_act_to_f16 applies bias, activation
+ *     and the single fp16 rounding.
+ *   - Token split (rows of X across GPUs, W replicated): every GPU's outlier
+ *     bitmap is all-gathered; llmint8_quantize_rowwise_given codes this GPU's
+ *     rows against their union; llmint8_matmul_codes gives its rows of Y.
+ */
+
+/* Output types of llmint8_matmul_codes. */
+#define LLMINT8_OUT_F16 0
+#define LLMINT8_OUT_F32 1
+
+/*
+ * Row-wise absmax quantization against a GIVEN outlier set ([Q], [M]).
+ *   X_f16          (device) fp16 [rows x cols], cols a multiple of 16.
+ *   outlier_bitmaps (device) uint32 [n_bitmaps x ceil(cols/32)]: the outlier
+ *                  set is the OR of the n_bitmaps bitmaps (n_bitmaps = 0: no
+ *                  outlier columns; the pointer may then be NULL).
+ *   row_absmax_in  (device, may be NULL) fp32 [rows]: if given, row i is
+ *                  coded with this absmax (e.g. the max all-reduced over the
+ *                  GPUs of a row split) and row_absmax_out is not written;
+ *                  if NULL, the absmax over the columns outside the set is
+ *                  computed and written to row_absmax_out (then required).
+ *   codes          (device) int8 [rows x cols] out: round-half-even(x * s),
+ *                  s = 127 / absmax in fp32 (0 for absmax 0); 0 in set columns.
+ *   bitmap_out     (device, may be NULL) uint32 [ceil(cols/32)] out: the union.
+ * No workspace. Errors: as llmint8_quantize_rowwise; n_bitmaps > 4096 or
+ * neither row_absmax pointer given is LLMINT8_ERR_INVALID_ARG.
+ */
+LLMINT8_API llmint8_status llmint8_quantize_rowwise_given(const void *X_f16, int64_t rows, int64_t cols,
+                                              const uint32_t *outlier_bitmaps, int n_bitmaps,
+                                              const float *row_absmax_in, int8_t *codes, float *row_absmax_out,
+                                              uint32_t *bitmap_out, llmint8_stream_t stream);
+
+/*
+ * The int8 GEMM with the LLM.int8() epilogue ([Q], [S], [M], [U]) on codes
+ * quantized beforehand:
+ *   Y[i,j] = act( acc[i,j] * SX[i] * SCB[j] / 127^2
+ *                 + sum_{c in O} X[i,c] * Wt[j,c] + bias[j] ),  acc = CX . CB^T (int32),
+ * with O the first *d_count entries of col_idx and Wt as in
+ * llmint8_matmul_mixed.
+ *   CX (device) int8 [M x K], SX (device) fp32 [M]: X's codes and row absmax
+ *   X_f16 (device) fp16 [M x K]: read only at the outlier columns
+ *   CB, SCB, W_f16 (may be NULL): as llmint8_matmul_mixed
+ *   col_idx (device) int32 [>= *d_count], d_count (device) int32 [1]: the
+ *       outlier columns (llmint8_find_outlier_cols), read on the device
+ *   bias_f16 (device, may be NULL), activation: as llmint8_matmul_mixed_ex
+ *   out_dtype LLMINT8_OUT_F16: Y fp16 [M x N]; LLMINT8_OUT_F32: Y fp32 [M x N]
+ *       (an unrounded partial sum, e.g. of a row split)
+ *   workspace (device) >= 256 bytes, zeroed once (only its status word is used)
+ * Errors as llmint8_matmul_mixed_ex; a bad out_dtype is LLMINT8_ERR_INVALID_ARG.
+ */
+LLMINT8_API llmint8_status llmint8_matmul_codes(const int8_t *CX, const float *SX, const void *X_f16, int64_t M,
+                                    int64_t K, const int8_t *CB, const float *SCB, const void *W_f16, int64_t N,
+                                    const int32_t *col_idx, const int32_t *d_count, const void *bias_f16,
+                                    int activation, int out_dtype, void *Y, void *workspace, size_t ws_bytes,
+                                    llmint8_stream_t stream);
+
+/* Y_f16[i,j] = fp16( act( Y32[i,j] + bias[j] ) ) in fp32 (the last step of a
+ * row split, after the partial outputs are summed). Y32 (device) fp32
+ * [M x N], N a multiple of 4; bias_f16 (device, may be NULL) fp16 [N];
+ * activation as llmint8_matmul_mixed_ex; Y_f16 (device) fp16 [M x N]. */
+LLMINT8_API llmint8_status llmint8_bias_act_to_f16(const float *Y32, int64_t M, int64_t N, const void *bias_f16,
+                                       int activation, void *Y_f16, llmint8_stream_t stream);
+
+/* dst[i, p*Nr + j] = src[p][i][j]: the column blocks [P][M x Nr] of a column
+ * split (as an all-gather leaves them) into one fp16 [M x P*Nr] matrix.
+ * src, dst (device) fp16, 16-byte aligned, Nr a multiple of 8. */
+LLMINT8_API llmint8_status llmint8_gather_column_blocks(const void *src_f16, int64_t P, int64_t M, int64_t Nr,
+                                            void *dst_f16, llmint8_stream_t stream);
+
+/*
  * Allocation-free row-wise quantizer. The source page has no counterpart: it
  * exists for callers that cannot allocate device memory, such as a server
  * that reserved all device memory for its own pool at start-up, a plugin in a

@@ -21,7 +21,8 @@ __all__ = [
     "gemm_s8s8s32", "Int8MixedLinear", "DEFAULT_THRESHOLD", "quantize_rowwise_noalloc", "noalloc_read_status",
     "matmul_mixed_fp16w",
     "workspace_size_fp16w", "ACTIVATIONS", "quantize_rowwise_asym", "code_row_sums", "workspace_size_asym",
-    "matmul_mixed_asym", "MAX_K_ASYM",
+    "matmul_mixed_asym", "MAX_K_ASYM", "quantize_rowwise_given", "matmul_codes", "bias_act_to_f16",
+    "gather_column_blocks", "OUT_F16", "OUT_F32", "outlier_bitmap",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libllmint8.so")
@@ -29,6 +30,7 @@ DEFAULT_THRESHOLD = 6.0
 MAX_K_ASYM = 132104  # LLMINT8_MAX_K_ASYM
 
 OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(7)
+OUT_F16, OUT_F32 = 0, 1  # LLMINT8_OUT_*
 
 class _Debug(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("row_absmax", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
@@ -58,6 +60,11 @@ _SIGNATURES = {
     "llmint8_gemm_s8s8s32": (_ST, [_P, _I64, _P, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
     "llmint8_quantize_rowwise_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
     "llmint8_noalloc_read_status": (_ST, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]),
+    "llmint8_quantize_rowwise_given": (_ST, [_P, _I64, _I64, _P, ctypes.c_int, _P, _P, _P, _P, _P]),
+    "llmint8_matmul_codes": (_ST, [_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, ctypes.c_int, ctypes.c_int,
+                                   _P, _P, ctypes.c_size_t, _P]),
+    "llmint8_bias_act_to_f16": (_ST, [_P, _I64, _I64, _P, ctypes.c_int, _P, _P]),
+    "llmint8_gather_column_blocks": (_ST, [_P, _I64, _I64, _I64, _P, _P]),
     "llmint8_quantize_rowwise_asym": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                             _P]),
     "llmint8_code_row_sums": (_ST, [_P, _I64, _I64, _P, _P]),
@@ -243,6 +250,17 @@ def quantize_rowwise_noalloc(X, threshold: float = 0.0, codes=None, row_absmax=N
                                      row_absmax.data_ptr(), _ptr(outlier_bitmap), _stream_ptr(dev)),
            "llmint8_quantize_rowwise_noalloc")
     return codes, row_absmax, outlier_bitmap
+
+
+def outlier_bitmap(X, threshold: float, out=None):
+    """int32 [ceil(cols/32)]: the outlier columns of fp16 X (all clear for
+    threshold <= 0 or no rows). The quantizer computes it; its codes and row
+    absmax are dropped."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    if out is None:
+        out = torch.empty((X.shape[1] + 31) // 32, dtype=torch.int32, device=X.device)
+    return quantize_rowwise(X, threshold, outlier_bitmap=out)[2]
 
 
 def find_outlier_cols(outlier_bitmap, cols: int, col_idx=None, d_count=None, sync_count: bool = True):
@@ -452,3 +470,98 @@ def matmul_mixed_asym(X, CB, SCB, CB_row_sums, W_f16=None, threshold: float = DE
                                         ctypes.byref(dbg) if dbg else None, _stream_ptr(dev)),
            "llmint8_matmul_mixed_asym")
     return Y
+
+
+# ---- tensor-parallel pieces (page "优化故事：Bloom 推理", section "支持 TP") ----------
+
+def quantize_rowwise_given(X, outlier_bitmaps=None, row_absmax=None, codes=None, row_absmax_out=None,
+                           bitmap_out=None):
+    """(codes int8 [rows x cols], row absmax fp32 [rows], union bitmap int32 words) of
+    fp16 X against a given outlier set: the OR of the bitmaps in
+    ``outlier_bitmaps`` (int32 [n, ceil(cols/32)] or [ceil(cols/32)], or None
+    for none). With ``row_absmax`` given (fp32 [rows], e.g. all-reduced over a
+    row split) the rows are coded with it and it is returned; otherwise the
+    absmax over the non-outlier columns is computed
+    (llmint8_quantize_rowwise_given)."""
+    torch = _torch()
+    _need_cuda(X, "X", torch.float16)
+    rows, cols = X.shape
+    dev = X.device
+    nw = (cols + 31) // 32
+    nbm = 0
+    if outlier_bitmaps is not None:
+        _need_cuda(outlier_bitmaps, "outlier_bitmaps", torch.int32)
+        if outlier_bitmaps.numel() % nw:
+            raise ValueError("outlier_bitmaps must hold whole bitmaps of ceil(cols/32) words")
+        nbm = outlier_bitmaps.numel() // nw
+    if row_absmax is not None:
+        _need_cuda(row_absmax, "row_absmax", torch.float32)
+    if codes is None:
+        codes = torch.empty((rows, cols), dtype=torch.int8, device=dev)
+    if row_absmax is None and row_absmax_out is None:
+        row_absmax_out = torch.empty(rows, dtype=torch.float32, device=dev)
+    if bitmap_out is None:
+        bitmap_out = torch.empty(nw, dtype=torch.int32, device=dev)
+    _check(load()["_quantize_rowwise_given"](X.data_ptr(), rows, cols, _ptr(outlier_bitmaps), nbm, _ptr(row_absmax),
+                                             codes.data_ptr(), _ptr(row_absmax_out), bitmap_out.data_ptr(),
+                                             _stream_ptr(dev)), "llmint8_quantize_rowwise_given")
+    return codes, (row_absmax if row_absmax is not None else row_absmax_out), bitmap_out
+
+
+def matmul_codes(CX, SX, X, CB, SCB, col_idx, d_count, W_f16=None, bias=None, activation=None, out_f32=False,
+                 Y=None, workspace=None):
+    """Y [M x N] (fp16, or fp32 with ``out_f32``) = the LLM.int8() GEMM and
+    epilogue on codes quantized beforehand: CX int8 [M x K], SX fp32 [M], X
+    fp16 [M x K] (outlier values), CB/SCB/W_f16 as matmul_mixed, the outlier
+    columns in col_idx int32 [K] / d_count int32 [1] (llmint8_matmul_codes)."""
+    torch = _torch()
+    _need_cuda(CX, "CX", torch.int8)
+    _need_cuda(SX, "SX", torch.float32)
+    _need_cuda(X, "X", torch.float16)
+    _need_cuda(CB, "CB", torch.int8)
+    _need_cuda(SCB, "SCB", torch.float32)
+    _need_cuda(col_idx, "col_idx", torch.int32)
+    _need_cuda(d_count, "d_count", torch.int32)
+    if W_f16 is not None:
+        _need_cuda(W_f16, "W_f16", torch.float16)
+    if bias is not None:
+        _need_cuda(bias, "bias", torch.float16)
+    if activation not in ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(k for k in ACTIVATIONS if k)} or None")
+    M, K = CX.shape
+    N = CB.shape[0]
+    dev = CX.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32 if out_f32 else torch.float16, device=dev)
+    ws = workspace if workspace is not None else get_workspace(4096, dev)
+    _check(load()["_matmul_codes"](CX.data_ptr(), SX.data_ptr(), X.data_ptr(), M, K, CB.data_ptr(), SCB.data_ptr(),
+                                   _ptr(W_f16), N, col_idx.data_ptr(), d_count.data_ptr(), _ptr(bias),
+                                   ACTIVATIONS[activation], OUT_F32 if out_f32 else OUT_F16, Y.data_ptr(),
+                                   ws.data_ptr(), ws.numel(), _stream_ptr(dev)), "llmint8_matmul_codes")
+    return Y
+
+
+def bias_act_to_f16(Y32, bias=None, activation=None, Y=None):
+    """fp16 act(Y32 + bias) of an fp32 [M x N] sum (llmint8_bias_act_to_f16)."""
+    torch = _torch()
+    _need_cuda(Y32, "Y32", torch.float32)
+    if bias is not None:
+        _need_cuda(bias, "bias", torch.float16)
+    M, N = Y32.shape
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=Y32.device)
+    _check(load()["_bias_act_to_f16"](Y32.data_ptr(), M, N, _ptr(bias), ACTIVATIONS[activation], Y.data_ptr(),
+                                      _stream_ptr(Y32.device)), "llmint8_bias_act_to_f16")
+    return Y
+
+
+def gather_column_blocks(blocks, out=None):
+    """fp16 [M x P*Nr] from column blocks fp16 [P, M, Nr] (llmint8_gather_column_blocks)."""
+    torch = _torch()
+    _need_cuda(blocks, "blocks", torch.float16)
+    P, M, Nr = blocks.shape
+    if out is None:
+        out = torch.empty((M, P * Nr), dtype=torch.float16, device=blocks.device)
+    _check(load()["_gather_column_blocks"](blocks.data_ptr(), P, M, Nr, out.data_ptr(), _stream_ptr(blocks.device)),
+           "llmint8_gather_column_blocks")
+    return out

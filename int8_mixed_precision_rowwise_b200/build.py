@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libllmint8.so")
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "decode.cu", "tp.cu", "noalloc.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "common.cuh"]
 
 NVCC_FLAGS = [

@@ -193,8 +193,9 @@ llmint8_status llmint8_quantize_rowwise(const void *X_f16, int64_t rows, int64_t
     const size_t need = carve(static_cast<char *>(workspace), rows, cols, false, false, &ws);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
-    if (rows == 0)
-        return LLMINT8_OK;
+    if (rows == 0) // no rows, no outlier columns: the bitmap is still written
+        return outlier_bitmap ? cuda_status(cudaMemsetAsync(outlier_bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream))
+                              : LLMINT8_OK;
     DeviceInfo dev;
     cudaError_t e = device_info(&dev);
     if (e != cudaSuccess)
@@ -481,8 +482,9 @@ llmint8_status llmint8_quantize_rowwise_asym(const void *X_f16, int64_t rows, in
     const size_t need = carve(static_cast<char *>(workspace), rows, cols, false, false, &ws);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
-    if (rows == 0)
-        return LLMINT8_OK;
+    if (rows == 0) // no rows, no outlier columns: the bitmap is still written
+        return outlier_bitmap ? cuda_status(cudaMemsetAsync(outlier_bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream))
+                              : LLMINT8_OK;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess)
         return LLMINT8_ERR_CUDA;

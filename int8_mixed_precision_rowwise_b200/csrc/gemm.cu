@@ -61,6 +61,7 @@ struct KParams {
     // Zero-point codes of X (null: absmax codes): sx holds the scale s per
     // row, zx the zero point, rsum the code row sums of W.
     const int32_t *zx, *rsum;
+    int out_f32;               // MixedFp16 epilogue: store fp32 (1) instead of fp16 (0)
 };
 
 template <int BN, int STAGES>
@@ -419,7 +420,19 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                         y[c] = bias_act(y[c], bv, p.act);
                     }
                 }
-                if (i < p.M) {
+                if (i < p.M && p.out_f32) {
+                    // fp32 partial output (tensor-parallel row split: summed across ranks afterwards)
+                    float *Yr = reinterpret_cast<float *>(p.Y) + (int64_t)i * p.N;
+                    if (j0 + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4)
+                            *reinterpret_cast<float4 *>(Yr + j0 + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
+                    } else {
+                        for (int c = 0; c < 32; ++c)
+                            if (j0 + c < p.N)
+                                Yr[j0 + c] = y[c];
+                    }
+                } else if (i < p.M) {
                     __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
                     if (j0 + 32 <= p.N && (p.N & 7) == 0) {
 #pragma unroll
@@ -511,7 +524,13 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                     for (int c = 0; c < BN; ++c)
                         y[c] = bias_act(y[c], bv, p.act);
                 }
-                if (j < p.N) {
+                if (j < p.N && p.out_f32) {
+                    float *Yc = reinterpret_cast<float *>(p.Y) + j;
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        if (brow0 + c < p.M)
+                            Yc[(int64_t)(brow0 + c) * p.N] = y[c];
+                } else if (j < p.N) {
                     __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
 #pragma unroll
                     for (int c = 0; c < BN; ++c)
@@ -1071,6 +1090,7 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     p.status = a.status;
     p.zx = a.zx;
     p.rsum = a.rsum;
+    p.out_f32 = a.out_f32;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int grid = std::min(tiles, dev.num_sms);
     return launch_dependent(kern, grid, L::ALLOC, stream, ta, tb, p);
@@ -1114,6 +1134,7 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.status = a.status;
     p.zx = a.zx;
     p.rsum = a.rsum;
+    p.out_f32 = a.out_f32;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int pairs = std::min(tiles, dev.num_sms / 2);
     return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, p);

@@ -174,6 +174,9 @@ struct GemmArgs {
     // per row, zx the zero point per row, rsum the code row sums of B.
     const int32_t *zx;
     const int32_t *rsum;
+    // MixedFp16 epilogue only: 1 stores Y as fp32 [M x N] (a partial sum of a
+    // tensor-parallel row split), 0 as fp16.
+    int out_f32;
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, const DeviceInfo &dev, cudaStream_t stream);

@@ -93,8 +93,11 @@ extern "C" llmint8_status llmint8_quantize_rowwise_noalloc(const void *X_f16, in
     if (!aligned16(X_f16) || !aligned16(codes) || !aligned16(row_absmax) ||
         (outlier_bitmap && !aligned16(outlier_bitmap)))
         return LLMINT8_ERR_ALIGNMENT;
-    if (rows == 0)
-        return LLMINT8_OK;
+    if (rows == 0) // no rows, no outlier columns: the bitmap is still written
+        return (!outlier_bitmap ||
+                cudaMemsetAsync(outlier_bitmap, 0, (size_t)((cols + 31) / 32) * 4, stream) == cudaSuccess)
+                   ? LLMINT8_OK
+                   : LLMINT8_ERR_CUDA;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess)
         return LLMINT8_ERR_CUDA;

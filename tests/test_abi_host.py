@@ -168,8 +168,8 @@ def test_quantize_argument_errors(lib):
     assert q(A, 32, 64, 6.0, A, A, None, A, ws, None) == lib.ERR_INVALID_ARG     # bitmap needed when t > 0
     assert q(A, 32, 64, 6.0, A, A + 1, A, A, ws, None) == lib.ERR_ALIGNMENT
     assert q(A, 32, 64, 6.0, A, A, A, A, 16, None) == lib.ERR_WORKSPACE
-    assert q(A, 0, 64, 6.0, A, A, A, A, ws, None) == lib.OK
-    assert q(A, 0, 64, 0.0, A, A, None, A, ws, None) == lib.OK                   # no bitmap when t <= 0
+    assert q(A, 0, 64, 0.0, A, A, None, A, ws, None) == lib.OK                   # no rows, no bitmap: nothing queued
+    # (no rows with a bitmap queues one memset of it: a GPU test covers that)
 
 
 def test_find_outlier_cols_argument_errors(lib):
@@ -197,3 +197,34 @@ def test_no_cpu_fallback(lib):
         lib.quantize_rowwise(X, 6.0)
     with pytest.raises(TypeError):
         lib.matmul_mixed(X, torch.zeros((4, 16), dtype=torch.int8), torch.zeros(4))
+
+
+def test_tensor_parallel_argument_errors(lib):
+    """The tensor-parallel pieces check their arguments before queuing work."""
+    qg = lib._quantize_rowwise_given
+    assert qg(A, 32, 64, A, 1, None, A, None, None, None) == lib.ERR_INVALID_ARG   # no absmax in or out
+    assert qg(A, 32, 64, None, 2, None, A, A, None, None) == lib.ERR_INVALID_ARG   # bitmaps missing
+    assert qg(A, 32, 60, None, 0, None, A, A, None, None) == lib.ERR_UNSUPPORTED_SHAPE
+    assert qg(A, 32, 64, A + 4, 1, None, A, A, None, None) == lib.ERR_ALIGNMENT
+    assert qg(A, 0, 64, None, 0, None, A, A, None, None) == lib.OK                 # no rows, no bitmap_out
+    mc = lib._matmul_codes
+
+    def call(out=lib.OUT_F16, wsb=256, K=128, Y=A, cnt=A, act=0):
+        return mc(A, A, A, 64, K, A, A, None, 64, A, cnt, None, act, out, Y, A, wsb, None)
+
+    assert call(out=2) == lib.ERR_INVALID_ARG
+    assert call(act=5) == lib.ERR_INVALID_ARG
+    assert call(cnt=None) == lib.ERR_INVALID_ARG
+    assert call(cnt=A + 2) == lib.ERR_ALIGNMENT
+    assert call(Y=A + 8) == lib.ERR_ALIGNMENT
+    assert call(wsb=64) == lib.ERR_WORKSPACE
+    assert call(K=100) == lib.ERR_UNSUPPORTED_SHAPE
+    ba = lib._bias_act_to_f16
+    assert ba(A, 8, 10, None, 0, A, None) == lib.ERR_UNSUPPORTED_SHAPE              # N % 4
+    assert ba(A, 8, 16, None, 2, A, None) == lib.ERR_INVALID_ARG
+    assert ba(A + 4, 8, 16, None, 0, A, None) == lib.ERR_ALIGNMENT
+    assert ba(A, 0, 16, None, 0, A, None) == lib.OK
+    gc = lib._gather_column_blocks
+    assert gc(A, 2, 8, 12, A, None) == lib.ERR_UNSUPPORTED_SHAPE                   # Nr % 8
+    assert gc(None, 2, 8, 16, A, None) == lib.ERR_INVALID_ARG
+    assert gc(A, 0, 8, 16, A, None) == lib.OK

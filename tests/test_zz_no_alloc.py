@@ -47,7 +47,7 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert f(A, 16, 65536 + 16, 6.0, A, A, A, None) == L.ERR_UNSUPPORTED_SHAPE
     assert f(A, 16, 1000, 6.0, A, A, A, None) == L.ERR_UNSUPPORTED_SHAPE   # cols % 16
     assert f(A, 16, 1024, 6.0, A, A, None, None) == L.ERR_INVALID_ARG      # bitmap needed for t > 0
-    assert f(A, 0, 1024, 6.0, A, A, A, None) == L.OK                       # empty: nothing queued
+    assert f(A, 0, 1024, 0.0, A, A, None, None) == L.OK                    # empty, no bitmap: nothing queued
     assert _status_fn(L.LIB_PATH)(0, None) == L.ERR_INVALID_ARG             # status reader needs `out`
 
 
