@@ -336,7 +336,9 @@ LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, cons
  *                  s = 127 / absmax in fp32 (0 for absmax 0); 0 in set columns.
  *   bitmap_out     (device, may be NULL) uint32 [ceil(cols/32)] out: the union.
  * No workspace. Errors: as llmint8_quantize_rowwise; n_bitmaps > 4096 or
- * neither row_absmax pointer given is LLMINT8_ERR_INVALID_ARG.
+ * neither row_absmax pointer given (rows > 0) is LLMINT8_ERR_INVALID_ARG.
+ * With rows == 0 only bitmap_out is written (X, codes and the absmax pointers
+ * may be NULL).
  */
 LLMINT8_API llmint8_status llmint8_quantize_rowwise_given(const void *X_f16, int64_t rows, int64_t cols,
                                               const uint32_t *outlier_bitmaps, int n_bitmaps,

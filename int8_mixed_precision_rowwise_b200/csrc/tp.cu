@@ -165,7 +165,9 @@ llmint8_status llmint8_quantize_rowwise_given(const void *X_f16, int64_t rows, i
         return st;
     if (rows > INT32_MAX || rows * cols > (int64_t)1 << 40)
         return LLMINT8_ERR_UNSUPPORTED_SHAPE;
-    if (!X_f16 || !codes || (n_bitmaps > 0 && !outlier_bitmaps) || (!row_absmax_in && !row_absmax_out))
+    // (with no rows, X, codes and the absmax pointers may be NULL: empty tensors)
+    if ((rows > 0 && (!X_f16 || !codes || (!row_absmax_in && !row_absmax_out))) ||
+        (n_bitmaps > 0 && !outlier_bitmaps))
         return LLMINT8_ERR_INVALID_ARG;
     if (!aligned16(X_f16) || !aligned16(codes) || (outlier_bitmaps && !aligned16(outlier_bitmaps)) ||
         (row_absmax_in && !aligned16(row_absmax_in)) || (row_absmax_out && !aligned16(row_absmax_out)) ||
