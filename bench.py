@@ -672,6 +672,22 @@ def run_profile_case(args):
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_pop()
         return
+    if args.profile_case.startswith("cublas_int8_"):
+        # cuBLAS's int8 GEMM (torch._int_mm) on a BLOOM linear's shape: the
+        # library kernel the measured int8 peak comes from, for comparison.
+        lin = {l.name: l for l in WORKLOAD.linears}[args.profile_case[len("cublas_int8_"):]]
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        A = torch.randint(-127, 128, (lin.M, lin.K), generator=g, device=dev, dtype=torch.int8)
+        B = torch.randint(-127, 128, (lin.N, lin.K), generator=g, device=dev, dtype=torch.int8).t()
+        torch._int_mm(A, B)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("timed_steps")
+        for _ in range(args.steps):
+            torch._int_mm(A, B)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        return
     if args.profile_case.startswith("decode_M"):
         lin = synthetic.decode_bloom(int(args.profile_case[len("decode_M"):])).linears[0]
         X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
@@ -714,7 +730,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--profile-case", default=None,
                     help="ncu driver: run only this BLOOM linear ('qkv', 'attn_out', 'fc1', 'fc2' or 'all'), "
-                         "the 4096 x 4096 'quantizer', or 'decode_M1' / 'decode_M8' / 'decode_M32'")
+                         "the 4096 x 4096 'quantizer', 'decode_M1' / 'decode_M8' / 'decode_M32', or "
+                         "cuBLAS's int8 GEMM on a linear's shape ('cublas_int8_attn_out', ...)")
     args = ap.parse_args()
     if args.profile_case:
         run_profile_case(args)

@@ -108,6 +108,24 @@ llmint8_status copy_debug(const llmint8_debug *dbg, const Workspace &ws, int64_t
     return LLMINT8_OK;
 }
 
+// The fused-epilogue GEMM of a linear. Prefill shapes (more than
+// kDecodeMaxM rows) with the workspace's gather regions first copy the outlier
+// operands into them, so that the epilogue stages each tile by bulk copies.
+cudaError_t gather_then_gemm(GemmArgs g, const Workspace &ws, const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (ws.wt_t && g.M > kDecodeMaxM) {
+        cudaError_t e = launch_gather_outliers(g, ws.wt_t, ws.sb_p, ws.xo_t, ws.np, ws.mp, dev, stream);
+        if (e != cudaSuccess)
+            return e;
+        g.wt_t = ws.wt_t;
+        g.sb_p = ws.sb_p;
+        g.xo_t = ws.xo_t;
+        g.np = ws.np;
+        g.mp = ws.mp;
+    }
+    return launch_gemm(g, dev, stream);
+}
+
 } // namespace
 
 extern "C" {
@@ -139,7 +157,8 @@ size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K)
 {
     if (M < 0 || N < 0 || K < 0)
         return 0;
-    return carve(nullptr, M, K, true, decode_shape(M, N), nullptr);
+    const bool dec = decode_shape(M, N);
+    return carve(nullptr, M, K, true, dec, nullptr, dec ? 0 : N);
 }
 
 size_t llmint8_workspace_size_fp16w(int64_t M, int64_t N, int64_t K)
@@ -277,7 +296,8 @@ llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, 
             return LLMINT8_ERR_ALIGNMENT;
     }
     Workspace ws;
-    const size_t need = carve(static_cast<char *>(workspace), M, K, true, decode_shape(M, N), &ws);
+    const bool dec = decode_shape(M, N);
+    const size_t need = carve(static_cast<char *>(workspace), M, K, true, dec, &ws, dec ? 0 : N);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
     if (M == 0 || N == 0)
@@ -337,7 +357,7 @@ llmint8_status llmint8_matmul_mixed_ex(const void *X_f16, int64_t M, int64_t K, 
     if (dbg && dbg->gemm_begin &&
         cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    if ((e = launch_gemm(g, dev, stream)) != cudaSuccess)
+    if ((e = gather_then_gemm(g, ws, dev, stream)) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     if (dbg && dbg->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
@@ -378,7 +398,8 @@ llmint8_status llmint8_matmul_mixed_fp16w(const void *X_f16, int64_t M, int64_t 
     int8_t *cb = reinterpret_cast<int8_t *>(w + base);
     float *sb = reinterpret_cast<float *>(w + base + align256((size_t)N * (size_t)K));
     Workspace ws;
-    carve(w, M, K, true, decode_shape(M, N), &ws);
+    const bool dec = decode_shape(M, N);
+    carve(w, M, K, true, dec, &ws, dec ? 0 : N);
     if (launch_quantize(W_f16, N, K, 0.f, cb, sb, nullptr, ws.col_idx, ws.count, ws.sync, ws.status, dev,
                         stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
@@ -457,8 +478,7 @@ size_t llmint8_workspace_size_asym(int64_t M, int64_t N, int64_t K)
 {
     if (M < 0 || N < 0 || K < 0)
         return 0;
-    (void)N;
-    return align256(carve(nullptr, M, K, true, false, nullptr)) + align256((size_t)M * 4);
+    return align256(carve(nullptr, M, K, true, false, nullptr, N)) + align256((size_t)M * 4);
 }
 
 llmint8_status llmint8_quantize_rowwise_asym(const void *X_f16, int64_t rows, int64_t cols, float threshold,
@@ -546,7 +566,7 @@ llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K
             return LLMINT8_ERR_ALIGNMENT;
     }
     Workspace ws;
-    const size_t base = align256(carve(static_cast<char *>(workspace), M, K, true, false, &ws));
+    const size_t base = align256(carve(static_cast<char *>(workspace), M, K, true, false, &ws, N));
     if (ws_bytes < base + align256((size_t)M * 4))
         return LLMINT8_ERR_WORKSPACE;
     int32_t *zx = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + base);
@@ -586,7 +606,7 @@ llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K
     if (dbg && dbg->gemm_begin &&
         cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    if ((e = launch_gemm(g, dev, stream)) != cudaSuccess)
+    if ((e = gather_then_gemm(g, ws, dev, stream)) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     if (dbg && dbg->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;

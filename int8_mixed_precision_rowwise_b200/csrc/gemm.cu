@@ -43,6 +43,7 @@ constexpr int BM = 128;       // MMA M: rows of the A operand per tile
 constexpr int BK = 128;       // K bytes per pipeline stage (one 128-byte swizzle row)
 constexpr int UK = 32;        // K per tcgen05.mma kind::i8
 constexpr int OC = 32;        // outlier columns staged per chunk in the epilogue
+static_assert(OC == kGatherCols, "the gathered staging fills s_side for up to OC columns");
 constexpr int NTHREADS = 192; // 6 warps
 constexpr float kInv127Sq = 1.0f / 16129.0f;
 
@@ -62,6 +63,11 @@ struct KParams {
     // row, zx the zero point, rsum the code row sums of W.
     const int32_t *zx, *rsum;
     int out_f32;               // MixedFp16 epilogue: store fp32 (1) instead of fp16 (0)
+    // Gathered outlier operands (null: gathered in place): W's outlier columns
+    // [kGatherCols x np] and SB [np] (staged per tile by bulk copies), X's
+    // outlier columns [kGatherCols x mp] (read per row).
+    const float *wt_t, *sb_p, *xo_t;
+    int np, mp;
 };
 
 template <int BN, int STAGES>
@@ -74,7 +80,7 @@ struct Smem {
     static constexpr int SCALE_OFF = SIDE_OFF + OC * BN * 4;           // float [BN]
     static constexpr int COLS_OFF = SCALE_OFF + BN * 4;                // int [OC] outlier columns
     static constexpr int BAR_OFF = COLS_OFF + OC * 4;                  // uint64 barriers
-    static constexpr int NBARS = 2 * STAGES + 5;                       // full, empty, tfull[2], tempty[2], drain
+    static constexpr int NBARS = 2 * STAGES + 6; // full, empty, tfull[2], tempty[2], drain, staging
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;               // tmem base, abort flag
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;                         // slack for 1024-byte alignment
@@ -165,7 +171,7 @@ __device__ __forceinline__ void stage_issue(const KParams &p, const int *s_cols,
 template <int BN, bool SWAP, bool RAW, bool PAIR>
 __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lane, float *s_side, float *s_scale,
                                              int *s_cols,
-                                             uint32_t tfull0, uint32_t tempty0, volatile int *s_abort,
+                                             uint32_t tfull0, uint32_t tempty0, uint32_t sbar, volatile int *s_abort,
                                              uint32_t tmem_base, int first_tile, int tile_step, int num_tiles,
                                              int a_tile_rows, int a_row_off)
 {
@@ -189,7 +195,31 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
     // them takes several microseconds, longer than a K = 4096 tile's MMAs).
     static_assert(RAW || SWAP || OC * BN >= (kPipeGather + kPipeCols) * 128,
                   "the pipelined staging keeps W's values and X's values in s_side");
-    const bool pipe = !RAW && !SWAP && fast && cnt <= kPipeCols && cnt * BN <= kPipeGather * 128;
+    // Gathered operands (a kernel before this one copied W's and X's outlier
+    // columns into contiguous arrays): the tile's slice of W's columns and of
+    // SB arrive by bulk copies on `sbar`, issued by one thread as soon as the
+    // previous tile's epilogue is done with s_side; no per-thread gathers run
+    // next to the MMAs.
+    const bool gathered = !RAW && !SWAP && p.wt_t != nullptr && fast;
+    // X's values of the CTA's 128 rows follow W's in s_side when both fit
+    const bool x_in_smem = gathered && cnt * (BN + 128) <= OC * BN;
+    const bool pipe = !gathered && !RAW && !SWAP && fast && cnt <= kPipeCols && cnt * BN <= kPipeGather * 128;
+    uint32_t sph = 0u;
+    bool staged_pending = false; // (thread et == 0) a staging copy is in flight
+    auto issue_staging = [&](int tile) {
+        const int brow0 = (tile / p.num_m_blk) * BN;
+        const int arow0 = (tile % p.num_m_blk) * a_tile_rows + a_row_off;
+        mbar_arrive_expect_tx(sbar, (uint32_t)(cnt + 1) * BN * 4u + (x_in_smem ? (uint32_t)cnt * 512u : 0u));
+        for (int k = 0; k < cnt; ++k)
+            bulk_load(smem_u32(s_side + k * BN), p.wt_t + (int64_t)k * p.np + brow0, BN * 4u, sbar);
+        if (x_in_smem)
+            for (int k = 0; k < cnt; ++k)
+                bulk_load(smem_u32(s_side + cnt * BN + k * 128), p.xo_t + (int64_t)k * p.mp + arow0, 512u, sbar);
+        bulk_load(smem_u32(s_scale), p.sb_p + brow0, BN * 4u, sbar);
+        staged_pending = true;
+    };
+    if (gathered && et == 0 && first_tile < num_tiles)
+        issue_staging(first_tile);
     StageRegs<BN> nx;
     if (pipe && first_tile < num_tiles)
         stage_issue<BN>(p, s_cols, cnt, first_tile, a_tile_rows, a_row_off, r_in_tile, et, nx);
@@ -204,7 +234,24 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
 #pragma unroll
         for (int k = 0; k < OC; ++k)
             own_side[k] = 0.f;
-        if (pipe) {
+        if (gathered) {
+            own_scale = arow < p.M ? p.sx[arow] : 0.f;
+            if (!x_in_smem) {
+                // too many columns for s_side: this row's outlier values into
+                // registers, one coalesced load per column
+#pragma unroll
+                for (int k = 0; k < OC; ++k)
+                    own_side[k] = (k < cnt && arow < p.M) ? __ldg(p.xo_t + (int64_t)k * p.mp + arow) : 0.f;
+            }
+            const bool landed = mbar_wait(sbar, sph);
+            if (named_barrier_or(1, 128, !landed)) {
+                if (!landed)
+                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                break;
+            }
+            sph ^= 1u;
+            staged_pending = false;
+        } else if (pipe) {
             named_barrier_sync(1, 128); // the previous tile's readers are done with s_side / s_scale
 #pragma unroll
             for (int u = 0; u < (BN + 127) / 128; ++u)
@@ -358,7 +405,23 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                     for (int c = 0; c < 32; ++c)
                         y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
                 }
-                if (pipe) {
+                if (gathered && x_in_smem) {
+                    // X's outlier values of this row, staged in s_side after W's
+                    const float *xs = s_side + cnt * BN + r_in_tile; // staged in row order
+#pragma unroll 1
+                    for (int k = 0; k < cnt; ++k) {
+                        const float xv = xs[k * 128];
+                        const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 w = wrow[c4];
+                            y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                            y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                            y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                            y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                        }
+                    }
+                } else if (pipe) {
                     // A loop over the actual columns: the form unrolled over
                     // OC below is about 1300 instructions per chunk, more
                     // than the instruction cache keeps next to the rest.
@@ -376,7 +439,7 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                             y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
                         }
                     }
-                } else if (fast) {
+                } else if (fast) { // (gathered with X's values in registers, or gathered in place)
 #pragma unroll
                     for (int k = 0; k < OC; ++k) {
                         if (k < cnt) {
@@ -547,7 +610,19 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
             else
                 mbar_arrive(tempty_bar(b));
         }
+        if (gathered) {
+            // every reader of s_side / s_scale is done: stage the next tile
+            named_barrier_sync(1, 128);
+            if (et == 0 && tile + tile_step < num_tiles) {
+                fence_proxy_async_smem();
+                issue_staging(tile + tile_step);
+            }
+        }
     }
+    // A staging copy still in flight (the loop was left early) lands before
+    // the CTA may exit.
+    if (gathered && et == 0 && staged_pending)
+        mbar_wait(sbar, sph);
 }
 
 template <int BN, int STAGES, bool SWAP, bool RAW>
@@ -570,6 +645,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    const uint32_t stage_bar = bar0 + 8u * (2 * STAGES + 5);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -583,6 +659,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(tempty_bar(b), 4); // one arrival per epilogue warp
         }
         mbar_init(drain_bar, 1);
+        mbar_init(stage_bar, 1);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -718,7 +795,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
         run_epilogue<BN, SWAP, RAW, false>(p, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
-                                           s_abort,
+                                           stage_bar, s_abort,
                                            tmem_base, blockIdx.x, gridDim.x, num_tiles, BM, 0);
     }
 
@@ -745,7 +822,7 @@ struct SmemPair {
     static constexpr int SCALE_OFF = SIDE_OFF + OC * BN * 4;
     static constexpr int COLS_OFF = SCALE_OFF + BN * 4;
     static constexpr int BAR_OFF = COLS_OFF + OC * 4;
-    static constexpr int NBARS = 2 * STAGES + 5;
+    static constexpr int NBARS = 2 * STAGES + 6;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;
@@ -789,6 +866,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    const uint32_t stage_bar = bar0 + 8u * (2 * STAGES + 5);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -802,6 +880,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             mbar_init(tempty_bar(b), 8); // 4 epilogue warps in each CTA
         }
         mbar_init(drain_bar, 1);
+        mbar_init(stage_bar, 1);         // this CTA's epilogue staging copies
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -939,7 +1018,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
         run_epilogue<BN, false, RAW, true>(p, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
-                                           s_abort,
+                                           stage_bar, s_abort,
                                            tmem_base, pair_id, num_pairs, num_tiles, 2 * BM, (int)rank * BM);
     }
 
@@ -948,6 +1027,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+    }
+}
+
+// The epilogue's outlier operands, gathered once per call (launch_gather_outliers):
+// wt_t[k][j] = Wt[j, col_k] (the fp16 weight, or CB * SB / 127 per output row,
+// in fp32), xo_t[k][i] = X[i, col_k], sb_p[j] = SB[j], zero past N, for the
+// first |O| <= kGatherCols outlier columns (none written for more: the
+// epilogue then gathers in place). One element a thread, so that every
+// scattered read is in flight at once.
+__global__ void __launch_bounds__(256)
+    k_gather_outliers(const KParams p, float *__restrict__ wt_t, float *__restrict__ sb_p, float *__restrict__ xo_t)
+{
+    __shared__ int s_c[kGatherCols];
+    griddep_wait(); // the quantizer's outlier list
+    griddep_release();
+    const int cnt = min(*p.count, p.K);
+    const int kk = cnt <= kGatherCols ? cnt : 0;
+    if ((int)threadIdx.x < kGatherCols)
+        s_c[threadIdx.x] = (int)threadIdx.x < kk ? p.col_idx[threadIdx.x] : 0;
+    __syncthreads();
+    const int64_t per = (int64_t)p.np + p.mp; // items of one outlier column
+    const int64_t total = (int64_t)(kk > 0 ? kk : 1) * per;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total;
+         t += (int64_t)gridDim.x * blockDim.x) {
+        const int k = (int)(t / per);
+        const int64_t r = t - (int64_t)k * per;
+        if (r < p.np) {
+            const int j = (int)r;
+            const bool in = j < p.N;
+            if (k == 0)
+                sb_p[j] = in ? p.sb[j] : 0.f;
+            if (kk > 0)
+                wt_t[(int64_t)k * p.np + j] = in ? wtilde(p, j, s_c[k]) : 0.f;
+        } else if (kk > 0) {
+            const int i = (int)(r - p.np);
+            if (i < p.M)
+                xo_t[(int64_t)k * p.mp + i] = __half2float(p.X16[(int64_t)i * p.K + s_c[k]]);
+        }
     }
 }
 
@@ -1091,6 +1208,11 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     p.zx = a.zx;
     p.rsum = a.rsum;
     p.out_f32 = a.out_f32;
+    p.wt_t = SWAP ? nullptr : a.wt_t;
+    p.sb_p = a.sb_p;
+    p.xo_t = a.xo_t;
+    p.np = (int)a.np;
+    p.mp = (int)a.mp;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int grid = std::min(tiles, dev.num_sms);
     return launch_dependent(kern, grid, L::ALLOC, stream, ta, tb, p);
@@ -1135,6 +1257,11 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.zx = a.zx;
     p.rsum = a.rsum;
     p.out_f32 = a.out_f32;
+    p.wt_t = a.wt_t;
+    p.sb_p = a.sb_p;
+    p.xo_t = a.xo_t;
+    p.np = (int)a.np;
+    p.mp = (int)a.mp;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int pairs = std::min(tiles, dev.num_sms / 2);
     return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, p);
@@ -1203,6 +1330,36 @@ cudaError_t run_prefill(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t s
 }
 
 } // namespace
+
+cudaError_t launch_gather_outliers(const GemmArgs &a, float *wt_t, float *sb_p, float *xo_t, int64_t np, int64_t mp,
+                                   const DeviceInfo &dev, cudaStream_t stream)
+{
+    KParams p{};
+    p.K = (int)a.K;
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.sb = a.sb;
+    p.X16 = reinterpret_cast<const __half *>(a.X16);
+    p.W16 = reinterpret_cast<const __half *>(a.W16);
+    p.CB = a.B;
+    p.col_idx = a.col_idx;
+    p.count = a.count;
+    p.np = (int)np;
+    p.mp = (int)mp;
+    const int64_t total = (int64_t)kGatherCols * (np + mp);
+    const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)dev.num_sms * 8);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_gather_outliers, p, wt_t, sb_p, xo_t);
+}
 
 cudaError_t launch_gemm(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
 {

@@ -17,6 +17,13 @@ constexpr int kDecodeMaxM = 32;
 constexpr int kDecodeMaxCtas = 160;
 constexpr int kHeaderBytes = 256;
 constexpr size_t kSetWords = (LLMINT8_MAX_K + 31) / 32; // bitmap words of the widest X
+// Outlier columns whose operands the prefill GEMM's epilogue reads from
+// per-call gathered copies (more columns: it gathers them in place).
+constexpr int kGatherCols = 32;
+// Row strides (in floats) of the gathered copies: the W side leaves room for
+// a whole last tile (up to 256 columns past N), both are 16-byte multiples.
+inline int64_t gather_stride_n(int64_t N) { return (N + 256 + 3) / 4 * 4; }
+inline int64_t gather_stride_m(int64_t M) { return (M + 3) / 4 * 4; }
 
 // Workspace layout (byte offsets; every region 256-byte aligned):
 //   [0]      uint32 status word (bits LLMINT8_DEV_*)
@@ -42,6 +49,10 @@ constexpr size_t kSetWords = (LLMINT8_MAX_K + 31) / 32; // bitmap words of the w
 //   ...      int32  partial accumulators per CTA [kDecodeMaxCtas x kDecodeMaxM x 128]
 //   ...      uint32 partial-ready flags per CTA [kDecodeMaxCtas] (tagged with the
 //            call's grid-barrier generation, so never cleared)
+//   prefill GEMM (gather_n > 0), rewritten by each call before it is read:
+//   ...      fp32   W's outlier columns, column-major [kGatherCols x np] (np = gather_stride_n(N))
+//   ...      fp32   SB, zero-padded [np]
+//   ...      fp32   X's outlier columns, column-major [kGatherCols x mp] (mp = gather_stride_m(M))
 struct Workspace {
     uint32_t *status;
     int32_t *count;
@@ -57,6 +68,10 @@ struct Workspace {
     float *prow;
     int32_t *slots;
     uint32_t *pflags;
+    float *wt_t;      // null without the gather regions
+    float *sb_p;
+    float *xo_t;
+    int64_t np, mp;
     size_t bytes;
 };
 
@@ -66,8 +81,10 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool decode_shape(int64_t M, int64_t N) { return M >= 1 && M <= kDecodeMaxM && N >= 1; }
 
 // Lay out (base != null) or size a workspace; `decode` adds the regions of
-// the fused decode kernel.
-inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool decode, Workspace *ws)
+// the fused decode kernel, gather_n > 0 those of the prefill GEMM's gathered
+// outlier operands for an N-row weight.
+inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool decode, Workspace *ws,
+                    int64_t gather_n = 0)
 {
     size_t off = 0;
     auto take = [&](size_t n) {
@@ -86,6 +103,11 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
     char *pr = decode ? take((size_t)kDecodeMaxCtas * kDecodeMaxM * 4) : nullptr;
     char *sl = decode ? take((size_t)kDecodeMaxCtas * kDecodeMaxM * 128 * 4) : nullptr;
     char *pf = decode ? take((size_t)kDecodeMaxCtas * 4) : nullptr;
+    const int64_t np = gather_n > 0 ? gather_stride_n(gather_n) : 0;
+    const int64_t mp = gather_n > 0 ? gather_stride_m(M) : 0;
+    char *wt = gather_n > 0 ? take((size_t)kGatherCols * np * 4) : nullptr;
+    char *sp = gather_n > 0 ? take((size_t)np * 4) : nullptr;
+    char *xo = gather_n > 0 ? take((size_t)kGatherCols * mp * 4) : nullptr;
     if (ws) {
         ws->status = reinterpret_cast<uint32_t *>(hdr);
         ws->count = hdr ? reinterpret_cast<int32_t *>(hdr + 4) : nullptr;
@@ -101,6 +123,11 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
         ws->prow = reinterpret_cast<float *>(pr);
         ws->slots = reinterpret_cast<int32_t *>(sl);
         ws->pflags = reinterpret_cast<uint32_t *>(pf);
+        ws->wt_t = reinterpret_cast<float *>(wt);
+        ws->sb_p = reinterpret_cast<float *>(sp);
+        ws->xo_t = reinterpret_cast<float *>(xo);
+        ws->np = np;
+        ws->mp = mp;
         ws->bytes = off;
     }
     return off;
@@ -177,9 +204,20 @@ struct GemmArgs {
     // MixedFp16 epilogue only: 1 stores Y as fp32 [M x N] (a partial sum of a
     // tensor-parallel row split), 0 as fp16.
     int out_f32;
+    // Gathered outlier operands (launch_gather_outliers; null: the epilogue
+    // gathers W's and X's outlier values in place).
+    const float *wt_t, *sb_p, *xo_t;
+    int64_t np, mp;
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, const DeviceInfo &dev, cudaStream_t stream);
+
+// Before the prefill GEMM, once per call: W's outlier columns (the fp16 W, or
+// CB * SB / 127 per row) and X's, column-major into the workspace's gather
+// regions, and SB zero-padded, when |O| <= kGatherCols. Launched as a
+// programmatic dependent of the quantizer (it waits for its outlier list).
+cudaError_t launch_gather_outliers(const GemmArgs &args, float *wt_t, float *sb_p, float *xo_t, int64_t np,
+                                   int64_t mp, const DeviceInfo &dev, cudaStream_t stream);
 
 // The whole LLM.int8() linear for at most kDecodeMaxM tokens in one kernel:
 // outlier detection, quantization of X, the int8 product streamed over all

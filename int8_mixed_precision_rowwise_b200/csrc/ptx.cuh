@@ -165,6 +165,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
+// Order this thread's earlier generic-proxy accesses of shared memory before
+// its later async-proxy ones (a bulk copy that overwrites what was read).
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- dependent launch
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel in the stream still runs; griddep_wait() blocks until
