@@ -71,6 +71,7 @@ typedef enum llmint8_status {
 #define LLMINT8_DEV_TIMEOUT_MMA 0x2u
 #define LLMINT8_DEV_TIMEOUT_EPILOGUE 0x4u
 #define LLMINT8_DEV_TIMEOUT_QUANT 0x8u
+#define LLMINT8_DEV_BAD_STORE 0x10u /* an epilogue store failed its self-check and was skipped */
 
 /* Human-readable name of a status code. Never NULL. */
 LLMINT8_API const char *llmint8_status_string(int status);

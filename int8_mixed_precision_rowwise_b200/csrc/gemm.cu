@@ -43,6 +43,7 @@ constexpr int BM = 128;       // MMA M: rows of the A operand per tile
 constexpr int BK = 128;       // K bytes per pipeline stage (one 128-byte swizzle row)
 constexpr int UK = 32;        // K per tcgen05.mma kind::i8
 constexpr int OC = 32;        // outlier columns staged per chunk in the epilogue
+constexpr int kStoreStage = 16384; // bytes at the end of s_side for the TMA-store staging (4 warps x 4 KB)
 static_assert(OC == kGatherCols, "the gathered staging fills s_side for up to OC columns");
 constexpr int NTHREADS = 192; // 6 warps
 constexpr float kInv127Sq = 1.0f / 16129.0f;
@@ -68,6 +69,7 @@ struct KParams {
     // outlier columns [kGatherCols x mp] (read per row).
     const float *wt_t, *sb_p, *xo_t;
     int np, mp;
+    int y_tma;                 // Y (fp16) has a TMA store map (tmY): 32-row x 64-column boxes
 };
 
 template <int BN, int STAGES>
@@ -169,8 +171,8 @@ __device__ __forceinline__ void stage_issue(const KParams &p, const int *s_cols,
 }
 
 template <int BN, bool SWAP, bool RAW, bool PAIR>
-__device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lane, float *s_side, float *s_scale,
-                                             int *s_cols,
+__device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap *tmY, int warp, int lane,
+                                             float *s_side, float *s_scale, int *s_cols,
                                              uint32_t tfull0, uint32_t tempty0, uint32_t sbar, volatile int *s_abort,
                                              uint32_t tmem_base, int first_tile, int tile_step, int num_tiles,
                                              int a_tile_rows, int a_row_off)
@@ -204,6 +206,14 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
     // X's values of the CTA's 128 rows follow W's in s_side when both fit
     const bool x_in_smem = gathered && cnt * (BN + 128) <= OC * BN;
     const bool pipe = !gathered && !RAW && !SWAP && fast && cnt <= kPipeCols && cnt * BN <= kPipeGather * 128;
+    // Output through shared memory and TMA stores (coalesced, async) when the
+    // staged operands leave the last 16 KB of s_side (OC * BN floats) free:
+    // each warp stages its 32 rows x 64 columns (fp16, 128-byte swizzle,
+    // 4 KB, 1024-byte aligned) there.
+    constexpr int kSideBytes = OC * BN * 4;
+    const bool tma_st = x_in_smem && p.y_tma && !p.out_f32 && cnt * (BN + 128) * 4 + kStoreStage <= kSideBytes;
+    uint8_t *obuf = reinterpret_cast<uint8_t *>(s_side) + (kSideBytes - kStoreStage) + q * 4096;
+    bool stores_pending = false; // (lane 0) TMA stores of this warp not yet complete
     uint32_t sph = 0u;
     bool staged_pending = false; // (thread et == 0) a staging copy is in flight
     auto issue_staging = [&](int tile) {
@@ -495,6 +505,45 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
                             if (j0 + c < p.N)
                                 Yr[j0 + c] = y[c];
                     }
+                } else if (tma_st && (g | 1) < BN / 32) {
+                    // chunk g is half of a full 64-column group: into this
+                    // warp's staging buffer (row = lane, 16-byte pieces
+                    // swizzled by row), and the group out by one TMA store
+                    if ((g & 1) == 0) {
+                        if (lane == 0 && stores_pending)
+                            bulk_wait_group_read0(); // the previous group has left obuf
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 pk;
+                        __half2 *h = reinterpret_cast<__half2 *>(&pk);
+                        h[0] = __floats2half2_rn(y[8 * c8 + 0], y[8 * c8 + 1]);
+                        h[1] = __floats2half2_rn(y[8 * c8 + 2], y[8 * c8 + 3]);
+                        h[2] = __floats2half2_rn(y[8 * c8 + 4], y[8 * c8 + 5]);
+                        h[3] = __floats2half2_rn(y[8 * c8 + 6], y[8 * c8 + 7]);
+                        const int piece = ((g & 1) * 4 + c8) ^ (lane & 7);
+                        *reinterpret_cast<uint4 *>(obuf + lane * 128 + piece * 16) = pk;
+                    }
+                    if (g & 1) {
+                        fence_proxy_async_smem(); // this lane's pieces, before the async proxy reads them
+                        __syncwarp();
+                        // (a box entirely past M or N has nothing to write; a
+                        // staging buffer off its 1024-byte alignment or outside
+                        // s_side, or a column not on a 16-byte boundary, is
+                        // reported and not stored)
+                        const int x0 = brow0 + (g - 1) * 32, y0 = arow - lane;
+                        const uint32_t ob = smem_u32(obuf), sb0 = smem_u32(s_side);
+                        const bool sane = (ob & 1023u) == 0 && ob >= sb0 && ob + 4096u <= sb0 + kSideBytes &&
+                                          (x0 & 7) == 0 && x0 >= 0 && y0 >= 0;
+                        if (lane == 0 && !sane)
+                            atomicOr(p.status, LLMINT8_DEV_BAD_STORE);
+                        if (lane == 0 && sane && y0 < p.M && x0 < p.N) {
+                            tma_store_2d(tmY, ob, x0, y0);
+                            bulk_commit_group();
+                            stores_pending = true;
+                        }
+                    }
                 } else if (i < p.M) {
                     __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
                     if (j0 + 32 <= p.N && (p.N & 7) == 0) {
@@ -619,15 +668,18 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, int warp, int lan
             }
         }
     }
-    // A staging copy still in flight (the loop was left early) lands before
-    // the CTA may exit.
+    // A staging copy still in flight (the loop was left early) lands, and
+    // this warp's TMA stores complete, before the CTA may exit.
     if (gathered && et == 0 && staged_pending)
         mbar_wait(sbar, sph);
+    if (lane == 0 && stores_pending)
+        bulk_wait_group0();
 }
 
 template <int BN, int STAGES, bool SWAP, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    k_gemm_i8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const KParams p)
+    k_gemm_i8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmY, const KParams p)
 {
     using L = Smem<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -670,6 +722,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.y_tma)
+            tma_prefetch_desc(&tmY);
     }
     tc_fence_before();
     __syncthreads();
@@ -794,7 +848,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
-        run_epilogue<BN, SWAP, RAW, false>(p, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
+        run_epilogue<BN, SWAP, RAW, false>(p, &tmY, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
                                            stage_bar, s_abort,
                                            tmem_base, blockIdx.x, gridDim.x, num_tiles, BM, 0);
     }
@@ -846,7 +900,7 @@ struct SmemPair {
 template <int BN, int STAGES, int KS, bool RAW>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     k_gemm_i8_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const KParams p)
+                   const __grid_constant__ CUtensorMap tmY, const KParams p)
 {
     using L = SmemPair<BN, STAGES, KS>;
     extern __shared__ uint8_t smem_raw[];
@@ -891,6 +945,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.y_tma)
+            tma_prefetch_desc(&tmY);
     }
     tc_fence_before();
     cluster_sync_all(); // barriers and TMEM of both CTAs ready before any cross-CTA traffic
@@ -1017,7 +1073,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
-        run_epilogue<BN, false, RAW, true>(p, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
+        run_epilogue<BN, false, RAW, true>(p, &tmY, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
                                            stage_bar, s_abort,
                                            tmem_base, pair_id, num_pairs, num_tiles, 2 * BM, (int)rank * BM);
     }
@@ -1075,7 +1131,7 @@ __global__ void __launch_bounds__(256)
 // before reading that kernel's output).
 template <typename Kern>
 cudaError_t launch_dependent(Kern kern, int grid, int smem, cudaStream_t stream, const CUtensorMap &ta,
-                             const CUtensorMap &tb, const KParams &p)
+                             const CUtensorMap &tb, const CUtensorMap &ty, const KParams &p)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -1087,7 +1143,7 @@ cudaError_t launch_dependent(Kern kern, int grid, int smem, cudaStream_t stream,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+    return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p);
 }
 
 } // namespace
@@ -1162,7 +1218,60 @@ bool make_map_i8(CUtensorMap *map, int device, const void *base, int64_t rows, i
     return true;
 }
 
+// Y fp16 [rows x cols] as a 2-D TMA map for the epilogue's stores: 64-column
+// (128-byte) x 32-row boxes, 128-byte swizzle; cached like the operand maps.
+bool make_map_y16(CUtensorMap *map, int device, const void *base, int64_t rows, int64_t cols)
+{
+    struct Entry {
+        int device;
+        const void *base;
+        int64_t rows, cols;
+        CUtensorMap map;
+    };
+    constexpr int kCache = 16;
+    static std::mutex mu;
+    static Entry cache[kCache];
+    static int used = 0, next = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i) {
+            const Entry &e = cache[i];
+            if (e.device == device && e.base == base && e.rows == rows && e.cols == cols) {
+                *map = e.map;
+                return true;
+            }
+        }
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry &e = cache[next];
+    e = Entry{device, base, rows, cols, *map};
+    next = (next + 1) % kCache;
+    used = used < kCache ? used + 1 : kCache;
+    return true;
+}
+
 namespace {
+
+// The fp16 output goes out by TMA stores when the epilogue produces fp16 and
+// Y's rows are 16-byte multiples (the map then describes it exactly).
+bool y_map(const GemmArgs &a, bool swap, const DeviceInfo &dev, CUtensorMap *ty)
+{
+    *ty = CUtensorMap{};
+    if (swap || a.epi != Epilogue::MixedFp16 || a.out_f32 || a.N % 8 != 0)
+        return false;
+    return make_map_y16(ty, dev.device, a.Y, a.M, a.N);
+}
 
 template <int BN, int STAGES, bool SWAP, bool RAW>
 cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
@@ -1213,9 +1322,11 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     p.xo_t = a.xo_t;
     p.np = (int)a.np;
     p.mp = (int)a.mp;
+    CUtensorMap ty;
+    p.y_tma = y_map(a, SWAP, dev, &ty) ? 1 : 0;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int grid = std::min(tiles, dev.num_sms);
-    return launch_dependent(kern, grid, L::ALLOC, stream, ta, tb, p);
+    return launch_dependent(kern, grid, L::ALLOC, stream, ta, tb, ty, p);
 }
 
 template <int BN, int STAGES, int KS, bool RAW>
@@ -1262,9 +1373,11 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.xo_t = a.xo_t;
     p.np = (int)a.np;
     p.mp = (int)a.mp;
+    CUtensorMap ty;
+    p.y_tma = y_map(a, false, dev, &ty) ? 1 : 0;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int pairs = std::min(tiles, dev.num_sms / 2);
-    return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, p);
+    return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, ty, p);
 }
 
 // Tile width for CTA-pair tiles (256 x BN): the one that minimises tile
