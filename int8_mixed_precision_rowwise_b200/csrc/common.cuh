@@ -63,6 +63,8 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 // rounded to nearest even, then rint() of it by adding 1.5 * 2^23 in
 // round-to-nearest-even (the low byte of the sum is the code). The two
 // roundings must stay separate (no fused multiply-add), as in the definition.
+// (Scalar on purpose: the packed fp32x2 multiply/add was checked on B200 and
+// gave different codes than the oracle for some values.)
 __device__ __forceinline__ uint2 codes8(const uint4 &v, float s)
 {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);

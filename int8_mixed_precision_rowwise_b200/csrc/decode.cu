@@ -619,6 +619,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
+    // Launched as a programmatic dependent: the set-up above overlapped the
+    // previous kernel's tail; nothing below reads or writes global memory
+    // before that kernel is complete.
+    griddep_wait();
     const int64_t G = gridDim.x, cta = blockIdx.x;
     const int64_t u0 = unit_begin(cta, p.units, G), u1 = unit_begin(cta + 1, p.units, G);
     const int64_t n = u1 - u0;
@@ -887,11 +891,13 @@ cudaError_t run_decode(const DecodeArgs &a, const DeviceInfo &dev, cudaStream_t 
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = L::ALLOC;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative; // the grid barrier needs every CTA resident
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization; // launch overlaps the previous tail
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
 }
 

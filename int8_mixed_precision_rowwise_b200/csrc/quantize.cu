@@ -328,6 +328,7 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     uint32_t *s_seed = s_dyn + nwords; // [nwords]
     uint32_t kb4[(V + 3) / 4];
     uint4 v[V];
+    griddep_wait();    // (a programmatic dependent) the previous kernel is complete
     griddep_release(); // the GEMM may start its weight stream now; it waits for this kernel's output
 
     if constexpr (!THR) {
@@ -507,11 +508,13 @@ cudaError_t launch_fused(const void *X, int64_t rows, int cols, float t, int8_t 
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative; // the barriers need every CTA resident
     attr[0].val.cooperative = THR ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization; // launch overlaps the previous tail
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const bool resident = (cols >> 3) <= 32 * WPR * V;
     const bool all_seeded = rows <= groups && (resident || seed_stride == 1);
     return cudaLaunchKernelEx(&cfg, kern, xp, rows, cols, t, t16, codes, absmax, bitmap, col_idx, count, sync,
@@ -544,15 +547,16 @@ cudaError_t launch_fused_v(const void *X, int64_t rows, int cols, float t, int8_
 // w, w + 15, ... as they land, a row in the warp's registers. Per row
 // (threshold on):
 //   detect - the row's outlier columns (|x| >= t16) join the CTA's set s_bm;
-//            a column new to it is also ORed (fire and forget) into this
-//            call's global bitmap, and then counted in s_cnt;
+//            a column new to it is counted in s_cnt;
 //   c      - the size of the set the row is quantized against: each lane
 //            caches the set bytes of its vectors, read after reading c, and
 //            reads them again when s_cnt has moved or the row added to it;
 //   row    - maximum over the columns outside the set, codes
 //            rint(x * 127 / absmax) (set columns 0) and absmax.
-// A control warp, once every row is detected, passes the grid barrier and
-// reads the complete set back. Sets only grow and every column counted in c
+// A control warp, once every row is detected, ORs the CTA's set into this
+// call's global bitmap, passes the grid barrier and reads the complete set
+// back. (The workers never wait for global memory: they start on the first
+// rows as soon as those land.) Sets only grow and every column counted in c
 // was in s_bm before the row read it, so a row whose c equals the size of
 // the complete set used exactly that set; the others (a column that only a
 // later row, or another CTA, saw) are quantized again from shared memory.
@@ -591,18 +595,18 @@ struct QsRow {
     __half t16;
     uint32_t *s_bm;  // the CTA's set (detection adds to it)
     int *s_cnt;      // its size
-    uint32_t *gset;  // this call's global bitmap
     int8_t *cr;      // the row's codes
     float *am;       // the row's absmax
     int lane;
 };
 
-// Add the outlier columns of vector v (x) to the CTA's set; columns new to
-// it are ORed into the global bitmap (no reply awaited), then counted.
-// Returns true if it added any. Out of line: it runs for the few vectors
-// holding an outlier, and inlined into every unrolled step it would crowd
-// the instruction cache that the common path runs from.
-__device__ __noinline__ bool qs_publish(uint4 x, int v, __half t16, uint32_t *s_bm, int *s_cnt, uint32_t *gset)
+// Add the outlier columns of vector v (x) to the CTA's set, then count the
+// ones new to it. (The control warp ORs the CTA's whole set into this call's
+// global bitmap once every row is detected.) Returns true if it added any.
+// Out of line: it runs for the few vectors holding an outlier, and inlined
+// into every unrolled step it would crowd the instruction cache that the
+// common path runs from.
+__device__ __noinline__ bool qs_publish(uint4 x, int v, __half t16, uint32_t *s_bm, int *s_cnt)
 {
     const uint32_t bits = hit_mask8(x, t16) << ((v & 3) * 8);
     const int w = v >> 2;
@@ -611,7 +615,6 @@ __device__ __noinline__ bool qs_publish(uint4 x, int v, __half t16, uint32_t *s_
         return false;
     __threadfence_block(); // the bits are in s_bm before the count says so
     atomicAdd(s_cnt, __popc(nb));
-    atomicOr(gset + w, nb); // after the fence: it would wait for this one to land
     return true;
 }
 
@@ -623,7 +626,7 @@ __device__ __forceinline__ __half2 qs_detect_vec(const QsRow &q, int v, const ui
     __half2 a[4];
     const __half2 m = vec_abs_max(x, a);
     if (__hge(__hmax(__low2half(m), __high2half(m)), q.t16) && (hit_mask8(x, q.t16) & ~known))
-        pub |= qs_publish(x, v, q.t16, q.s_bm, q.s_cnt, q.gset);
+        pub |= qs_publish(x, v, q.t16, q.s_bm, q.s_cnt);
     return m;
 }
 
@@ -674,12 +677,11 @@ __device__ __forceinline__ void qs_load_set(QsSetCache &sc, const uint32_t *bm, 
     sc.count = count;
 }
 
-// Before the warp's last arrival at the detection barrier: the lanes that
-// ORed into the global bitmap wait for those operations to land.
+// The warp's last arrival at the detection barrier (its rows' columns are in
+// the CTA's set; the barrier orders them before the control warp reads it).
 __device__ __forceinline__ void qs_arrive_detected(bool pub)
 {
-    if (pub)
-        __threadfence();
+    (void)pub;
     named_barrier_arrive(2, kQsThreads);
 }
 
@@ -727,7 +729,7 @@ __device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub,
             __half2 a[4];
             const __half2 mk = vec_abs_max(x[k], a);
             if (__hge(__hmax(__low2half(mk), __high2half(mk)), q.t16))
-                pub |= qs_publish(x[k], q.lane + 32 * k, q.t16, q.s_bm, q.s_cnt, q.gset);
+                pub |= qs_publish(x[k], q.lane + 32 * k, q.t16, q.s_bm, q.s_cnt);
         }
         qs_load_set(sc, q.s_bm, q.nvec, q.lane, qs_count(q));
         rm = __float2half2_rn(0.f);
@@ -778,6 +780,9 @@ __global__ void __launch_bounds__(kQsThreads, 1)
     const uint32_t xbytes = (uint32_t)nr * (uint32_t)cols * 2u;
     uint32_t *s_bm = reinterpret_cast<uint32_t *>(q_smem + ((xbytes + 15u) & ~15u)); // the CTA's set
     uint32_t *s_gbm = s_bm + nwords;                                                  // the complete set
+    // Launched as a programmatic dependent: the kernel before this one may
+    // still be finishing; nothing here touches global memory before it has.
+    griddep_wait();
     griddep_release();
 
     if (warp == kQsWarps) {
@@ -823,8 +828,6 @@ __global__ void __launch_bounds__(kQsThreads, 1)
                 s_target = a - a % (unsigned long long)G + (unsigned long long)G;
             }
         }
-        if (THR)
-            named_barrier_arrive(4, kQsThreads); // s_call and s_target are set
         if (lane == 0) {
             for (int j = kQsInFlight; j < nch; ++j) {
                 if (!mbar_wait(smem_u32(&s_bars[j - kQsInFlight]), 0u))
@@ -833,7 +836,25 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             }
         }
         if (THR) {
-            named_barrier_sync(2, kQsThreads); // every row detected, its new columns in the global bitmap
+            named_barrier_sync(2, kQsThreads); // every row detected, its columns in s_bm
+            __syncwarp();
+            const uint32_t call = __shfl_sync(0xffffffffu, s_call, 0);
+            // The CTA's set into this call's global bitmap (nonzero words only);
+            // CTA 0 also clears the other bitmap for the next call, which no
+            // CTA of this call reads.
+            uint32_t *myset = sets + (call & 1u) * kSetWords;
+            for (int w = lane; w < nwords; w += 32) {
+                const uint32_t b = s_bm[w];
+                if (b)
+                    atomicOr(myset + w, b);
+            }
+            if (c == 0) {
+                uint32_t *next = sets + ((call + 1u) & 1u) * kSetWords;
+                for (int w = lane; w < (int)kSetWords; w += 32)
+                    next[w] = 0u;
+            }
+            __threadfence(); // this lane's ORs (and clears) before lane 0's release below
+            __syncwarp();
             bool passed = true;
             if (lane == 0) {
                 // Grid barrier: one posted add per CTA (release: the CTA's
@@ -877,19 +898,11 @@ __global__ void __launch_bounds__(kQsThreads, 1)
         for (int w = tid; w < nwords; w += kQsWorkers)
             s_bm[w] = 0u;
         __syncthreads();
-        if (THR)
-            named_barrier_sync(4, kQsThreads); // the control warp has read the counters
-        if (THR && c == 0) { // the other bitmap, for the next call
-            uint32_t *next = sets + ((s_call + 1u) & 1u) * kSetWords;
-            for (int w = tid; w < (int)kSetWords; w += kQsWorkers)
-                next[w] = 0u;
-        }
         QsRow q;
         q.nvec = nvec;
         q.t16 = t16;
         q.s_bm = s_bm;
         q.s_cnt = &s_cnt;
-        q.gset = sets + (s_call & 1u) * kSetWords;
         q.lane = lane;
         QsSetCache sc;
         sc.count = -1;
@@ -1053,11 +1066,15 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
     cfg.blockDim = dim3(kQsThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative; // the grid barrier needs every CTA resident
     attr[0].val.cooperative = 1;
+    // the launch itself may overlap the previous kernel's tail (the kernel
+    // waits for it before reading anything): ~1 us a call on B200
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const uint4 *>(X), (int)rows, (int)cols,
                               threshold_fp16(t), codes, absmax, bitmap_out, sets, calls, arrivals, col_idx, count, status);
 }
