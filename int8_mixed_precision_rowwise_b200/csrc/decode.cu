@@ -104,12 +104,16 @@ struct DSmem {
     static constexpr int WV_OFF = ACC_OFF + TM * (BN + 1) * 4;       // float [OC][TM]: outlier weights
     static constexpr int BAR_OFF = WV_OFF + OC * TM * 4;             // uint64 barriers
     static constexpr int NBARS = 2 * STAGES + 7;                     // full, empty, tfull[2], tempty[2], drain, xloaded, ready
-    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;             // tmem base, abort, last, grid flag, generation
+    static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;             // tmem base, abort, last, grid flag, generation, outlier count
     static constexpr int BYTES = MISC_OFF + 32;
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : 64;
     static_assert(ALLOC <= 232448, "shared memory over the 227 KB per-CTA limit");
     static_assert(W_BYTES % 1024 == 0 && X_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+    // The accumulator rows and outlier weights double as the scratch of the
+    // outlier-mask compaction (K / 8 bytes, at most kMaxVecPerCta per CTA).
+    static_assert(WV_OFF + OC * TM * 4 - ACC_OFF >= kMaxVecPerCta * kDecodeMaxCtas + 16 && ACC_OFF % 16 == 0,
+                  "mask scratch");
 };
 
 __device__ __forceinline__ void report(const DParams &p, volatile int *s_abort, uint32_t bit)
@@ -160,16 +164,35 @@ __device__ __forceinline__ int64_t unit_order(int64_t u0, int64_t u1, int KB, in
 }
 
 // Ascending list of the outlier columns from the per-8-column masks
-// hitmask[0 .. nvec), by the NHELP helper threads of one CTA.
-__device__ void compact_masks(const uint8_t *hitmask, int nvec, int32_t *col_idx, int32_t *count, int et,
-                              int *s_pfx)
+// hitmask[0 .. nvec), by the NHELP helper threads of one CTA: the first `cap`
+// columns into s_cols and their number into *s_count; with g_idx non-null
+// the whole list and its length also into g_idx / *g_count. The masks are
+// read once into s_scratch with 16-byte loads, all in flight together (each
+// dependent global round trip costs microseconds behind the weight stream);
+// the workspace region of the masks is padded to 256 bytes, and the bytes
+// at or past nvec are never counted.
+__device__ void compact_masks(const uint8_t *hitmask, int nvec, uint8_t *s_scratch, int *s_cols, int32_t *s_count,
+                              int cap, int32_t *g_idx, int32_t *g_count, int et, int *s_pfx)
 {
+    const int nq = (nvec + 15) >> 4;
+    for (int q0 = et; q0 < nq; q0 += 4 * NHELP) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (q0 + u * NHELP < nq)
+                v[u] = __ldcg(reinterpret_cast<const uint4 *>(hitmask) + q0 + u * NHELP);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (q0 + u * NHELP < nq)
+                reinterpret_cast<uint4 *>(s_scratch)[q0 + u * NHELP] = v[u];
+    }
+    named_barrier_sync(1, NHELP);
     const int lane = et & 31, w = et >> 5;
     const int per = (nvec + NHELP - 1) / NHELP;
     const int b0 = min(et * per, nvec), b1 = min(b0 + per, nvec);
     int cnt = 0;
     for (int b = b0; b < b1; ++b)
-        cnt += __popc((uint32_t)__ldcg(hitmask + b));
+        cnt += __popc((uint32_t)s_scratch[b]);
     int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -183,18 +206,26 @@ __device__ void compact_masks(const uint8_t *hitmask, int nvec, int32_t *col_idx
     int base = 0;
     for (int i = 0; i < w; ++i)
         base += s_pfx[i];
-    if (et == NHELP - 1)
-        *count = base + incl;
+    if (et == NHELP - 1) {
+        *s_count = base + incl;
+        if (g_idx)
+            *g_count = base + incl;
+    }
     int pos = base + incl - cnt;
     for (int b = b0; b < b1; ++b) {
-        uint32_t bits = __ldcg(hitmask + b);
+        uint32_t bits = s_scratch[b];
         while (bits) {
             const int e = __ffs(bits) - 1;
-            col_idx[pos++] = b * 8 + e;
+            if (pos < cap)
+                s_cols[pos] = b * 8 + e;
+            if (g_idx)
+                g_idx[pos] = b * 8 + e;
+            ++pos;
             bits &= bits - 1u;
         }
     }
-    __threadfence();
+    if (g_idx)
+        __threadfence();
     named_barrier_sync(1, NHELP);
 }
 
@@ -361,23 +392,6 @@ __device__ bool row_scales(const DParams &p, int et, uint32_t xloaded_bar, uint3
     return *s_flag != 0;
 }
 
-// The ascending outlier columns and their count, by CTA 0's helper warps
-// after the codes are out (off the critical path: the epilogues need the
-// list much later); then the list flag sync[3] is set to `gen`.
-template <bool THR>
-__device__ void publish_outlier_list(const DParams &p, int et, int *s_pfx, uint32_t gen)
-{
-    if constexpr (THR) {
-        compact_masks(p.hitmask, p.K >> 3, p.col_idx, p.count, et, s_pfx);
-    } else if (et == 0) {
-        *p.count = 0;
-    }
-    if (et == NHELP - 1 || (!THR && et == 0)) {
-        __threadfence();
-        asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p.sync + 3), "r"(gen) : "memory");
-    }
-}
-
 // Outlier weights W~[j, cols[k]] of this thread's weight row j for k < nk
 // into s_wv[k][r], eight loads in flight at a time.
 __device__ __forceinline__ void load_wv(const DParams &p, int j, int r, const int *cols, int nk, float *s_wv)
@@ -394,36 +408,64 @@ __device__ __forceinline__ void load_wv(const DParams &p, int j, int r, const in
     }
 }
 
+// y[0..8) += W~[j, col k] * X[c0 + u, col k] over the staged outlier columns
+// k < nk, k ascending: s_wv points at this row's first weight, side at token
+// c0 of column 0. One weight load and two broadcast loads of X per column
+// feed eight independent FMA chains (one chain per token would wait on the
+// shared-memory latency at every column); each token's sum keeps the column
+// order.
+template <int BN>
+__device__ __forceinline__ void outlier_fma8(float (&y)[8], const float *s_wv, const float *side, int nk)
+{
+#pragma unroll 2
+    for (int k = 0; k < nk; ++k) {
+        const float w = s_wv[k * TM];
+        const float4 a = *reinterpret_cast<const float4 *>(side + k * BN);
+        const float4 b = *reinterpret_cast<const float4 *>(side + k * BN + 4);
+        y[0] = fmaf(w, a.x, y[0]);
+        y[1] = fmaf(w, a.y, y[1]);
+        y[2] = fmaf(w, a.z, y[2]);
+        y[3] = fmaf(w, a.w, y[3]);
+        y[4] = fmaf(w, b.x, y[4]);
+        y[5] = fmaf(w, b.y, y[5]);
+        y[6] = fmaf(w, b.z, y[6]);
+        y[7] = fmaf(w, b.w, y[7]);
+    }
+}
+
 // Dequantize this thread's accumulator row acc[0..M) (weight row j), add the
 // outlier product and store Y (and the raw products when asked). All NHELP
 // helper threads call it together: with more than OC outlier columns the
-// columns are staged in chunks behind named barriers.
+// columns are staged in chunks behind named barriers. The row's outputs are
+// kept in place of the accumulators (fp32) until the final stores.
 template <int BN>
 __device__ void finalize_row(const DParams &p, int j, int r, int32_t *acc, const float *s_amax, float *s_side,
                              int *s_cols, float *s_wv, int cnt, int et)
 {
+    static_assert(BN % 8 == 0, "tokens are processed in groups of eight");
     const int M = p.M;
     if (p.acc_out && j < p.N)
         for (int c = 0; c < M; ++c)
             p.acc_out[(int64_t)c * p.N + j] = acc[c];
     const float sbj = j < p.N ? p.sb[j] : 0.f;
     const float bj = (p.bias && j < p.N) ? __half2float(p.bias[j]) : 0.f;
-    if (cnt <= OC) {
-        // s_side holds X at the outlier columns for all tokens (staged once per
-        // CTA), s_wv this row's outlier weights (loaded before the accumulator).
-        for (int c = 0; c < M; ++c) {
-            float y = (float)acc[c] * (sbj * s_amax[c]) * kInv127Sq;
-            for (int k = 0; k < cnt; ++k)
-                y = fmaf(s_wv[k * TM + r], s_side[k * BN + c], y);
-            if (j < p.N)
-                p.Y[(int64_t)c * p.N + j] = __float2half_rn(bias_act(y, bj, p.act));
-        }
-        return;
-    }
     float *yr = reinterpret_cast<float *>(acc); // in place: one float per token
-    for (int c = 0; c < M; ++c)
-        yr[c] = (float)acc[c] * (sbj * s_amax[c]) * kInv127Sq;
-    for (int ch = 0; ch < cnt; ch += OC) {
+    // With at most OC outlier columns s_side holds X at all of them for every
+    // token (staged once per CTA) and s_wv this row's outlier weights (loaded
+    // before the accumulator).
+    const int nk0 = cnt <= OC ? cnt : 0;
+    for (int c0 = 0; c0 < M; c0 += 8) {
+        float y[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            y[u] = c0 + u < M ? (float)acc[c0 + u] * (sbj * s_amax[c0 + u]) * kInv127Sq : 0.f;
+        outlier_fma8<BN>(y, s_wv + r, s_side + c0, nk0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (c0 + u < M)
+                yr[c0 + u] = y[u];
+    }
+    for (int ch = 0; cnt > OC && ch < cnt; ch += OC) {
         const int nk = min(OC, cnt - ch);
         named_barrier_sync(1, NHELP);
         if (et < nk)
@@ -436,9 +478,17 @@ __device__ void finalize_row(const DParams &p, int j, int r, int32_t *acc, const
         }
         load_wv(p, j, r, s_cols, nk, s_wv);
         named_barrier_sync(1, NHELP);
-        for (int c = 0; c < M; ++c)
-            for (int k = 0; k < nk; ++k)
-                yr[c] = fmaf(s_wv[k * TM + r], s_side[k * BN + c], yr[c]);
+        for (int c0 = 0; c0 < M; c0 += 8) {
+            float y[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                y[u] = c0 + u < M ? yr[c0 + u] : 0.f;
+            outlier_fma8<BN>(y, s_wv + r, s_side + c0, nk);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (c0 + u < M)
+                    yr[c0 + u] = y[u];
+        }
     }
     if (j < p.N)
         for (int c = 0; c < M; ++c)
@@ -459,7 +509,7 @@ __device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, i
                                  int64_t se,
                                  int seg, uint32_t tmem_base, uint32_t tfull_b, uint32_t tempty_b, uint32_t &tph_b,
                                  const float *s_amax, float *s_side, int *s_cols, int32_t *s_acc, float *s_wv,
-                                 int cnt, uint32_t gen, volatile int *s_abort, volatile int *s_last)
+                                 int cnt, bool wv_loaded, uint32_t gen, volatile int *s_abort, volatile int *s_last)
 {
     const int64_t G = gridDim.x, cta = blockIdx.x;
     const int KB = p.num_kb, M = p.M;
@@ -479,7 +529,7 @@ __device__ bool epilogue_segment(const DParams &p, int et, int warp, int lane, i
         // Everything that does not need this CTA's accumulator first, while
         // its last MMAs run: this row's outlier weights and the partial sums
         // the tile's other CTAs parked (normally long ready).
-        if (cnt <= OC)
+        if (cnt <= OC && !wv_loaded)
             load_wv(p, j, r, s_cols, cnt, s_wv);
         for (int c = 0; c < M; ++c)
             acc[c] = 0;
@@ -591,6 +641,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     volatile int *s_last = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 8);
     volatile int *s_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 12);
     volatile uint32_t *s_gen = reinterpret_cast<volatile uint32_t *>(smem + L::MISC_OFF + 16);
+    int32_t *s_cnt = reinterpret_cast<int32_t *>(smem + L::MISC_OFF + 20);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -781,47 +832,83 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 report(p, s_abort, LLMINT8_DEV_TIMEOUT_QUANT);
             mbar_arrive(ready_bar); // the producer may add the codes to its stages
         }
-        if (ok && blockIdx.x == 0)
-            publish_outlier_list<THR>(p, et, s_pfx, gen);
+        int cnt = 0;
+        bool go = ok;
         if (ok) {
-            // The outlier list of CTA 0 (ready long before the first segment ends).
-            if (et == 0) {
-                const uint64_t t0 = global_timer_ns();
-                uint32_t f;
-                for (;;) {
-                    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(f) : "l"(p.sync + 3) : "memory");
-                    if (f == gen || global_timer_ns() - t0 > kWaitLimitNs)
-                        break;
-                    __nanosleep(200);
-                }
-                *s_flag = f == gen ? 1 : 0;
-                if (f != gen)
-                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+            // This CTA's own copy of the first OC outlier columns and their
+            // number, from the masks that every CTA published before the
+            // first grid barrier (no wait on another CTA). CTA 0 also writes
+            // the whole list and its length to the workspace and then sets
+            // the list flag sync[3] to `gen`; only with more than OC columns
+            // do the epilogues read that list.
+            const bool publish = blockIdx.x == 0;
+            if constexpr (THR) {
+                compact_masks(p.hitmask, p.K >> 3, reinterpret_cast<uint8_t *>(s_acc), s_cols, s_cnt, OC,
+                              publish ? p.col_idx : nullptr, p.count, et, s_pfx);
+            } else if (et == 0) {
+                *s_cnt = 0;
+                if (publish)
+                    *p.count = 0;
+            }
+            if (publish && et == 0) {
+                __threadfence();
+                asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p.sync + 3), "r"(gen) : "memory");
             }
             named_barrier_sync(1, NHELP);
-        }
-        if (ok && *s_flag) {
-            const int cnt = min(__ldcg(p.count), p.K);
-            if (cnt <= OC) {
-                if (et < cnt)
-                    s_cols[et] = __ldcg(p.col_idx + et);
+            cnt = *s_cnt;
+            if (cnt > OC) {
+                // More columns than one staging chunk: the epilogues read the
+                // whole list, CTA 0's.
+                if (et == 0) {
+                    const uint64_t t0 = global_timer_ns();
+                    uint32_t f;
+                    for (;;) {
+                        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(f) : "l"(p.sync + 3) : "memory");
+                        if (f == gen || global_timer_ns() - t0 > kWaitLimitNs)
+                            break;
+                        __nanosleep(200);
+                    }
+                    *s_flag = f == gen ? 1 : 0;
+                    if (f != gen)
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                }
+                named_barrier_sync(1, NHELP);
+                go = *s_flag != 0;
+            } else {
                 // X at the outlier columns, for every tile of this CTA.
                 for (int idx = et; idx < cnt * BN; idx += NHELP) {
                     const int k = idx / BN, c = idx - k * BN;
-                    s_side[idx] = c < p.M ? __half2float(reinterpret_cast<const __half *>(p.X)[(int64_t)c * p.K +
-                                                                                            __ldcg(p.col_idx + k)])
-                                          : 0.f;
+                    s_side[idx] =
+                        c < p.M ? __half2float(reinterpret_cast<const __half *>(p.X)[(int64_t)c * p.K + s_cols[k]])
+                                : 0.f;
                 }
             }
             named_barrier_sync(1, NHELP);
+        }
+        if (go) {
             uint32_t tph[2] = {0u, 0u};
             int seg = 0;
+            bool wv_loaded = false; // s_wv holds the outlier weights of the segment processed next
             for (int64_t seg_end = u1; seg_end > u0; ++seg) { // segments from the last to the first
                 const int64_t su = max(u0, ((seg_end - 1) / KB) * KB);
                 const int b = seg & 1;
+                const bool wv_now = wv_loaded;
+                wv_loaded = false;
+                // Only the first segment processed can be a parked one (a tile
+                // head); every segment after it ends at a tile end and is
+                // finished here. Its outlier weights (a round trip to HBM) are
+                // fetched before the parked segment's epilogue, off the path
+                // that follows the last MMA.
+                const int64_t tile_u0 = (su / KB) * KB;
+                const bool parks = seg_end % KB != 0 && owner_of(tile_u0 + KB - 1, p.units, G) != (int)cta;
+                if (parks && su > u0 && cnt <= OC) {
+                    const int r = (warp & 3) * 32 + lane;
+                    load_wv(p, (int)((su - 1) / KB) * TM + r, r, s_cols, cnt, s_wv);
+                    wv_loaded = true;
+                }
                 if (!epilogue_segment<BN>(p, et, warp, lane, u0, u1, su, seg_end, seg, tmem_base, tfull_bar(b),
-                                          tempty_bar(b), tph[b], s_amax, s_side, s_cols, s_acc, s_wv, cnt, gen,
-                                          s_abort, s_last))
+                                          tempty_bar(b), tph[b], s_amax, s_side, s_cols, s_acc, s_wv, cnt, wv_now,
+                                          gen, s_abort, s_last))
                     break;
                 seg_end = su;
             }

@@ -375,6 +375,23 @@ def test_decode_split_tiles(lib, dev, oracle_mod, M, N, K):
     check_full(lib, dev, oracle_mod, X16, W16, 6.0, give_w16=False)
 
 
+@pytest.mark.parametrize("n_cols,give_w16", [(32, False), (33, True), (33, False), (1, True)])
+def test_decode_outlier_count_at_staging_limit(lib, dev, oracle_mod, n_cols, give_w16):
+    """Every CTA of the decode kernel keeps its own list of the first 32
+    outlier columns; with one more it reads the whole list that CTA 0
+    publishes, in chunks. Columns spread over the K range, some in the last
+    8-column group."""
+    M, N, K = 5, 700, 2048
+    X16 = make_random((M, K), seed=31)
+    cols = np.unique(np.concatenate([np.linspace(3, K - 2, n_cols - 1).astype(np.int64), [K - 1]]))
+    assert cols.size == n_cols
+    rng = np.random.default_rng(n_cols)
+    X16[rng.integers(0, M, cols.size), cols] = (40.0 * rng.choice([-1.0, 1.0], cols.size)).astype(np.float16)
+    W16 = make_random((N, K), seed=32, scale=0.02)
+    g, r = check_full(lib, dev, oracle_mod, X16, W16, 6.0, give_w16=give_w16)
+    assert np.array_equal(np.sort(r["O"]), cols)
+
+
 def test_decode_threshold_off(lib, dev, oracle_mod):
     X16 = make_random((5, 2048), seed=21)
     W16 = make_random((700, 2048), seed=22, scale=0.02)
