@@ -1014,6 +1014,12 @@ cudaError_t launch_quantize(const void *X, int64_t rows, int64_t cols64, float t
     if (nvec <= 256 * 32 && nvec > 256 * 16)
         return launch_fused_v<8, 32>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
                                      stream);
+    // Rows of exactly 7 vectors a thread (14336 columns, BLOOM-176B's hidden
+    // width): no empty eighth vector and no bounds checks (measured on B200:
+    // 2048 x 14336 in 27.0 instead of 28.7 us).
+    if (nvec == 256 * 7)
+        return launch_fused_v<8, 7>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev,
+                                    stream);
     return launch_fused_v<8, 8>(X, rows, cols, t, codes, absmax, bitmap, col_idx, count, sync, status, dev, stream);
 }
 

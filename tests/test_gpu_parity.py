@@ -162,23 +162,28 @@ def test_quantize_edge_rows(lib, dev, oracle_mod):
     assert np.array_equal(codes.cpu().numpy(), c_ref)
 
 
-def test_quantize_late_outlier_column(lib, dev, oracle_mod):
-    """8192 x 4096 (too large for the shared-memory quantizer, so the
-    streaming one with its seed runs): the seed reads each warp's first row
-    only, so a column that crosses the threshold only in row 8100 is found
-    late, while rows 7000.. already took their maximum (5.5) in it. The result
-    must still be the definition's (every row re-quantized against the final
-    set)."""
-    X = np.random.default_rng(8).standard_normal((8192, 4096)).astype(np.float32)
+@pytest.mark.parametrize("M,K,late_row,from_row", [
+    (8192, 4096, 8100, 7000),    # a warp per row
+    (2048, 14336, 2000, 1500),   # the CTA per row, 7 vectors a thread (BLOOM's hidden width)
+    (1024, 57344, 1000, 700),    # the CTA per row, 32 vectors a thread (BLOOM's fc2 input)
+])
+def test_quantize_late_outlier_column(lib, dev, oracle_mod, M, K, late_row, from_row):
+    """Shapes too large for the shared-memory quantizer, so the streaming one
+    with its seed runs: the seed reads each group's first row only, so a
+    column that crosses the threshold only in row `late_row` is found late,
+    while rows from `from_row` on already took their maximum (5.5) in it. The
+    result must still be the definition's (every row re-quantized against the
+    final set)."""
+    X = np.random.default_rng(8).standard_normal((M, K)).astype(np.float32)
     X[:, 100] *= 0.1
-    X[7000:, 100] = 5.5
-    X[8100, 100] = 50.0
+    X[from_row:, 100] = 5.5
+    X[late_row, 100] = 50.0
     X16 = X.astype(np.float16)
     codes, absmax, bm = lib.quantize_rowwise(to_dev(X16, dev), 6.0)
     mask = oracle_mod.outlier_mask(X16, 6.0)
     assert mask[100]
     c_ref, a_ref = oracle_mod.quantize_rowwise(X16, mask)
-    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), 4096), mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
     assert np.array_equal(absmax.cpu().numpy().view(np.uint32), a_ref.view(np.uint32))
     assert np.array_equal(codes.cpu().numpy(), c_ref)
 
