@@ -576,15 +576,13 @@ llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K
     if (device_info(&dev) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     const float t = effective_threshold(threshold);
-    cudaError_t e = cudaSuccess;
     if (t > 0.f) {
-        if ((e = detect_outliers(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws, dev, stream)) != cudaSuccess)
+        if (detect_outliers(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws, dev, stream) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
-    } else if ((e = cudaMemsetAsync(ws.count, 0, sizeof(int32_t), stream)) != cudaSuccess) {
+    } else if (cudaMemsetAsync(ws.count, 0, sizeof(int32_t), stream) != cudaSuccess) {
         return LLMINT8_ERR_CUDA;
     }
-    if ((e = launch_quantize_asym(X_f16, M, K, t > 0.f ? ws.bitmap : nullptr, ws.cx, ws.sx, zx, dev, stream)) !=
-        cudaSuccess)
+    if (launch_quantize_asym(X_f16, M, K, t > 0.f ? ws.bitmap : nullptr, ws.cx, ws.sx, zx, dev, stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     GemmArgs g{};
     g.A = ws.cx;
@@ -606,7 +604,7 @@ llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K
     if (dbg && dbg->gemm_begin &&
         cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_begin), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-    if ((e = gather_then_gemm(g, ws, dev, stream)) != cudaSuccess)
+    if (gather_then_gemm(g, ws, dev, stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     if (dbg && dbg->gemm_end && cudaEventRecord(static_cast<cudaEvent_t>(dbg->gemm_end), stream) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
