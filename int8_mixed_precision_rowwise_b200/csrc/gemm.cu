@@ -376,6 +376,47 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
 
         if constexpr (!SWAP) {
             const int i = arow;
+            // More outlier columns than s_side holds at once: the columns go
+            // in chunks of OC, outermost. Each chunk's W values are staged
+            // for the whole tile (one round of gathers, eight in flight per
+            // thread) and this row's X values go to registers once; between
+            // chunks the partial sums wait in the tile's own TMEM accumulator
+            // (fp32 bits in place of the int32 products), so each output
+            // still adds its outlier products in ascending column order.
+            const int nch = (RAW || fast) ? 1 : (cnt + OC - 1) / OC;
+            for (int ch = 0; ch < nch; ++ch) {
+            const int nk = min(OC, cnt - ch * OC);
+            if (!RAW && !fast) {
+                named_barrier_sync(1, 128); // the previous chunk's readers are done with s_side / s_cols
+                if (et < nk)
+                    s_cols[et] = p.col_idx[ch * OC + et];
+                named_barrier_sync(1, 128);
+                for (int base = 0; base < nk * BN; base += 32 * 128) { // 32 gathers in flight per thread
+                    float vals[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int idx = base + u * 128 + et;
+                        float v = 0.f;
+                        if (idx < nk * BN) {
+                            const int k = idx / BN, r = brow0 + (idx - k * BN);
+                            if (r < p.N)
+                                v = wtilde(p, r, s_cols[k]);
+                        }
+                        vals[u] = v;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int idx = base + u * 128 + et;
+                        if (idx < nk * BN)
+                            s_side[idx] = vals[u];
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < OC; ++k)
+                    own_side[k] = (k < nk && arow < p.M) ? __half2float(p.X16[(int64_t)arow * p.K + s_cols[k]]) : 0.f;
+                named_barrier_sync(1, 128);
+            }
+            const bool last_chunk = ch == nch - 1;
 #pragma unroll 1
             for (int g = 0; g < BN / 32; ++g) {
                 uint32_t acc[32];
@@ -399,7 +440,11 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                     continue;
                 }
                 float y[32];
-                if (p.zx) {
+                if (ch > 0) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        y[c] = __uint_as_float(acc[c]); // the partial sums the previous chunk left
+                } else if (p.zx) {
                     // Zero-point codes: sum_k (q - z_i) CB[j,k] = acc + (128 - z_i) R[j],
                     // dequantized by SB[j] / (127 s_i) (s_i = 0: an all-zero row).
                     const float zc = (float)(128 - own_z);
@@ -466,23 +511,30 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                         }
                     }
                 } else {
-                    // More outlier columns than one staged chunk holds.
-                    for (int ch = 0; ch < cnt; ch += OC) {
-                        const int nk = min(OC, cnt - ch);
-                        named_barrier_sync(1, 128);
-                        for (int idx = et; idx < nk * 32; idx += 128) {
-                            const int k = idx >> 5, c = idx & 31;
-                            const int j = j0 + c;
-                            s_side[idx] = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
-                        }
-                        named_barrier_sync(1, 128);
-                        for (int k = 0; k < nk; ++k) {
-                            const float xv =
-                                i < p.M ? __half2float(p.X16[(int64_t)i * p.K + p.col_idx[ch + k]]) : 0.f;
+                    // chunk ch of the outlier columns (staged above; unrolled
+                    // over the OC slots so that own_side stays in registers)
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                y[c] = fmaf(xv, s_side[k * 32 + c], y[c]);
+                    for (int k = 0; k < OC; ++k) {
+                        if (k < nk) {
+                            const float xv = own_side[k];
+                            const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                            for (int c4 = 0; c4 < 8; ++c4) {
+                                const float4 w = wrow[c4];
+                                y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                            }
                         }
+                    }
+                    if (!last_chunk) {
+                        uint32_t part[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            part[c] = __float_as_uint(y[c]);
+                        tmem_st_32x32b_x32(tbase + g * 32, part);
+                        continue;
                     }
                 }
                 if (p.bias || p.act) {
@@ -563,6 +615,9 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                                 Yr[j0 + c] = __float2half_rn(y[c]);
                     }
                 }
+            }
+            if (!last_chunk)
+                tmem_wait_st(); // the partial sums are in TMEM before the next chunk reads them
             }
         } else {
             // Decode form: this thread owns output feature j = arow; the

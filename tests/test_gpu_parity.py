@@ -338,7 +338,9 @@ def test_tiny_workload(lib, dev, oracle_mod):
     # the epilogue's pipelined staging: at its column limit, one past it, both W sources,
     # the single-CTA form, and more tiles than CTA pairs (each pair prefetches its next tile)
     (300, 1000, 1024, 8, True), (300, 1000, 1024, 8, False), (300, 1000, 1024, 9, False),
-    (100, 700, 1024, 8, False), (1024, 8192, 256, 6, True), (1024, 8192, 256, 6, False)])
+    (100, 700, 1024, 8, False), (1024, 8192, 256, 6, True), (1024, 8192, 256, 6, False),
+    # more outlier columns than one staged chunk: chunks outermost, partial sums kept in TMEM
+    (512, 700, 1024, 33, True), (512, 700, 1024, 70, False), (300, 1000, 2048, 64, True)])
 def test_matmul_mixed_matches_oracle(lib, dev, oracle_mod, M, N, K, nout, give_w16):
     lin = Linear("t", M, N, K, nout, 60.0)
     X16, cols = make_activations(lin, seed=M + N)
@@ -446,11 +448,13 @@ def test_decode_repeat_and_graph(lib, dev):
 
 @pytest.mark.parametrize("M,N,K,act", [(300, 520, 1040, "gelu_tanh"), (300, 520, 1040, None),
                                        (100, 384, 512, "gelu_tanh"), (5, 640, 1024, "gelu_tanh"),
-                                       (32, 300, 2048, None), (7, 136, 96, "gelu_tanh")])
+                                       (32, 300, 2048, None), (7, 136, 96, "gelu_tanh"),
+                                       (300, 520, 96, "gelu_tanh")])
 def test_matmul_mixed_bias_activation(lib, dev, oracle_mod, M, N, K, act):
     """llmint8_matmul_mixed_ex: Y = fp16(act(linear + bias)) on every path
-    (CTA-pair prefill, single-CTA prefill, fused decode; the last shape sends
-    every column to the fp16 side). The tolerance is the linear's, carried
+    (CTA-pair prefill, single-CTA prefill, fused decode; the K = 96 shapes send
+    every column to the fp16 side, 96 columns in three chunks on the CTA-pair
+    path). The tolerance is the linear's, carried
     through the activation: GELU's slope is at most 1.13, and the fp16
     rounding now happens after it."""
     lin = Linear("ba", M, N, K, 5, 60.0)
