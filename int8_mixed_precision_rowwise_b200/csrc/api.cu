@@ -508,6 +508,9 @@ llmint8_status llmint8_quantize_rowwise_asym(const void *X_f16, int64_t rows, in
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
+    if (quantize_smem_fits(rows, cols, dev)) // X fits in shared memory: one kernel, one read of X
+        return cuda_status(launch_quantize_smem(X_f16, rows, cols, t, codes, scale, outlier_bitmap, ws.sets, ws.calls,
+                                                ws.arrivals, ws.col_idx, ws.count, ws.status, dev, stream, zero));
     cudaError_t e = cudaSuccess;
     if (t > 0.f) {
         if ((e = detect_outliers(X_f16, rows, cols, t, codes, scale, outlier_bitmap, ws, dev, stream)) != cudaSuccess)
@@ -576,14 +579,22 @@ llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t M, int64_t K
     if (device_info(&dev) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     const float t = effective_threshold(threshold);
-    if (t > 0.f) {
-        if (detect_outliers(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws, dev, stream) != cudaSuccess)
+    if (quantize_smem_fits(M, K, dev)) {
+        // X fits in shared memory: detection and the zero-point codes in one kernel, one read of X
+        if (launch_quantize_smem(X_f16, M, K, t, ws.cx, ws.sx, nullptr, ws.sets, ws.calls, ws.arrivals, ws.col_idx,
+                                 ws.count, ws.status, dev, stream, zx) != cudaSuccess)
             return LLMINT8_ERR_CUDA;
-    } else if (cudaMemsetAsync(ws.count, 0, sizeof(int32_t), stream) != cudaSuccess) {
-        return LLMINT8_ERR_CUDA;
+    } else {
+        if (t > 0.f) {
+            if (detect_outliers(X_f16, M, K, t, ws.cx, ws.sx, ws.bitmap, ws, dev, stream) != cudaSuccess)
+                return LLMINT8_ERR_CUDA;
+        } else if (cudaMemsetAsync(ws.count, 0, sizeof(int32_t), stream) != cudaSuccess) {
+            return LLMINT8_ERR_CUDA;
+        }
+        if (launch_quantize_asym(X_f16, M, K, t > 0.f ? ws.bitmap : nullptr, ws.cx, ws.sx, zx, dev, stream) !=
+            cudaSuccess)
+            return LLMINT8_ERR_CUDA;
     }
-    if (launch_quantize_asym(X_f16, M, K, t > 0.f ? ws.bitmap : nullptr, ws.cx, ws.sx, zx, dev, stream) != cudaSuccess)
-        return LLMINT8_ERR_CUDA;
     GemmArgs g{};
     g.A = ws.cx;
     g.B = CB;

@@ -160,12 +160,15 @@ __half threshold_fp16(float t);
 // `sets`/`calls`/`arrivals` are the workspace's two bitmaps, call counter and
 // barrier arrival counter,
 // bitmap_out (may be null) receives the outlier bitmap, col_idx/count the
-// ascending outlier columns.
+// ascending outlier columns. With `zero` the codes are the zero-point ones
+// (as launch_quantize_asym writes them against the complete set): absmax
+// then receives the scale s and zero the zero point of each row.
 bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev);
 cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
                                  uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls,
                                  unsigned long long *arrivals, int32_t *col_idx, int32_t *count,
-                                 uint32_t *status, const DeviceInfo &dev, cudaStream_t stream);
+                                 uint32_t *status, const DeviceInfo &dev, cudaStream_t stream,
+                                 int32_t *zero = nullptr);
 
 // Zero-point codes of X's rows against a complete outlier bitmap (null: no
 // outliers): codes int8 (q - 128), scale s and zero point z per row.

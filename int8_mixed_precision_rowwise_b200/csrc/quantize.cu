@@ -596,7 +596,8 @@ struct QsRow {
     uint32_t *s_bm;  // the CTA's set (detection adds to it)
     int *s_cnt;      // its size
     int8_t *cr;      // the row's codes
-    float *am;       // the row's absmax
+    float *am;       // the row's absmax (zero-point codes: its scale s)
+    int32_t *zp;     // zero-point codes: the row's zero point
     int lane;
 };
 
@@ -692,7 +693,14 @@ __device__ __forceinline__ void qs_arrive_detected(bool pub)
 // have, and only then is the row's new part of the set published and the
 // maximum taken again against the set read afresh. Returns the count the
 // row's set was read after (0 when !THR or fixed).
-template <bool THR, bool FULL>
+// ASYM: zero-point codes instead (page "Hugging Face 将 LLM.int8() 8-bit 量化
+// 集成进 transformers 与 accelerate", section "模型量化简介"): over the row's
+// values with the known columns zeroed, [lo, hi] = [min(0, min x),
+// max(0, max x)] on packed fp16, s = 255 / (hi - lo) in fp32 (0 for an
+// all-zero row), z = rint(-lo * s), q = clamp(rint(x * s) + z, 0, 255)
+// stored as q - 128 (a zeroed column gets q = z). rint is the 1.5 * 2^23
+// addition in round-to-nearest-even, exact here: |x * s| <= 255 (+ rounding).
+template <bool THR, bool FULL, bool ASYM>
 __device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub, bool arrive)
 {
     uint4 x[kQsRegVec];
@@ -744,25 +752,73 @@ __device__ int qs_row_reg(const QsRow &q, QsSetCache &sc, bool fixed, bool &pub,
     }
     if (THR && arrive)
         qs_arrive_detected(pub);
-    const float amax = warp_max(fmaxf(__low2float(rm), __high2float(rm)));
-    const float s = qs_scale(amax);
+    if constexpr (ASYM) {
+        __half2 lo2 = __float2half2_rn(0.f), hi2 = __float2half2_rn(0.f);
 #pragma unroll
-    for (int k = 0; k < kQsRegVec; ++k) {
-        const int v = q.lane + 32 * k;
-        if (FULL || v < q.nvec)
-            *reinterpret_cast<uint2 *>(q.cr + (int64_t)v * 8) = codes8(x[k], s);
+        for (int k = 0; k < kQsRegVec; ++k) {
+            const __half2 *h = reinterpret_cast<const __half2 *>(&x[k]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                lo2 = __hmin2(lo2, h[i]);
+                hi2 = __hmax2(hi2, h[i]);
+            }
+        }
+        float lo = fminf(__low2float(lo2), __high2float(lo2));
+        float hi = fmaxf(__low2float(hi2), __high2float(hi2));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        const float range = __fsub_rn(hi, lo);
+        const float s = range > 0.f ? __fdiv_rn(255.0f, range) : 0.f;
+        const int z = (int)(__float_as_uint(__fadd_rn(__fmul_rn(-lo, s), 12582912.0f)) - 0x4B400000u);
+        // rint(x s) + z = (bits of x s + 1.5 * 2^23) - 0x4B400000 + z
+        const int zoff = z - (int)0x4B400000u;
+#pragma unroll
+        for (int k = 0; k < kQsRegVec; ++k) {
+            const int v = q.lane + 32 * k;
+            if (FULL || v < q.nvec) {
+                const __half2 *h = reinterpret_cast<const __half2 *>(&x[k]);
+                uint32_t b[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __half22float2(h[i]);
+                    const int q0 = (int)__float_as_uint(__fadd_rn(__fmul_rn(f.x, s), 12582912.0f)) + zoff;
+                    const int q1 = (int)__float_as_uint(__fadd_rn(__fmul_rn(f.y, s), 12582912.0f)) + zoff;
+                    b[2 * i] = (uint32_t)(min(max(q0, 0), 255) - 128) & 0xFFu;
+                    b[2 * i + 1] = (uint32_t)(min(max(q1, 0), 255) - 128) & 0xFFu;
+                }
+                *reinterpret_cast<uint2 *>(q.cr + (int64_t)v * 8) =
+                    make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                               b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+            }
+        }
+        if (q.lane == 0) {
+            *q.am = s;
+            *q.zp = z;
+        }
+    } else {
+        const float amax = warp_max(fmaxf(__low2float(rm), __high2float(rm)));
+        const float s = qs_scale(amax);
+#pragma unroll
+        for (int k = 0; k < kQsRegVec; ++k) {
+            const int v = q.lane + 32 * k;
+            if (FULL || v < q.nvec)
+                *reinterpret_cast<uint2 *>(q.cr + (int64_t)v * 8) = codes8(x[k], s);
+        }
+        if (q.lane == 0)
+            *q.am = amax;
     }
-    if (q.lane == 0)
-        *q.am = amax;
     return (THR && !fixed) ? sc.count : 0;
 }
 
-template <bool THR, bool FULL>
+template <bool THR, bool FULL, bool ASYM>
 __global__ void __launch_bounds__(kQsThreads, 1)
     k_quant_smem(const uint4 *__restrict__ X, int rows, int cols, __half t16, int8_t *__restrict__ codes,
-                 float *__restrict__ absmax, uint32_t *__restrict__ bitmap_out, uint32_t *sets, uint32_t *calls,
-                 unsigned long long *arrivals, int32_t *__restrict__ col_idx, int32_t *__restrict__ count,
-                 uint32_t *__restrict__ status)
+                 float *__restrict__ absmax, int32_t *__restrict__ zero, uint32_t *__restrict__ bitmap_out,
+                 uint32_t *sets, uint32_t *calls, unsigned long long *arrivals, int32_t *__restrict__ col_idx,
+                 int32_t *__restrict__ count, uint32_t *__restrict__ status)
 {
     extern __shared__ __align__(1024) uint8_t q_smem[];
     __shared__ uint64_t s_bars[kQsMaxChunks];
@@ -941,7 +997,8 @@ __global__ void __launch_bounds__(kQsThreads, 1)
             q.xr = sx + (int64_t)r * nvec;
             q.cr = codes + (int64_t)(r0 + r) * cols;
             q.am = absmax + r0 + r;
-            cmin = min(cmin, qs_row_reg<THR, FULL>(q, sc, false, pub, last));
+            q.zp = zero + r0 + r;
+            cmin = min(cmin, qs_row_reg<THR, FULL, ASYM>(q, sc, false, pub, last));
         }
         if (THR) {
             named_barrier_sync(3, kQsThreads);
@@ -953,7 +1010,8 @@ __global__ void __launch_bounds__(kQsThreads, 1)
                         q.xr = sx + (int64_t)r * nvec;
                         q.cr = codes + (int64_t)(r0 + r) * cols;
                         q.am = absmax + r0 + r;
-                        qs_row_reg<THR, FULL>(q, sc, true, pub, false);
+                        q.zp = zero + r0 + r;
+                        qs_row_reg<THR, FULL, ASYM>(q, sc, true, pub, false);
                     }
                 }
             }
@@ -1047,18 +1105,21 @@ bool quantize_smem_fits(int64_t rows, int64_t cols, const DeviceInfo &dev)
 cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, float t, int8_t *codes, float *absmax,
                                  uint32_t *bitmap_out, uint32_t *sets, uint32_t *calls,
                                  unsigned long long *arrivals, int32_t *col_idx, int32_t *count,
-                                 uint32_t *status, const DeviceInfo &dev, cudaStream_t stream)
+                                 uint32_t *status, const DeviceInfo &dev, cudaStream_t stream, int32_t *zero)
 {
     const bool thr = t > 0.f;
     const bool full = cols / 8 == 32 * kQsRegVec;
-    auto kern = thr ? (full ? k_quant_smem<true, true> : k_quant_smem<true, false>)
-                    : (full ? k_quant_smem<false, true> : k_quant_smem<false, false>);
+    const bool asym = zero != nullptr;
+    auto kern = asym ? (thr ? (full ? k_quant_smem<true, true, true> : k_quant_smem<true, false, true>)
+                            : (full ? k_quant_smem<false, true, true> : k_quant_smem<false, false, true>))
+                     : (thr ? (full ? k_quant_smem<true, true, false> : k_quant_smem<true, false, false>)
+                            : (full ? k_quant_smem<false, true, false> : k_quant_smem<false, false, false>));
     const size_t smem = quant_smem_bytes(rows, cols, dev.num_sms);
     static std::mutex mu;
     static std::map<std::pair<int, int>, size_t> configured; // (device, variant) -> bytes set
     {
         std::lock_guard<std::mutex> lock(mu);
-        size_t &have = configured[std::make_pair(dev.device, (thr ? 1 : 0) + (full ? 2 : 0))];
+        size_t &have = configured[std::make_pair(dev.device, (thr ? 1 : 0) + (full ? 2 : 0) + (asym ? 4 : 0))];
         if (have < smem) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  dev.max_smem_optin - 1024);
@@ -1082,7 +1143,8 @@ cudaError_t launch_quantize_smem(const void *X, int64_t rows, int64_t cols, floa
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const uint4 *>(X), (int)rows, (int)cols,
-                              threshold_fp16(t), codes, absmax, bitmap_out, sets, calls, arrivals, col_idx, count, status);
+                              threshold_fp16(t), codes, absmax, zero, bitmap_out, sets, calls, arrivals, col_idx, count,
+                              status);
 }
 
 namespace {

@@ -61,6 +61,32 @@ def test_quantize_asym_matches_oracle(lib, dev, oracle_mod, M, K, nout, t):
     assert np.array_equal(codes.cpu().numpy(), c_ref)
 
 
+@pytest.mark.parametrize("M,K,rows_hit", [(4096, 4096, [4095]), (1000, 2064, [0, 999]), (150, 4096, [149])])
+def test_quantize_asym_resident_stale_rows(lib, dev, oracle_mod, M, K, rows_hit):
+    """Shapes that fit the shared-memory quantizer (detection and zero-point
+    codes in one kernel): two outlier columns that only a few rows cross,
+    while other rows take their maximum (column 37) or their minimum (column
+    38) in them. Rows coded before the columns were known are coded again
+    against the complete set: codes, scales and zero points are still the
+    definition's."""
+    X = np.random.default_rng(13).standard_normal((M, K)).astype(np.float32)
+    X[:, 37] *= 0.1
+    X[:, 37] += 5.5 * (np.arange(M) % 3 == 0)
+    X[:, 38] *= 0.1
+    X[:, 38] -= 5.5 * (np.arange(M) % 5 == 0)
+    for r in rows_hit:
+        X[r, 37], X[r, 38] = 50.0, -50.0
+    X16 = X.astype(np.float16)
+    codes, scale, zero, bm = lib.quantize_rowwise_asym(to_dev(X16, dev), 6.0)
+    mask = oracle_mod.outlier_mask(X16, 6.0)
+    assert mask[37] and mask[38]
+    c_ref, s_ref, z_ref = oracle_mod.quantize_rowwise_asym(X16, mask)
+    assert np.array_equal(bitmap_to_mask(bm.cpu().numpy(), K), mask)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(zero.cpu().numpy(), z_ref)
+    assert np.array_equal(codes.cpu().numpy(), c_ref)
+
+
 def test_code_row_sums_exact(lib, dev, oracle_mod):
     rng = np.random.default_rng(2)
     CB = rng.integers(-127, 128, size=(1000, 4096), dtype=np.int8)
