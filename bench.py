@@ -243,29 +243,65 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device status word {status:#x}: a kernel gave up on a bounded wait")
 
     # e2e: the same step through the public API with host buffers: X from pinned
-    # host memory to the device, the layer, Y back to pinned host memory.
+    # host memory to the device, the layer, Y back to pinned host memory. The
+    # copies run on streams of their own (PCIe is full duplex: inputs in and
+    # outputs out at once) and overlap the layers: linear i's X goes in while
+    # earlier linears compute, its Y comes out while later ones do. Every
+    # step still moves all of its inputs in and all of its outputs out.
     xh = [x.cpu().pin_memory() for x in xs]
     yh = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in ys]
+    xd = [torch.empty_like(x) for x in xs]
+    yd = [torch.empty_like(y) for y in ys]
     e2e_steps = max(3, min(args.steps, 20))
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nl = len(layers)
+    ev_in = [torch.cuda.Event() for _ in range(nl)]
+    ev_cmp = [torch.cuda.Event() for _ in range(nl)]
+    ev_out = [torch.cuda.Event() for _ in range(nl)]
+    started = [False]
 
     def e2e_step():
+        for i in range(nl):
+            with torch.cuda.stream(s_in):
+                if started[0]:
+                    s_in.wait_event(ev_cmp[i])   # the previous step's layer i has read xd[i]
+                xd[i].copy_(xh[i], non_blocking=True)
+                ev_in[i].record(s_in)
         for i, layer in enumerate(layers):
-            xd = xh[i].to(dev, non_blocking=True)
-            yd = layer(xd)
-            yh[i].copy_(yd, non_blocking=True)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                if started[0]:
+                    s_cmp.wait_event(ev_out[i])  # the previous step's Y of layer i is out
+                layer(xd[i], yd[i])
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                yh[i].copy_(yd[i], non_blocking=True)
+                ev_out[i].record(s_out)
+        started[0] = True
 
+    cur = torch.cuda.current_stream(dev)
+    for s_ in (s_in, s_cmp, s_out):
+        s_.wait_stream(cur)
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
+    a.record(cur)
+    for s_ in (s_in, s_cmp, s_out):
+        s_.wait_stream(cur)
     for _ in range(e2e_steps):
         e2e_step()
-    b.record()
+    for s_ in (s_in, s_cmp, s_out):
+        cur.wait_stream(s_)
+    b.record(cur)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
+    # the host copies hold what the device computed
+    if not all(torch.equal(yh[i], yd[i].cpu()) for i in range(nl)):
+        raise RuntimeError("end-to-end outputs on the host differ from the device's")
 
     int8_measured = measure_int8_peak(dev, local_rank) if rank == 0 else None
     secondary = measure_secondary(L, dev, local_rank) if rank == 0 else None
