@@ -303,7 +303,11 @@ constexpr int kMaxLate = 64; // late outlier columns handled by the cheap path
 // Without a threshold only the quantize step runs. FULL: the row length is a
 // multiple of the chunk (no bounds checks). A row of at most 32 * WPR * V
 // 16-byte vectors stays in registers between its maximum and its codes; a
-// longer one is read twice.
+// longer one is read twice. The next row of a CTA comes in while this one is
+// reduced and coded: into a second register set when a thread holds at most
+// 16 vectors, else (rows of more than 4096 vectors, one CTA per SM) into a
+// shared-memory buffer by bulk copies that one thread issues, from which the
+// threads read it into registers when its turn comes.
 template <int WPR, int V, bool THR, bool FULL>
 __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X, int64_t rows, int cols, float t,
                                                      __half t16, int8_t *__restrict__ codes,
@@ -316,6 +320,7 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     constexpr int GS = 32 * WPR;    // threads per group
     extern __shared__ uint32_t s_dyn[];
     __shared__ float s_red[2][8];
+    __shared__ __align__(8) uint64_t s_rowbar; // the buffered row has landed
     __shared__ int s_flag, s_nlate;
     __shared__ int s_late[kMaxLate];
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -328,8 +333,30 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     uint32_t *s_seed = s_dyn + nwords; // [nwords]
     uint32_t kb4[(V + 3) / 4];
     uint4 v[V];
+    // The next row's buffer (rows of more than 16 vectors a thread): after the
+    // sets, 128-byte aligned.
+    constexpr bool BULK = WPR > 1 && V > 16;
+    const bool bulk = BULK && resident;
+    const uint32_t row_bytes = (uint32_t)cols * 2u;
+    const int buf_off = THR ? ((2 * nwords * 4 + 127) & ~127) : 0;
+    const uint4 *rowbuf = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(s_dyn) + buf_off);
+    const uint32_t rowbar = smem_u32(&s_rowbar);
+    bool row_inflight = false; // (thread 0) a copy into the buffer has not been waited for
+    auto issue_row = [&](int64_t r) { // thread 0: row r into the buffer
+        mbar_arrive_expect_tx(rowbar, row_bytes);
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(X + r * (int64_t)nvec);
+        for (uint32_t off = 0; off < row_bytes; off += 32768u)
+            bulk_load(smem_u32(rowbuf) + off, src + off, min(32768u, row_bytes - off), rowbar);
+        row_inflight = true;
+    };
+    if (bulk && tid == 0) {
+        mbar_init(rowbar, 1);
+        fence_barrier_init();
+    }
     griddep_wait();    // (a programmatic dependent) the previous kernel is complete
     griddep_release(); // the GEMM may start its weight stream now; it waits for this kernel's output
+    if (!THR)
+        __syncthreads(); // the buffer's barrier is initialised
 
     if constexpr (!THR) {
         if (blockIdx.x == 0 && tid == 0 && count)
@@ -349,6 +376,8 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
         // seed_stride-th group reads its first row only to seed.
         if (gid < rows && (resident || gid % seed_stride == 0))
             row_seed<GS, V, FULL>(X + gid * (int64_t)nvec, nvec, gl, t16, s_known, bitmap, v);
+        if (bulk && tid == 0 && gid + G < rows)
+            issue_row(gid + G); // the group's second row comes in during the barrier
         __syncthreads();
         if (tid == 0) {
             s_flag = grid_barrier(sync, gridDim.x) ? 1 : 0;
@@ -356,8 +385,11 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
                 atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT);
         }
         __syncthreads();
-        if (!s_flag)
+        if (!s_flag) {
+            if (row_inflight)
+                mbar_wait(rowbar, 0u); // the copy lands before the CTA exits
             return;
+        }
         for (int w = tid; w < nwords; w += 256)
             s_known[w] = s_seed[w] = __ldcg(bitmap + w);
         __syncthreads();
@@ -381,8 +413,32 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
     };
     uint4 vn[PREFETCH ? V : 1];
     int it = 0;
+    bool row_ok = true;
     for (int64_t r = gid; r < rows; r += G, ++it) {
         bool pre = THR && resident && it == 0; // the seed step left the first row in v
+        if (BULK && bulk) {
+            if (it == 0 && !pre) {
+                load_row(r, v);
+                pre = true;
+            } else if (it > 0) {
+                // this row came into the buffer during the previous one
+                row_ok = row_ok && mbar_wait(rowbar, (uint32_t)(it - 1) & 1u);
+#pragma unroll
+                for (int u = 0; u < V; ++u) {
+                    const int vi = u * GS + gl;
+                    v[u] = (FULL || vi < nvec) ? rowbuf[vi] : make_uint4(0u, 0u, 0u, 0u);
+                }
+                pre = true;
+            }
+            __syncthreads(); // every thread has its values: the buffer takes the next row
+            if (tid == 0) {
+                row_inflight = false;
+                if (r + G < rows && !(THR && it == 0)) { // (with a threshold row 1 went out before the barrier)
+                    fence_proxy_async_smem();
+                    issue_row(r + G);
+                }
+            }
+        }
         if constexpr (PREFETCH) {
             if (resident) {
                 if (it == 0 && !pre)
@@ -402,6 +458,8 @@ __global__ void __launch_bounds__(256) k_quant_fused(const uint4 *__restrict__ X
             }
         }
     }
+    if (BULK && bulk && !row_ok && gl == 0)
+        atomicOr(status, LLMINT8_DEV_TIMEOUT_QUANT); // a buffered row did not land in time
     if constexpr (!THR)
         return;
     if (all_seeded)
@@ -471,8 +529,26 @@ cudaError_t launch_fused(const void *X, int64_t rows, int cols, float t, int8_t 
                          const DeviceInfo &dev, cudaStream_t stream)
 {
     constexpr int GROUPS = 8 / WPR;
-    const size_t smem = THR ? (size_t)((cols + 31) / 32) * 4 * 2 : 0;
+    const size_t sets = THR ? (size_t)((cols + 31) / 32) * 4 * 2 : 0;
+    // rows of more than 16 vectors a thread held in registers: the next row's buffer after the sets
+    const bool bulk = WPR > 1 && V > 16 && (cols >> 3) <= 32 * WPR * V;
+    const size_t smem = bulk ? ((sets + 127) & ~(size_t)127) + (size_t)cols * 2 : sets;
     auto kern = k_quant_fused<WPR, V, THR, FULL>;
+    if (smem > 48 * 1024) {
+        static std::mutex amu;
+        static int attr_dev = -1;
+        std::lock_guard<std::mutex> lock(amu);
+        if (attr_dev != dev.device) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         dev.max_smem_optin - (int)fa.sharedSizeBytes);
+            if (e != cudaSuccess)
+                return e;
+            attr_dev = dev.device;
+        }
+    }
     // Resident CTAs per SM, cached per (kernel, device, shared memory in 1 KB steps).
     static std::mutex mu;
     static std::map<std::pair<int, size_t>, int> occ;
