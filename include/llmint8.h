@@ -79,7 +79,9 @@ LLMINT8_API const char *llmint8_status_string(int status);
 /* Bytes of workspace needed by llmint8_quantize_rowwise for `rows` x `cols`. */
 LLMINT8_API size_t llmint8_quantize_workspace_size(int64_t rows, int64_t cols);
 
-/* Bytes of workspace needed by llmint8_matmul_mixed for X [M x K], W [N x K]. */
+/* Bytes of workspace needed by llmint8_matmul_mixed for X [M x K], W [N x K].
+ * For M >= 256 it includes about 21 MB of stream-K slots: the CTA-pair GEMM
+ * may split its last tiles over the SMs by K and sum the int32 parts there. */
 LLMINT8_API size_t llmint8_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* Zero a workspace (a cudaMemsetAsync). A workspace must be zeroed once before
@@ -288,8 +290,8 @@ LLMINT8_API llmint8_status llmint8_matmul_mixed_asym(const void *X_f16, int64_t 
  * Plain int8 GEMM with int32 output: acc[i,j] = sum_k A[i,k] * B[j,k]
  * (the int8 product of vector-wise quantization, [Q]).
  *   A (device) int8 [M x K], B (device) int8 [N x K], acc (device) int32 [M x N].
- *   workspace: >= llmint8_workspace_size(M, N, K) bytes, zeroed once (only
- *   its status word is used).
+ *   workspace: >= llmint8_workspace_size(M, N, K) bytes, zeroed once (its
+ *   status word, and for M >= 256 its stream-K slots and flags).
  */
 LLMINT8_API llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B, int64_t N,
                                     int64_t K, int32_t *acc, void *workspace, size_t ws_bytes,

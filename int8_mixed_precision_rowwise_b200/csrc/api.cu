@@ -123,6 +123,8 @@ cudaError_t gather_then_gemm(GemmArgs g, const Workspace &ws, const DeviceInfo &
         g.np = ws.np;
         g.mp = ws.mp;
     }
+    g.sk_part = ws.sk_part;
+    g.sk_flag = ws.sk_flag;
     return launch_gemm(g, dev, stream);
 }
 
@@ -422,7 +424,8 @@ llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B,
     if (!aligned16(A) || !aligned16(B) || !aligned16(acc) || !aligned16(workspace))
         return LLMINT8_ERR_ALIGNMENT;
     Workspace ws;
-    const size_t need = carve(static_cast<char *>(workspace), M, K, true, false, &ws);
+    const bool dec = decode_shape(M, N);
+    const size_t need = carve(static_cast<char *>(workspace), M, K, true, dec, &ws, dec ? 0 : N);
     if (ws_bytes < need)
         return LLMINT8_ERR_WORKSPACE;
     if (M == 0 || N == 0)
@@ -431,6 +434,8 @@ llmint8_status llmint8_gemm_s8s8s32(const int8_t *A, int64_t M, const int8_t *B,
     if (device_info(&dev) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     GemmArgs g{};
+    g.sk_part = ws.sk_part;
+    g.sk_flag = ws.sk_flag;
     g.A = A;
     g.B = B;
     g.M = M;

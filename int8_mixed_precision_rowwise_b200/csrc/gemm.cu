@@ -70,7 +70,66 @@ struct KParams {
     const float *wt_t, *sb_p, *xo_t;
     int np, mp;
     int y_tma;                 // Y (fp16) has a TMA store map (tmY): 32-row x 64-column boxes
+    // Stream-K (CTA-pair kernel only; 0: none): the last sk_tiles tiles are
+    // split over the pairs by K stages. A split tile's first part parks its
+    // int32 partial accumulator in the parking pair's slot of sk_part
+    // ([pairs][2 CTAs][BN/32][8][128 rows][4]) and raises that pair's flag in
+    // sk_flag ([pairs][2]); the pair holding the tile's last stage adds it.
+    int sk_tiles;
+    int32_t *sk_part;
+    uint32_t *sk_flag;
 };
+
+// One unit of a CTA's (or pair's) work: K stages [st0, st1) of a tile.
+struct Seg {
+    int tile, st0, st1;
+};
+
+// The work of one CTA (or pair) `first` of `step`, in processing order:
+// whole tiles first, first + step, ... below the stream-K tiles; then its
+// share of the stream-K tiles' stages, a contiguous range of the stages of
+// those tiles in order, cut at tile boundaries and taken from its end to its
+// start. Each range spans at least one tile's stages and fewer than three
+// tiles (the stream-K tiles number between one and two per pair), so a
+// range is at most three segments: the part of a tile it ends in (parked
+// for the pair that holds the tile's last stage, and processed first, so
+// that no pair waits for one that is itself waiting), whole tiles, and the
+// part of a tile it starts in (whose other part the previous pair parked;
+// processed last).
+struct Sched {
+    int first, step, ndp, nseg, S;
+    Seg seg[3];
+    __device__ __forceinline__ int count() const { return ndp + nseg; }
+    __device__ __forceinline__ Seg item(int w) const
+    {
+        if (w < ndp)
+            return Seg{first + w * step, 0, S};
+        return seg[w - ndp];
+    }
+};
+
+__device__ __forceinline__ Sched make_sched(int num_tiles, int sk_tiles, int first, int step, int S)
+{
+    Sched sc;
+    sc.first = first;
+    sc.step = step;
+    sc.S = S;
+    sc.nseg = 0;
+    const int dp_end = num_tiles - sk_tiles;
+    sc.ndp = first < dp_end ? (dp_end - first + step - 1) / step : 0;
+    if (sk_tiles > 0) {
+        const int64_t U = (int64_t)sk_tiles * S;
+        const int64_t g0 = U * first / step;
+        int64_t e = U * (first + 1) / step;
+        while (e > g0 && sc.nseg < 3) {
+            const int64_t t = (e - 1) / S;
+            const int64_t lo = max(g0, t * S);
+            sc.seg[sc.nseg++] = Seg{dp_end + (int)t, (int)(lo - t * S), (int)(e - t * S)};
+            e = lo;
+        }
+    }
+    return sc;
+}
 
 template <int BN, int STAGES>
 struct Smem {
@@ -111,7 +170,10 @@ __device__ __forceinline__ void report(const KParams &p, volatile int *s_abort, 
 // outlier operands and scales while the tile's MMAs run, wait for the
 // accumulator, then dequantize, add the outlier product and store (or store
 // the raw int32 accumulators), and hand the TMEM buffer back to the MMA
-// issuer. Tiles are first_tile, first_tile + tile_step, ...; this CTA's
+// issuer. Its work items are those of `sc` (whole tiles, and for CTA pairs
+// the parts of stream-K tiles: a parked part only stores its int32 partials
+// for the next pair; the part holding a tile's last stage adds the parked
+// partials, copied into `sk_buf`, before the usual epilogue); this CTA's
 // accumulator rows are a_row_off .. a_row_off + 127 of each a_tile_rows-row
 // A tile.
 // One tile's staging loads held in registers as they arrive (raw: no
@@ -174,8 +236,8 @@ template <int BN, bool SWAP, bool RAW, bool PAIR>
 __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap *tmY, int warp, int lane,
                                              float *s_side, float *s_scale, int *s_cols,
                                              uint32_t tfull0, uint32_t tempty0, uint32_t sbar, volatile int *s_abort,
-                                             uint32_t tmem_base, int first_tile, int tile_step, int num_tiles,
-                                             int a_tile_rows, int a_row_off)
+                                             uint32_t tmem_base, const Sched &sc, int a_tile_rows, int a_row_off,
+                                             uint8_t *sk_buf)
 {
     auto tfull_bar = [&](int b) { return tfull0 + 8u * b; };
     auto tempty_bar = [&](int b) { return tempty0 + 8u * b; };
@@ -228,12 +290,21 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
         bulk_load(smem_u32(s_scale), p.sb_p + brow0, BN * 4u, sbar);
         staged_pending = true;
     };
-    if (gathered && et == 0 && first_tile < num_tiles)
-        issue_staging(first_tile);
+    const int nwork = sc.count();
+    if (gathered && et == 0 && nwork > 0)
+        issue_staging(sc.item(0).tile);
     StageRegs<BN> nx;
-    if (pipe && first_tile < num_tiles)
-        stage_issue<BN>(p, s_cols, cnt, first_tile, a_tile_rows, a_row_off, r_in_tile, et, nx);
-    for (int tile = first_tile; tile < num_tiles; tile += tile_step, ++local) {
+    if (pipe && nwork > 0)
+        stage_issue<BN>(p, s_cols, cnt, sc.item(0).tile, a_tile_rows, a_row_off, r_in_tile, et, nx);
+    // Stream-K slots of this CTA (rank a_row_off / BM of its pair) and of the
+    // previous pair's CTA of the same rank, 128 rows x BN int32 each.
+    constexpr int kSlotVec = (BN >= 32 ? BN / 32 : 1) * 8 * 128; // int4 vectors per CTA slot
+    const int rank = a_row_off / BM;
+    for (int w = 0; w < nwork; ++w, ++local) {
+        const Seg it = sc.item(w);
+        const int tile = it.tile;
+        const bool park = PAIR && it.st1 < sc.S;             // K stages [0, st1): parked for the next pair
+        const bool owner = PAIR && !park && it.st0 > 0;      // the previous pair parked stages [0, st0)
         const int b = local & 1;
         const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
         const int arow = mb * a_tile_rows + a_row_off + r_in_tile; // A-operand row of this thread
@@ -285,8 +356,8 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                 if (k < cnt)
                     s_own[k * 128 + et] = __half2float(__ushort_as_half((unsigned short)nx.own_side[k]));
             named_barrier_sync(1, 128);
-            if (tile + tile_step < num_tiles)
-                stage_issue<BN>(p, s_cols, cnt, tile + tile_step, a_tile_rows, a_row_off, r_in_tile, et, nx);
+            if (w + 1 < nwork)
+                stage_issue<BN>(p, s_cols, cnt, sc.item(w + 1).tile, a_tile_rows, a_row_off, r_in_tile, et, nx);
         } else if (!RAW) {
             // Stage the tile's scales and outlier operands while the MMAs run.
             // Every load of the first round goes out before any is used (with
@@ -374,6 +445,64 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
         tc_fence_after();
         const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * BN);
 
+        if (park) {
+            // The tile's first stages: this row's int32 partials to the
+            // pair's slot (a warp stores 512 contiguous bytes per vector).
+            int4 *dst = reinterpret_cast<int4 *>(p.sk_part) + (size_t)(sc.first * 2 + rank) * kSlotVec + r_in_tile;
+#pragma unroll 1
+            for (int g = 0; g < BN / 32; ++g) {
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(tbase + g * 32, acc);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                    dst[(g * 8 + c4) * 128] = make_int4((int)acc[4 * c4], (int)acc[4 * c4 + 1], (int)acc[4 * c4 + 2],
+                                                        (int)acc[4 * c4 + 3]);
+            }
+        } else {
+        if (PAIR && owner) {
+            // The tile's last stages: the partials the previous pair parked
+            // (normally long ready) into this CTA's pipeline buffers, free
+            // now that its last MMAs are complete, by bulk copies.
+            bool ok = true;
+            if (et == 0) {
+                uint32_t *flag = p.sk_flag + (sc.first - 1) * 2 + rank;
+                uint32_t f = 0u;
+                const uint64_t t0 = global_timer_ns();
+                for (;;) {
+                    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(f) : "l"(flag) : "memory");
+                    if (f == 1u || global_timer_ns() - t0 > kWaitLimitNs)
+                        break;
+                    __nanosleep(64);
+                }
+                ok = f == 1u;
+                if (ok) {
+                    *flag = 0u; // ready for the next call
+                    fence_proxy_async_global();
+                    const uint8_t *src = reinterpret_cast<const uint8_t *>(
+                        reinterpret_cast<const int4 *>(p.sk_part) + (size_t)((sc.first - 1) * 2 + rank) * kSlotVec);
+                    constexpr uint32_t bytes = (uint32_t)kSlotVec * 16u;
+                    mbar_arrive_expect_tx(sbar, bytes);
+                    for (uint32_t off = 0; off < bytes; off += 32768u)
+                        bulk_load(smem_u32(sk_buf) + off, src + off, min(32768u, bytes - off), sbar);
+                    staged_pending = true;
+                }
+            }
+            if (named_barrier_or(1, 128, !ok)) {
+                if (!ok)
+                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                break;
+            }
+            const bool landed = mbar_wait(sbar, sph);
+            if (named_barrier_or(1, 128, !landed)) {
+                if (!landed)
+                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                break;
+            }
+            sph ^= 1u;
+            staged_pending = false;
+        }
+
         if constexpr (!SWAP) {
             const int i = arow;
             // More outlier columns than s_side holds at once: the columns go
@@ -422,6 +551,18 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                 uint32_t acc[32];
                 tmem_ld_32x32b_x32(tbase + g * 32, acc);
                 tmem_wait_ld();
+                if (owner && ch == 0) {
+                    // the parked partial products of this row's 32 columns
+                    const int4 *pp = reinterpret_cast<const int4 *>(sk_buf) + g * 8 * 128 + r_in_tile;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const int4 v = pp[c4 * 128];
+                        acc[4 * c4] += (uint32_t)v.x;
+                        acc[4 * c4 + 1] += (uint32_t)v.y;
+                        acc[4 * c4 + 2] += (uint32_t)v.z;
+                        acc[4 * c4 + 3] += (uint32_t)v.w;
+                    }
+                }
                 const int j0 = brow0 + g * 32;
                 if constexpr (RAW) {
                     int32_t *Yr = reinterpret_cast<int32_t *>(p.Y) + (int64_t)i * p.N;
@@ -706,6 +847,7 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                 }
             }
         }
+        } // not a parked part
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -714,18 +856,25 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
             else
                 mbar_arrive(tempty_bar(b));
         }
+        if (park) {
+            // every row of the CTA stored, then the flag (release)
+            __threadfence();
+            named_barrier_sync(1, 128);
+            if (et == 0)
+                asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p.sk_flag + sc.first * 2 + rank), "r"(1u) : "memory");
+        }
         if (gathered) {
             // every reader of s_side / s_scale is done: stage the next tile
             named_barrier_sync(1, 128);
-            if (et == 0 && tile + tile_step < num_tiles) {
+            if (et == 0 && w + 1 < nwork) {
                 fence_proxy_async_smem();
-                issue_staging(tile + tile_step);
+                issue_staging(sc.item(w + 1).tile);
             }
         }
     }
-    // A staging copy still in flight (the loop was left early) lands, and
-    // this warp's TMA stores complete, before the CTA may exit.
-    if (gathered && et == 0 && staged_pending)
+    // A staging or stream-K copy still in flight (the loop was left early)
+    // lands, and this warp's TMA stores complete, before the CTA may exit.
+    if (et == 0 && staged_pending)
         mbar_wait(sbar, sph);
     if (lane == 0 && stores_pending)
         bulk_wait_group0();
@@ -903,9 +1052,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
+        const Sched sc = make_sched(num_tiles, 0, blockIdx.x, gridDim.x, p.num_kb);
         run_epilogue<BN, SWAP, RAW, false>(p, &tmY, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
-                                           stage_bar, s_abort,
-                                           tmem_base, blockIdx.x, gridDim.x, num_tiles, BM, 0);
+                                           stage_bar, s_abort, tmem_base, sc, BM, 0, nullptr);
     }
 
     __syncthreads();
@@ -939,6 +1088,7 @@ struct SmemPair {
     static_assert(ALLOC <= 232448, "shared memory over the 227 KB per-CTA limit");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1024-byte alignment");
     static_assert(BN % 32 == 0 && BN <= 256, "pair MMA needs N a multiple of 32, at most 256");
+    static_assert(BM * BN * 4 <= SIDE_OFF, "a parked stream-K partial fits in the pipeline buffers");
 };
 
 // The prefill GEMM on CTA pairs (a cluster of two CTAs on one TPC). Each pair
@@ -1012,6 +1162,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     const int num_st = (p.num_kb + KS - 1) / KS; // stages per tile
     // K slices in stage `st` of a tile (the last one may hold fewer).
     auto slices = [&](int st) { return min(KS, p.num_kb - st * KS); };
+    // Whole tiles pair_id, pair_id + num_pairs, ..., then this pair's share
+    // of the stream-K tiles' stages; every role walks the same list.
+    const Sched sc = make_sched(num_tiles, p.sk_tiles, pair_id, num_pairs, num_st);
+    const int nwork = sc.count();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -1023,29 +1177,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             // The weight half (B) of the first stages goes out before the wait
             // for the quantizer's codes (A).
             int pre = 0;
-            if (pair_id < num_tiles) {
-                const int nb = pair_id / p.num_m_blk;
+            if (nwork > 0) {
+                const Seg f = sc.item(0);
+                const int nb = f.tile / p.num_m_blk;
                 const int b_row = nb * BN + (int)rank * (BN / 2);
-                pre = min(STAGES, num_st);
+                pre = min(STAGES, f.st1 - f.st0);
                 for (int s = 0; s < pre; ++s) {
-                    const int ns = slices(s);
+                    const int ns = slices(f.st0 + s);
                     if (leader)
                         mbar_arrive_expect_tx(full_bar(s), tx(ns));
                     for (int j = 0; j < ns; ++j)
                         tma_load_2d_pair(sbase + L::B_OFF + s * L::B_BYTES + j * L::B_SUB, &tmB, full_bar(s),
-                                         (s * KS + j) * BK, b_row);
+                                         ((f.st0 + s) * KS + j) * BK, b_row);
                 }
             }
             griddep_wait();
-            for (int tile = pair_id; tile < num_tiles && !*s_abort; tile += num_pairs) {
-                const int mb = tile % p.num_m_blk, nb = tile / p.num_m_blk;
+            for (int w = 0; w < nwork && !*s_abort; ++w) {
+                const Seg it = sc.item(w);
+                const int mb = it.tile % p.num_m_blk, nb = it.tile / p.num_m_blk;
                 const int a_row = mb * 2 * BM + (int)rank * BM;
                 const int b_row = nb * BN + (int)rank * (BN / 2);
-                for (int st = 0; st < num_st; ++st) {
+                for (int st = it.st0; st < it.st1; ++st) {
                     const int ns = slices(st);
                     const uint32_t a_dst = sbase + L::A_OFF + stage * L::A_BYTES;
                     const uint32_t b_dst = sbase + L::B_OFF + stage * L::B_BYTES;
-                    if (tile == pair_id && st < pre) {
+                    if (w == 0 && st - it.st0 < pre) {
                         for (int j = 0; j < ns; ++j)
                             tma_load_2d_pair(a_dst + j * L::A_SUB, &tmA, full_bar(stage), (st * KS + j) * BK, a_row);
                         if (++stage == STAGES) {
@@ -1082,7 +1238,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
             uint32_t tph[2] = {0u, 0u};
             constexpr uint32_t IDESC = idesc_i8(2 * BM, BN);
             int local = 0;
-            for (int tile = pair_id; tile < num_tiles && !*s_abort; tile += num_pairs, ++local) {
+            for (int w = 0; w < nwork && !*s_abort; ++w, ++local) {
+                const Seg it = sc.item(w);
                 const int b = local & 1;
                 if (!mbar_wait_cluster(tempty_bar(b), tph[b] ^ 1u)) {
                     report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
@@ -1092,7 +1249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
                 bool ok = true;
-                for (int st = 0; st < num_st; ++st) {
+                for (int st = it.st0; st < it.st1; ++st) {
                     if (!mbar_wait_poll(full_bar(stage), phase)) {
                         report(p, s_abort, LLMINT8_DEV_TIMEOUT_MMA);
                         ok = false;
@@ -1108,7 +1265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                             for (int k = 0; k < BK / UK; ++k)
                                 mma_i8_pair(d_tmem, smem_desc_k128(a0 + k * UK), smem_desc_k128(b0 + k * UK), IDESC,
-                                            (st | j | k) != 0 ? 1u : 0u);
+                                            (st != it.st0 || j != 0 || k != 0) ? 1u : 0u);
                         }
                     }
                     mma_commit_pair_mc(empty_bar(stage), 0x3); // both CTAs' stage is free
@@ -1129,8 +1286,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     } else {
         griddep_wait(); // SX, |O| and the outlier columns come from the quantizer
         run_epilogue<BN, false, RAW, true>(p, &tmY, warp, lane, s_side, s_scale, s_cols, tfull_bar(0), tempty_bar(0),
-                                           stage_bar, s_abort,
-                                           tmem_base, pair_id, num_pairs, num_tiles, 2 * BM, (int)rank * BM);
+                                           stage_bar, s_abort, tmem_base, sc, 2 * BM, (int)rank * BM,
+                                           smem + L::A_OFF);
     }
 
     tc_fence_before();
@@ -1349,7 +1506,7 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
     CUtensorMap ta, tb;
     if (!make_map_i8(&ta, dev.device, Aop, rows_a, a.K, BM) || !make_map_i8(&tb, dev.device, Bop, rows_b, a.K, BN))
         return cudaErrorInvalidValue;
-    KParams p;
+    KParams p{};
     p.rows_a = (int)rows_a;
     p.rows_b = (int)rows_b;
     p.K = (int)a.K;
@@ -1385,7 +1542,7 @@ cudaError_t run(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
 }
 
 template <int BN, int STAGES, int KS, bool RAW>
-cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream, bool stream_k)
 {
     using L = SmemPair<BN, STAGES, KS>;
     auto kern = k_gemm_i8_pair<BN, STAGES, KS, RAW>;
@@ -1400,7 +1557,7 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     CUtensorMap ta, tb;
     if (!make_map_i8(&ta, dev.device, a.A, a.M, a.K, BM) || !make_map_i8(&tb, dev.device, a.B, a.N, a.K, BN / 2))
         return cudaErrorInvalidValue;
-    KParams p;
+    KParams p{};
     p.rows_a = (int)a.M;
     p.rows_b = (int)a.N;
     p.K = (int)a.K;
@@ -1432,27 +1589,55 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.y_tma = y_map(a, false, dev, &ty) ? 1 : 0;
     const int tiles = p.num_m_blk * p.num_n_blk;
     const int pairs = std::min(tiles, dev.num_sms / 2);
+    // Stream-K: the last one to two rounds' worth of tiles (at least one tile
+    // per pair) split evenly over the pairs by K stages.
+    p.sk_tiles = 0;
+    p.sk_part = a.sk_part;
+    p.sk_flag = a.sk_flag;
+    if (stream_k) {
+        if (!a.sk_part || !a.sk_flag || pairs > kSkMaxPairs || tiles <= pairs)
+            return cudaErrorInvalidValue;
+        p.sk_tiles = tiles - (tiles / pairs - 1) * pairs;
+    }
     return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, ty, p);
 }
 
-// Tile width for CTA-pair tiles (256 x BN): the one that minimises tile
-// rounds times the time of one tile. A tile's time is proportional to its
-// width divided by the tensor pipe's efficiency at that width (measured on
-// B200: N = 224 runs at about 95% of the per-column rate of N = 256).
-int pick_bn_pair(int64_t M, int64_t N, int num_pairs)
+// Tile width for CTA-pair tiles (256 x BN), and whether the last tiles run
+// stream-K: the plan that minimises the tile rounds times the time of one
+// tile. A tile's time is proportional to its width divided by the tensor
+// pipe's efficiency at that width (measured on B200: N = 224 runs at about
+// 95% of the per-column rate of N = 256). Stream-K (N = 256 tiles, when the
+// workspace has the slots and a tile has at least two K stages) spreads the
+// tiles' work evenly over the pairs; its fix-ups (a parked partial per pair,
+// stored once and read once) are charged as 2% of the total.
+struct PairPlan {
+    int bn;
+    bool stream_k;
+};
+
+PairPlan pick_pair_plan(int64_t M, int64_t N, int64_t K, int num_pairs, bool sk_slots)
 {
     static const int cands[] = {256, 224, 192, 128};
     static const int eff_permille[] = {1000, 946, 920, 950};
-    int best = 256;
+    const int64_t m_blk = (M + 2 * BM - 1) / (2 * BM);
+    PairPlan best{256, false};
     int64_t best_cost = INT64_MAX;
     for (int i = 0; i < 4; ++i) {
         const int bn = cands[i];
-        const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + bn - 1) / bn);
-        const int64_t cost = ((tiles + num_pairs - 1) / num_pairs) * bn * 1000000 / eff_permille[i];
+        const int64_t tiles = m_blk * ((N + bn - 1) / bn);
+        const int64_t pairs = std::min<int64_t>(tiles, num_pairs);
+        const int64_t cost = ((tiles + pairs - 1) / pairs) * bn * 1000000 / eff_permille[i];
         if (cost < best_cost) {
             best_cost = cost;
-            best = bn;
+            best = PairPlan{bn, false};
         }
+    }
+    const int64_t tiles = m_blk * ((N + 255) / 256);
+    const int64_t stages = ((K + BK - 1) / BK + 1) / 2; // K stages of a tile (two 128-byte slices each)
+    if (sk_slots && num_pairs <= kSkMaxPairs && tiles > num_pairs && tiles % num_pairs != 0 && stages >= 2) {
+        const int64_t cost = tiles * 256 * 1020 / num_pairs;
+        if (cost < best_cost)
+            best = PairPlan{256, true};
     }
     return best;
 }
@@ -1482,11 +1667,12 @@ template <bool RAW>
 cudaError_t run_prefill(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
 {
     if (a.M >= 2 * BM && dev.num_sms >= 2) {
-        switch (pick_bn_pair(a.M, a.N, dev.num_sms / 2)) {
-        case 224: return run_pair<224, 3, 2, RAW>(a, dev, stream);
-        case 192: return run_pair<192, 3, 2, RAW>(a, dev, stream);
-        case 128: return run_pair<128, 4, 2, RAW>(a, dev, stream);
-        default: return run_pair<256, 3, 2, RAW>(a, dev, stream);
+        const PairPlan plan = pick_pair_plan(a.M, a.N, a.K, dev.num_sms / 2, a.sk_part && a.sk_flag);
+        switch (plan.bn) {
+        case 224: return run_pair<224, 3, 2, RAW>(a, dev, stream, false);
+        case 192: return run_pair<192, 3, 2, RAW>(a, dev, stream, false);
+        case 128: return run_pair<128, 4, 2, RAW>(a, dev, stream, false);
+        default: return run_pair<256, 3, 2, RAW>(a, dev, stream, plan.stream_k);
         }
     }
     switch (pick_bn(a.M, a.N, dev.num_sms)) {

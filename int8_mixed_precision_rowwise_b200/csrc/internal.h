@@ -20,6 +20,10 @@ constexpr size_t kSetWords = (LLMINT8_MAX_K + 31) / 32; // bitmap words of the w
 // Outlier columns whose operands the prefill GEMM's epilogue reads from
 // per-call gathered copies (more columns: it gathers them in place).
 constexpr int kGatherCols = 32;
+// Stream-K slots of the CTA-pair GEMM: one per pair (two CTAs x 128 rows x
+// up to 256 int32 columns) and a ready flag per CTA.
+constexpr int kSkMaxPairs = 80;
+constexpr size_t kSkSlotBytes = 2 * 128 * 256 * 4;
 // Row strides (in floats) of the gathered copies: the W side leaves room for
 // a whole last tile (up to 256 columns past N), both are 16-byte multiples.
 inline int64_t gather_stride_n(int64_t N) { return (N + 256 + 3) / 4 * 4; }
@@ -53,6 +57,11 @@ inline int64_t gather_stride_m(int64_t M) { return (M + 3) / 4 * 4; }
 //   ...      fp32   W's outlier columns, column-major [kGatherCols x np] (np = gather_stride_n(N))
 //   ...      fp32   SB, zero-padded [np]
 //   ...      fp32   X's outlier columns, column-major [kGatherCols x mp] (mp = gather_stride_m(M))
+//   CTA-pair GEMM (gather_n > 0 and M >= 256):
+//   ...      int32  stream-K partial accumulators [kSkMaxPairs] x kSkSlotBytes, rewritten
+//            by each call before they are read
+//   ...      uint32 stream-K ready flags [kSkMaxPairs x 2]: raised (1) by the parking CTA,
+//            cleared by the CTA that reads the partial, so 0 between calls
 struct Workspace {
     uint32_t *status;
     int32_t *count;
@@ -72,6 +81,8 @@ struct Workspace {
     float *sb_p;
     float *xo_t;
     int64_t np, mp;
+    int32_t *sk_part; // null without the stream-K regions
+    uint32_t *sk_flag;
     size_t bytes;
 };
 
@@ -108,6 +119,9 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
     char *wt = gather_n > 0 ? take((size_t)kGatherCols * np * 4) : nullptr;
     char *sp = gather_n > 0 ? take((size_t)np * 4) : nullptr;
     char *xo = gather_n > 0 ? take((size_t)kGatherCols * mp * 4) : nullptr;
+    const bool sk = gather_n > 0 && M >= 256;
+    char *skp = sk ? take((size_t)kSkMaxPairs * kSkSlotBytes) : nullptr;
+    char *skf = sk ? take((size_t)kSkMaxPairs * 2 * 4) : nullptr;
     if (ws) {
         ws->status = reinterpret_cast<uint32_t *>(hdr);
         ws->count = hdr ? reinterpret_cast<int32_t *>(hdr + 4) : nullptr;
@@ -128,6 +142,8 @@ inline size_t carve(char *base, int64_t M, int64_t K, bool with_codes, bool deco
         ws->xo_t = reinterpret_cast<float *>(xo);
         ws->np = np;
         ws->mp = mp;
+        ws->sk_part = reinterpret_cast<int32_t *>(skp);
+        ws->sk_flag = reinterpret_cast<uint32_t *>(skf);
         ws->bytes = off;
     }
     return off;
@@ -211,6 +227,9 @@ struct GemmArgs {
     // gathers W's and X's outlier values in place).
     const float *wt_t, *sb_p, *xo_t;
     int64_t np, mp;
+    // Stream-K slots and flags of the CTA-pair GEMM (null: whole tiles only).
+    int32_t *sk_part;
+    uint32_t *sk_flag;
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, const DeviceInfo &dev, cudaStream_t stream);

@@ -172,6 +172,14 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's earlier generic-proxy view of global memory (data it
+// acquired from another SM's stores) before its later async-proxy reads of
+// it (a bulk copy of that data into shared memory).
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 2-D tiled bulk copy shared -> global (TMA store) of the box at {x, y}; the
 // tensor map clips the parts of the box outside the tensor. Tracked as one
 // bulk async-group of the issuing thread.

@@ -322,6 +322,67 @@ def test_gemm_matches_torch_int_mm(lib, dev):
     assert torch.equal(acc, ref)
 
 
+# Stream-K: on a GPU with P = SMs / 2 CTA pairs, a prefill GEMM (M >= 256)
+# whose 256 x 256 tiles number more than P and not a multiple of P, with at
+# least two K stages (256 bytes of K) a tile, splits its last tiles over the
+# pairs by K stages when that beats every whole-tile width (charging the
+# split 2%). These shapes take that path on a 148-SM B200; the parked partial
+# sums must add up to the same int32 products bit for bit.
+def _takes_stream_k(M, N, K, sms):
+    P = sms // 2
+    m_blk = (M + 255) // 256
+    best = None
+    for bn, eff in ((256, 1000), (224, 946), (192, 920), (128, 950)):
+        tiles = m_blk * ((N + bn - 1) // bn)
+        pairs = min(tiles, P)
+        cost = (tiles + pairs - 1) // pairs * bn * 1000000 // eff
+        best = cost if best is None else min(best, cost)
+    tiles = m_blk * ((N + 255) // 256)
+    stages = ((K + 127) // 128 + 1) // 2
+    return tiles > P and tiles % P != 0 and stages >= 2 and tiles * 256 * 1020 // P < best
+
+
+STREAM_K_SHAPES = [(512, 10240, 4096), (300, 19000, 384), (256, 20480, 1152), (2048, 14336, 4224)]
+
+
+@pytest.mark.parametrize("M,N,K", STREAM_K_SHAPES)
+def test_gemm_stream_k_exact(lib, dev, M, N, K):
+    """The int32 product on the stream-K path (ragged M, N and last K stage
+    among the shapes) against torch._int_mm (cuBLAS), twice on one workspace
+    (the stream-K flags must be back at zero after a call) and once more from
+    a CUDA-graph replay."""
+    if torch.cuda.get_device_properties(dev).multi_processor_count == 148:
+        assert _takes_stream_k(M, N, K, 148)
+    rng = np.random.default_rng(M + N + K)
+    A = torch.from_numpy(rng.integers(-127, 128, size=(M, K), dtype=np.int8)).to(dev)
+    B = torch.from_numpy(rng.integers(-127, 128, size=(N, K), dtype=np.int8)).to(dev)
+    ref = torch._int_mm(A, B.t().contiguous())
+    ws = lib.get_workspace(lib.workspace_size(M, N, K), dev)
+    for _ in range(2):
+        acc = lib.gemm_s8s8s32(A, B, workspace=ws)
+        assert torch.equal(acc, ref)
+    acc.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lib.gemm_s8s8s32(A, B, acc=acc, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref)
+    del g
+    assert lib.read_status(ws, clear=False) == 0
+
+
+@pytest.mark.parametrize("M,N,K,nout", [(256, 20480, 1152, 5), (300, 19000, 384, 3)])
+def test_matmul_mixed_stream_k(lib, dev, oracle_mod, M, N, K, nout):
+    """The whole linear on the stream-K path against the oracle, every element."""
+    if torch.cuda.get_device_properties(dev).multi_processor_count == 148:
+        assert _takes_stream_k(M, N, K, 148)
+    lin = Linear("sk", M, N, K, nout, 40.0)
+    X16, _ = make_activations(lin, seed=5)
+    W16 = make_weight(lin, seed=5)
+    check_full(lib, dev, oracle_mod, X16, W16, 6.0)
+
+
 # ------------------------------------------------------------------ full linear
 
 def test_tiny_workload(lib, dev, oracle_mod):
