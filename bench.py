@@ -44,7 +44,8 @@ WORKLOAD = synthetic.BLOOM_BLOCK_2048
 METRIC = "int8-mixed linear TOPS (BLOOM-176B block linears, 2048 tokens)"
 UNIT = "TOPS"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_gemm_i8_bloom_block_traffic.txt")
-GEMM_SOURCES = [os.path.join(ROOT, "int8_mixed_precision_rowwise_b200", "csrc", f) for f in ("gemm.cu", "ptx.cuh")]
+GEMM_SOURCES = [os.path.join(ROOT, "int8_mixed_precision_rowwise_b200", "csrc", f)
+                for f in ("gemm.cu", "ptx.cuh", "sched.h")]
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")

@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libllmint8.so")
 SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "decode.cu", "tp.cu", "noalloc.cu"]
-HEADERS = ["internal.h", "ptx.cuh", "common.cuh"]
+HEADERS = ["internal.h", "ptx.cuh", "common.cuh", "sched.h"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -34,6 +34,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
+#include "sched.h"
 
 namespace llmint8 {
 
@@ -41,6 +42,7 @@ namespace {
 
 constexpr int BM = 128;       // MMA M: rows of the A operand per tile
 constexpr int BK = 128;       // K bytes per pipeline stage (one 128-byte swizzle row)
+static_assert(2 * BM == kPairRows && BK == kSliceBytes, "the pair plan's tile and slice sizes");
 constexpr int UK = 32;        // K per tcgen05.mma kind::i8
 constexpr int OC = 32;        // outlier columns staged per chunk in the epilogue
 constexpr int kStoreStage = 16384; // bytes at the end of s_side for the TMA-store staging (4 warps x 4 KB)
@@ -79,57 +81,6 @@ struct KParams {
     int32_t *sk_part;
     uint32_t *sk_flag;
 };
-
-// One unit of a CTA's (or pair's) work: K stages [st0, st1) of a tile.
-struct Seg {
-    int tile, st0, st1;
-};
-
-// The work of one CTA (or pair) `first` of `step`, in processing order:
-// whole tiles first, first + step, ... below the stream-K tiles; then its
-// share of the stream-K tiles' stages, a contiguous range of the stages of
-// those tiles in order, cut at tile boundaries and taken from its end to its
-// start. Each range spans at least one tile's stages and fewer than three
-// tiles (the stream-K tiles number between one and two per pair), so a
-// range is at most three segments: the part of a tile it ends in (parked
-// for the pair that holds the tile's last stage, and processed first, so
-// that no pair waits for one that is itself waiting), whole tiles, and the
-// part of a tile it starts in (whose other part the previous pair parked;
-// processed last).
-struct Sched {
-    int first, step, ndp, nseg, S;
-    Seg seg[3];
-    __device__ __forceinline__ int count() const { return ndp + nseg; }
-    __device__ __forceinline__ Seg item(int w) const
-    {
-        if (w < ndp)
-            return Seg{first + w * step, 0, S};
-        return seg[w - ndp];
-    }
-};
-
-__device__ __forceinline__ Sched make_sched(int num_tiles, int sk_tiles, int first, int step, int S)
-{
-    Sched sc;
-    sc.first = first;
-    sc.step = step;
-    sc.S = S;
-    sc.nseg = 0;
-    const int dp_end = num_tiles - sk_tiles;
-    sc.ndp = first < dp_end ? (dp_end - first + step - 1) / step : 0;
-    if (sk_tiles > 0) {
-        const int64_t U = (int64_t)sk_tiles * S;
-        const int64_t g0 = U * first / step;
-        int64_t e = U * (first + 1) / step;
-        while (e > g0 && sc.nseg < 3) {
-            const int64_t t = (e - 1) / S;
-            const int64_t lo = max(g0, t * S);
-            sc.seg[sc.nseg++] = Seg{dp_end + (int)t, (int)(lo - t * S), (int)(e - t * S)};
-            e = lo;
-        }
-    }
-    return sc;
-}
 
 template <int BN, int STAGES>
 struct Smem {
@@ -460,394 +411,396 @@ __device__ __forceinline__ void run_epilogue(const KParams &p, const CUtensorMap
                                                         (int)acc[4 * c4 + 3]);
             }
         } else {
-        if (PAIR && owner) {
-            // The tile's last stages: the partials the previous pair parked
-            // (normally long ready) into this CTA's pipeline buffers, free
-            // now that its last MMAs are complete, by bulk copies.
-            bool ok = true;
-            if (et == 0) {
-                uint32_t *flag = p.sk_flag + (sc.first - 1) * 2 + rank;
-                uint32_t f = 0u;
-                const uint64_t t0 = global_timer_ns();
-                for (;;) {
-                    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(f) : "l"(flag) : "memory");
-                    if (f == 1u || global_timer_ns() - t0 > kWaitLimitNs)
-                        break;
-                    __nanosleep(64);
+            if (PAIR && owner) {
+                // The tile's last stages: the partials the previous pair parked
+                // (normally long ready) into this CTA's pipeline buffers, free
+                // now that its last MMAs are complete, by bulk copies.
+                bool ok = true;
+                if (et == 0) {
+                    uint32_t *flag = p.sk_flag + (sc.first - 1) * 2 + rank;
+                    uint32_t f = 0u;
+                    const uint64_t t0 = global_timer_ns();
+                    for (;;) {
+                        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(f) : "l"(flag) : "memory");
+                        if (f == 1u || global_timer_ns() - t0 > kWaitLimitNs)
+                            break;
+                        __nanosleep(64);
+                    }
+                    ok = f == 1u;
+                    if (ok) {
+                        *flag = 0u; // ready for the next call
+                        fence_proxy_async_global();
+                        const uint8_t *src = reinterpret_cast<const uint8_t *>(
+                            reinterpret_cast<const int4 *>(p.sk_part) + (size_t)((sc.first - 1) * 2 + rank) * kSlotVec);
+                        constexpr uint32_t bytes = (uint32_t)kSlotVec * 16u;
+                        mbar_arrive_expect_tx(sbar, bytes);
+                        for (uint32_t off = 0; off < bytes; off += 32768u)
+                            bulk_load(smem_u32(sk_buf) + off, src + off, min(32768u, bytes - off), sbar);
+                        staged_pending = true;
+                    }
                 }
-                ok = f == 1u;
-                if (ok) {
-                    *flag = 0u; // ready for the next call
-                    fence_proxy_async_global();
-                    const uint8_t *src = reinterpret_cast<const uint8_t *>(
-                        reinterpret_cast<const int4 *>(p.sk_part) + (size_t)((sc.first - 1) * 2 + rank) * kSlotVec);
-                    constexpr uint32_t bytes = (uint32_t)kSlotVec * 16u;
-                    mbar_arrive_expect_tx(sbar, bytes);
-                    for (uint32_t off = 0; off < bytes; off += 32768u)
-                        bulk_load(smem_u32(sk_buf) + off, src + off, min(32768u, bytes - off), sbar);
-                    staged_pending = true;
+                if (named_barrier_or(1, 128, !ok)) {
+                    if (!ok)
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                    break;
                 }
+                const bool landed = mbar_wait(sbar, sph);
+                if (named_barrier_or(1, 128, !landed)) {
+                    if (!landed)
+                        report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+                    break;
+                }
+                sph ^= 1u;
+                staged_pending = false;
             }
-            if (named_barrier_or(1, 128, !ok)) {
-                if (!ok)
-                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
-                break;
-            }
-            const bool landed = mbar_wait(sbar, sph);
-            if (named_barrier_or(1, 128, !landed)) {
-                if (!landed)
-                    report(p, s_abort, LLMINT8_DEV_TIMEOUT_EPILOGUE);
-                break;
-            }
-            sph ^= 1u;
-            staged_pending = false;
-        }
 
-        if constexpr (!SWAP) {
-            const int i = arow;
-            // More outlier columns than s_side holds at once: the columns go
-            // in chunks of OC, outermost. Each chunk's W values are staged
-            // for the whole tile (one round of gathers, eight in flight per
-            // thread) and this row's X values go to registers once; between
-            // chunks the partial sums wait in the tile's own TMEM accumulator
-            // (fp32 bits in place of the int32 products), so each output
-            // still adds its outlier products in ascending column order.
-            const int nch = (RAW || fast) ? 1 : (cnt + OC - 1) / OC;
-            for (int ch = 0; ch < nch; ++ch) {
-            const int nk = min(OC, cnt - ch * OC);
-            if (!RAW && !fast) {
-                named_barrier_sync(1, 128); // the previous chunk's readers are done with s_side / s_cols
-                if (et < nk)
-                    s_cols[et] = p.col_idx[ch * OC + et];
-                named_barrier_sync(1, 128);
-                for (int base = 0; base < nk * BN; base += 32 * 128) { // 32 gathers in flight per thread
-                    float vals[32];
+            if constexpr (!SWAP) {
+                const int i = arow;
+                // More outlier columns than s_side holds at once: the columns go
+                // in chunks of OC, outermost. Each chunk's W values are staged
+                // for the whole tile (one round of gathers, eight in flight per
+                // thread) and this row's X values go to registers once; between
+                // chunks the partial sums wait in the tile's own TMEM accumulator
+                // (fp32 bits in place of the int32 products), so each output
+                // still adds its outlier products in ascending column order.
+                const int nch = (RAW || fast) ? 1 : (cnt + OC - 1) / OC;
+                for (int ch = 0; ch < nch; ++ch) {
+                const int nk = min(OC, cnt - ch * OC);
+                if (!RAW && !fast) {
+                    named_barrier_sync(1, 128); // the previous chunk's readers are done with s_side / s_cols
+                    if (et < nk)
+                        s_cols[et] = p.col_idx[ch * OC + et];
+                    named_barrier_sync(1, 128);
+                    for (int base = 0; base < nk * BN; base += 32 * 128) { // 32 gathers in flight per thread
+                        float vals[32];
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int idx = base + u * 128 + et;
-                        float v = 0.f;
-                        if (idx < nk * BN) {
-                            const int k = idx / BN, r = brow0 + (idx - k * BN);
-                            if (r < p.N)
-                                v = wtilde(p, r, s_cols[k]);
+                        for (int u = 0; u < 32; ++u) {
+                            const int idx = base + u * 128 + et;
+                            float v = 0.f;
+                            if (idx < nk * BN) {
+                                const int k = idx / BN, r = brow0 + (idx - k * BN);
+                                if (r < p.N)
+                                    v = wtilde(p, r, s_cols[k]);
+                            }
+                            vals[u] = v;
                         }
-                        vals[u] = v;
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const int idx = base + u * 128 + et;
+                            if (idx < nk * BN)
+                                s_side[idx] = vals[u];
+                        }
                     }
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int idx = base + u * 128 + et;
-                        if (idx < nk * BN)
-                            s_side[idx] = vals[u];
-                    }
+                    for (int k = 0; k < OC; ++k)
+                        own_side[k] =
+                            (k < nk && arow < p.M) ? __half2float(p.X16[(int64_t)arow * p.K + s_cols[k]]) : 0.f;
+                    named_barrier_sync(1, 128);
                 }
-#pragma unroll
-                for (int k = 0; k < OC; ++k)
-                    own_side[k] = (k < nk && arow < p.M) ? __half2float(p.X16[(int64_t)arow * p.K + s_cols[k]]) : 0.f;
-                named_barrier_sync(1, 128);
-            }
-            const bool last_chunk = ch == nch - 1;
+                const bool last_chunk = ch == nch - 1;
 #pragma unroll 1
-            for (int g = 0; g < BN / 32; ++g) {
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(tbase + g * 32, acc);
-                tmem_wait_ld();
-                if (owner && ch == 0) {
-                    // the parked partial products of this row's 32 columns
-                    const int4 *pp = reinterpret_cast<const int4 *>(sk_buf) + g * 8 * 128 + r_in_tile;
+                for (int g = 0; g < BN / 32; ++g) {
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(tbase + g * 32, acc);
+                    tmem_wait_ld();
+                    if (owner && ch == 0) {
+                        // the parked partial products of this row's 32 columns
+                        const int4 *pp = reinterpret_cast<const int4 *>(sk_buf) + g * 8 * 128 + r_in_tile;
 #pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        const int4 v = pp[c4 * 128];
-                        acc[4 * c4] += (uint32_t)v.x;
-                        acc[4 * c4 + 1] += (uint32_t)v.y;
-                        acc[4 * c4 + 2] += (uint32_t)v.z;
-                        acc[4 * c4 + 3] += (uint32_t)v.w;
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const int4 v = pp[c4 * 128];
+                            acc[4 * c4] += (uint32_t)v.x;
+                            acc[4 * c4 + 1] += (uint32_t)v.y;
+                            acc[4 * c4 + 2] += (uint32_t)v.z;
+                            acc[4 * c4 + 3] += (uint32_t)v.w;
+                        }
                     }
-                }
-                const int j0 = brow0 + g * 32;
-                if constexpr (RAW) {
-                    int32_t *Yr = reinterpret_cast<int32_t *>(p.Y) + (int64_t)i * p.N;
-                    if (i < p.M) {
+                    const int j0 = brow0 + g * 32;
+                    if constexpr (RAW) {
+                        int32_t *Yr = reinterpret_cast<int32_t *>(p.Y) + (int64_t)i * p.N;
+                        if (i < p.M) {
+                            if (j0 + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+                                for (int c = 0; c < 32; c += 4)
+                                    *reinterpret_cast<uint4 *>(Yr + j0 + c) =
+                                        make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                            } else {
+                                for (int c = 0; c < 32; ++c)
+                                    if (j0 + c < p.N)
+                                        Yr[j0 + c] = (int32_t)acc[c];
+                            }
+                        }
+                        continue;
+                    }
+                    float y[32];
+                    if (ch > 0) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            y[c] = __uint_as_float(acc[c]); // the partial sums the previous chunk left
+                    } else if (p.zx) {
+                        // Zero-point codes: sum_k (q - z_i) CB[j,k] = acc + (128 - z_i) R[j],
+                        // dequantized by SB[j] / (127 s_i) (s_i = 0: an all-zero row).
+                        const float zc = (float)(128 - own_z);
+                        const float inv = own_scale > 0.f ? __frcp_rn(127.0f * own_scale) : 0.f;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int j = j0 + c;
+                            const float rj = j < p.N ? (float)__ldg(p.rsum + j) : 0.f;
+                            y[c] = fmaf(zc, rj, (float)(int32_t)acc[c]) * (s_scale[g * 32 + c] * inv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
+                    }
+                    if (gathered && x_in_smem) {
+                        // X's outlier values of this row, staged in s_side after W's
+                        const float *xs = s_side + cnt * BN + r_in_tile; // staged in row order
+#pragma unroll 1
+                        for (int k = 0; k < cnt; ++k) {
+                            const float xv = xs[k * 128];
+                            const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                            for (int c4 = 0; c4 < 8; ++c4) {
+                                const float4 w = wrow[c4];
+                                y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                            }
+                        }
+                    } else if (pipe) {
+                        // A loop over the actual columns: the form unrolled over
+                        // OC below is about 1300 instructions per chunk, more
+                        // than the instruction cache keeps next to the rest.
+                        const float *s_own = s_side + cnt * BN;
+#pragma unroll 1
+                        for (int k = 0; k < cnt; ++k) {
+                            const float xv = s_own[k * 128 + et];
+                            const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                            for (int c4 = 0; c4 < 8; ++c4) {
+                                const float4 w = wrow[c4];
+                                y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                            }
+                        }
+                    } else if (fast) { // (gathered with X's values in registers, or gathered in place)
+#pragma unroll
+                        for (int k = 0; k < OC; ++k) {
+                            if (k < cnt) {
+                                const float xv = own_side[k];
+                                const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                                for (int c4 = 0; c4 < 8; ++c4) {
+                                    const float4 w = wrow[c4];
+                                    y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                    y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                    y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                    y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                                }
+                            }
+                        }
+                    } else {
+                        // chunk ch of the outlier columns (staged above; unrolled
+                        // over the OC slots so that own_side stays in registers)
+#pragma unroll
+                        for (int k = 0; k < OC; ++k) {
+                            if (k < nk) {
+                                const float xv = own_side[k];
+                                const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
+#pragma unroll
+                                for (int c4 = 0; c4 < 8; ++c4) {
+                                    const float4 w = wrow[c4];
+                                    y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
+                                    y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
+                                    y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
+                                    y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                                }
+                            }
+                        }
+                        if (!last_chunk) {
+                            uint32_t part[32];
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                part[c] = __float_as_uint(y[c]);
+                            tmem_st_32x32b_x32(tbase + g * 32, part);
+                            continue;
+                        }
+                    }
+                    if (p.bias || p.act) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int j = j0 + c;
+                            const float bv = (p.bias && j < p.N) ? __half2float(__ldg(p.bias + j)) : 0.f;
+                            y[c] = bias_act(y[c], bv, p.act);
+                        }
+                    }
+                    if (i < p.M && p.out_f32) {
+                        // fp32 partial output (tensor-parallel row split: summed across ranks afterwards)
+                        float *Yr = reinterpret_cast<float *>(p.Y) + (int64_t)i * p.N;
                         if (j0 + 32 <= p.N && (p.N & 3) == 0) {
 #pragma unroll
                             for (int c = 0; c < 32; c += 4)
-                                *reinterpret_cast<uint4 *>(Yr + j0 + c) =
-                                    make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                                *reinterpret_cast<float4 *>(Yr + j0 + c) =
+                                    make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
                         } else {
                             for (int c = 0; c < 32; ++c)
                                 if (j0 + c < p.N)
-                                    Yr[j0 + c] = (int32_t)acc[c];
+                                    Yr[j0 + c] = y[c];
                         }
-                    }
-                    continue;
-                }
-                float y[32];
-                if (ch > 0) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        y[c] = __uint_as_float(acc[c]); // the partial sums the previous chunk left
-                } else if (p.zx) {
-                    // Zero-point codes: sum_k (q - z_i) CB[j,k] = acc + (128 - z_i) R[j],
-                    // dequantized by SB[j] / (127 s_i) (s_i = 0: an all-zero row).
-                    const float zc = (float)(128 - own_z);
-                    const float inv = own_scale > 0.f ? __frcp_rn(127.0f * own_scale) : 0.f;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int j = j0 + c;
-                        const float rj = j < p.N ? (float)__ldg(p.rsum + j) : 0.f;
-                        y[c] = fmaf(zc, rj, (float)(int32_t)acc[c]) * (s_scale[g * 32 + c] * inv);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[g * 32 + c]) * kInv127Sq;
-                }
-                if (gathered && x_in_smem) {
-                    // X's outlier values of this row, staged in s_side after W's
-                    const float *xs = s_side + cnt * BN + r_in_tile; // staged in row order
-#pragma unroll 1
-                    for (int k = 0; k < cnt; ++k) {
-                        const float xv = xs[k * 128];
-                        const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
-#pragma unroll
-                        for (int c4 = 0; c4 < 8; ++c4) {
-                            const float4 w = wrow[c4];
-                            y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
-                            y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
-                            y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
-                            y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
+                    } else if (tma_st && (g | 1) < BN / 32) {
+                        // chunk g is half of a full 64-column group: into this
+                        // warp's staging buffer (row = lane, 16-byte pieces
+                        // swizzled by row), and the group out by one TMA store
+                        if ((g & 1) == 0) {
+                            if (lane == 0 && stores_pending)
+                                bulk_wait_group_read0(); // the previous group has left obuf
+                            __syncwarp();
                         }
-                    }
-                } else if (pipe) {
-                    // A loop over the actual columns: the form unrolled over
-                    // OC below is about 1300 instructions per chunk, more
-                    // than the instruction cache keeps next to the rest.
-                    const float *s_own = s_side + cnt * BN;
-#pragma unroll 1
-                    for (int k = 0; k < cnt; ++k) {
-                        const float xv = s_own[k * 128 + et];
-                        const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
 #pragma unroll
-                        for (int c4 = 0; c4 < 8; ++c4) {
-                            const float4 w = wrow[c4];
-                            y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
-                            y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
-                            y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
-                            y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
-                        }
-                    }
-                } else if (fast) { // (gathered with X's values in registers, or gathered in place)
-#pragma unroll
-                    for (int k = 0; k < OC; ++k) {
-                        if (k < cnt) {
-                            const float xv = own_side[k];
-                            const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
-#pragma unroll
-                            for (int c4 = 0; c4 < 8; ++c4) {
-                                const float4 w = wrow[c4];
-                                y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
-                                y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
-                                y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
-                                y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
-                            }
-                        }
-                    }
-                } else {
-                    // chunk ch of the outlier columns (staged above; unrolled
-                    // over the OC slots so that own_side stays in registers)
-#pragma unroll
-                    for (int k = 0; k < OC; ++k) {
-                        if (k < nk) {
-                            const float xv = own_side[k];
-                            const float4 *wrow = reinterpret_cast<const float4 *>(s_side + k * BN + g * 32);
-#pragma unroll
-                            for (int c4 = 0; c4 < 8; ++c4) {
-                                const float4 w = wrow[c4];
-                                y[4 * c4 + 0] = fmaf(xv, w.x, y[4 * c4 + 0]);
-                                y[4 * c4 + 1] = fmaf(xv, w.y, y[4 * c4 + 1]);
-                                y[4 * c4 + 2] = fmaf(xv, w.z, y[4 * c4 + 2]);
-                                y[4 * c4 + 3] = fmaf(xv, w.w, y[4 * c4 + 3]);
-                            }
-                        }
-                    }
-                    if (!last_chunk) {
-                        uint32_t part[32];
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            part[c] = __float_as_uint(y[c]);
-                        tmem_st_32x32b_x32(tbase + g * 32, part);
-                        continue;
-                    }
-                }
-                if (p.bias || p.act) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int j = j0 + c;
-                        const float bv = (p.bias && j < p.N) ? __half2float(__ldg(p.bias + j)) : 0.f;
-                        y[c] = bias_act(y[c], bv, p.act);
-                    }
-                }
-                if (i < p.M && p.out_f32) {
-                    // fp32 partial output (tensor-parallel row split: summed across ranks afterwards)
-                    float *Yr = reinterpret_cast<float *>(p.Y) + (int64_t)i * p.N;
-                    if (j0 + 32 <= p.N && (p.N & 3) == 0) {
-#pragma unroll
-                        for (int c = 0; c < 32; c += 4)
-                            *reinterpret_cast<float4 *>(Yr + j0 + c) = make_float4(y[c], y[c + 1], y[c + 2], y[c + 3]);
-                    } else {
-                        for (int c = 0; c < 32; ++c)
-                            if (j0 + c < p.N)
-                                Yr[j0 + c] = y[c];
-                    }
-                } else if (tma_st && (g | 1) < BN / 32) {
-                    // chunk g is half of a full 64-column group: into this
-                    // warp's staging buffer (row = lane, 16-byte pieces
-                    // swizzled by row), and the group out by one TMA store
-                    if ((g & 1) == 0) {
-                        if (lane == 0 && stores_pending)
-                            bulk_wait_group_read0(); // the previous group has left obuf
-                        __syncwarp();
-                    }
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 pk;
-                        __half2 *h = reinterpret_cast<__half2 *>(&pk);
-                        h[0] = __floats2half2_rn(y[8 * c8 + 0], y[8 * c8 + 1]);
-                        h[1] = __floats2half2_rn(y[8 * c8 + 2], y[8 * c8 + 3]);
-                        h[2] = __floats2half2_rn(y[8 * c8 + 4], y[8 * c8 + 5]);
-                        h[3] = __floats2half2_rn(y[8 * c8 + 6], y[8 * c8 + 7]);
-                        const int piece = ((g & 1) * 4 + c8) ^ (lane & 7);
-                        *reinterpret_cast<uint4 *>(obuf + lane * 128 + piece * 16) = pk;
-                    }
-                    if (g & 1) {
-                        fence_proxy_async_smem(); // this lane's pieces, before the async proxy reads them
-                        __syncwarp();
-                        // (a box entirely past M or N has nothing to write; a
-                        // staging buffer off its 1024-byte alignment or outside
-                        // s_side, or a column not on a 16-byte boundary, is
-                        // reported and not stored)
-                        const int x0 = brow0 + (g - 1) * 32, y0 = arow - lane;
-                        const uint32_t ob = smem_u32(obuf), sb0 = smem_u32(s_side);
-                        const bool sane = (ob & 1023u) == 0 && ob >= sb0 && ob + 4096u <= sb0 + kSideBytes &&
-                                          (x0 & 7) == 0 && x0 >= 0 && y0 >= 0;
-                        if (lane == 0 && !sane)
-                            atomicOr(p.status, LLMINT8_DEV_BAD_STORE);
-                        if (lane == 0 && sane && y0 < p.M && x0 < p.N) {
-                            tma_store_2d(tmY, ob, x0, y0);
-                            bulk_commit_group();
-                            stores_pending = true;
-                        }
-                    }
-                } else if (i < p.M) {
-                    __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
-                    if (j0 + 32 <= p.N && (p.N & 7) == 0) {
-#pragma unroll
-                        for (int c = 0; c < 32; c += 8) {
+                        for (int c8 = 0; c8 < 4; ++c8) {
                             uint4 pk;
                             __half2 *h = reinterpret_cast<__half2 *>(&pk);
-                            h[0] = __floats2half2_rn(y[c + 0], y[c + 1]);
-                            h[1] = __floats2half2_rn(y[c + 2], y[c + 3]);
-                            h[2] = __floats2half2_rn(y[c + 4], y[c + 5]);
-                            h[3] = __floats2half2_rn(y[c + 6], y[c + 7]);
-                            *reinterpret_cast<uint4 *>(Yr + j0 + c) = pk;
+                            h[0] = __floats2half2_rn(y[8 * c8 + 0], y[8 * c8 + 1]);
+                            h[1] = __floats2half2_rn(y[8 * c8 + 2], y[8 * c8 + 3]);
+                            h[2] = __floats2half2_rn(y[8 * c8 + 4], y[8 * c8 + 5]);
+                            h[3] = __floats2half2_rn(y[8 * c8 + 6], y[8 * c8 + 7]);
+                            const int piece = ((g & 1) * 4 + c8) ^ (lane & 7);
+                            *reinterpret_cast<uint4 *>(obuf + lane * 128 + piece * 16) = pk;
+                        }
+                        if (g & 1) {
+                            fence_proxy_async_smem(); // this lane's pieces, before the async proxy reads them
+                            __syncwarp();
+                            // (a box entirely past M or N has nothing to write; a
+                            // staging buffer off its 1024-byte alignment or outside
+                            // s_side, or a column not on a 16-byte boundary, is
+                            // reported and not stored)
+                            const int x0 = brow0 + (g - 1) * 32, y0 = arow - lane;
+                            const uint32_t ob = smem_u32(obuf), sb0 = smem_u32(s_side);
+                            const bool sane = (ob & 1023u) == 0 && ob >= sb0 && ob + 4096u <= sb0 + kSideBytes &&
+                                              (x0 & 7) == 0 && x0 >= 0 && y0 >= 0;
+                            if (lane == 0 && !sane)
+                                atomicOr(p.status, LLMINT8_DEV_BAD_STORE);
+                            if (lane == 0 && sane && y0 < p.M && x0 < p.N) {
+                                tma_store_2d(tmY, ob, x0, y0);
+                                bulk_commit_group();
+                                stores_pending = true;
+                            }
+                        }
+                    } else if (i < p.M) {
+                        __half *Yr = reinterpret_cast<__half *>(p.Y) + (int64_t)i * p.N;
+                        if (j0 + 32 <= p.N && (p.N & 7) == 0) {
+#pragma unroll
+                            for (int c = 0; c < 32; c += 8) {
+                                uint4 pk;
+                                __half2 *h = reinterpret_cast<__half2 *>(&pk);
+                                h[0] = __floats2half2_rn(y[c + 0], y[c + 1]);
+                                h[1] = __floats2half2_rn(y[c + 2], y[c + 3]);
+                                h[2] = __floats2half2_rn(y[c + 4], y[c + 5]);
+                                h[3] = __floats2half2_rn(y[c + 6], y[c + 7]);
+                                *reinterpret_cast<uint4 *>(Yr + j0 + c) = pk;
+                            }
+                        } else {
+                            for (int c = 0; c < 32; ++c)
+                                if (j0 + c < p.N)
+                                    Yr[j0 + c] = __float2half_rn(y[c]);
+                        }
+                    }
+                }
+                if (!last_chunk)
+                    tmem_wait_st(); // the partial sums are in TMEM before the next chunk reads them
+                }
+            } else {
+                // Decode form: this thread owns output feature j = arow; the
+                // accumulator columns are tokens brow0 .. brow0 + BN - 1.
+                const int j = arow;
+                uint32_t acc[BN];
+                if constexpr (BN == 32) {
+                    tmem_ld_32x32b_x32(tbase, acc);
+                } else {
+                    tmem_ld_32x32b_x16(tbase, acc);
+                }
+                tmem_wait_ld();
+                if constexpr (RAW) {
+                    if (j < p.N) {
+                        int32_t *Yc = reinterpret_cast<int32_t *>(p.Y) + j;
+#pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            if (brow0 + c < p.M)
+                                Yc[(int64_t)(brow0 + c) * p.N] = (int32_t)acc[c];
+                    }
+                } else {
+                    float y[BN];
+                    if (p.zx) {
+                        // Zero-point codes (see the other form): token c = brow0 + c.
+                        const float rj = j < p.N ? (float)__ldg(p.rsum + j) : 0.f;
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) {
+                            const int r = brow0 + c;
+                            const float zc = r < p.M ? (float)(128 - __ldg(p.zx + r)) : 0.f;
+                            const float sc = s_scale[c];
+                            const float inv = sc > 0.f ? __frcp_rn(127.0f * sc) : 0.f;
+                            y[c] = fmaf(zc, rj, (float)(int32_t)acc[c]) * (own_scale * inv);
                         }
                     } else {
-                        for (int c = 0; c < 32; ++c)
-                            if (j0 + c < p.N)
-                                Yr[j0 + c] = __float2half_rn(y[c]);
+#pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
                     }
-                }
-            }
-            if (!last_chunk)
-                tmem_wait_st(); // the partial sums are in TMEM before the next chunk reads them
-            }
-        } else {
-            // Decode form: this thread owns output feature j = arow; the
-            // accumulator columns are tokens brow0 .. brow0 + BN - 1.
-            const int j = arow;
-            uint32_t acc[BN];
-            if constexpr (BN == 32) {
-                tmem_ld_32x32b_x32(tbase, acc);
-            } else {
-                tmem_ld_32x32b_x16(tbase, acc);
-            }
-            tmem_wait_ld();
-            if constexpr (RAW) {
-                if (j < p.N) {
-                    int32_t *Yc = reinterpret_cast<int32_t *>(p.Y) + j;
+                    if (fast) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (brow0 + c < p.M)
-                            Yc[(int64_t)(brow0 + c) * p.N] = (int32_t)acc[c];
-                }
-            } else {
-                float y[BN];
-                if (p.zx) {
-                    // Zero-point codes (see the other form): token c = brow0 + c.
-                    const float rj = j < p.N ? (float)__ldg(p.rsum + j) : 0.f;
+                        for (int k = 0; k < OC; ++k) {
+                            if (k < cnt) {
+                                const float wv = own_side[k];
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        const int r = brow0 + c;
-                        const float zc = r < p.M ? (float)(128 - __ldg(p.zx + r)) : 0.f;
-                        const float sc = s_scale[c];
-                        const float inv = sc > 0.f ? __frcp_rn(127.0f * sc) : 0.f;
-                        y[c] = fmaf(zc, rj, (float)(int32_t)acc[c]) * (own_scale * inv);
-                    }
-                } else {
+                                for (int c = 0; c < BN; ++c)
+                                    y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                            }
+                        }
+                    } else {
+                        for (int ch = 0; ch < cnt; ch += OC) {
+                            const int nk = min(OC, cnt - ch);
+                            named_barrier_sync(1, 128);
+                            for (int idx = et; idx < nk * BN; idx += 128) {
+                                const int k = idx / BN, c = idx - k * BN;
+                                const int r = brow0 + c;
+                                s_side[idx] =
+                                    r < p.M ? __half2float(p.X16[(int64_t)r * p.K + p.col_idx[ch + k]]) : 0.f;
+                            }
+                            named_barrier_sync(1, 128);
+                            for (int k = 0; k < nk; ++k) {
+                                const float wv = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        y[c] = (float)(int32_t)acc[c] * (own_scale * s_scale[c]) * kInv127Sq;
-                }
-                if (fast) {
-#pragma unroll
-                    for (int k = 0; k < OC; ++k) {
-                        if (k < cnt) {
-                            const float wv = own_side[k];
-#pragma unroll
-                            for (int c = 0; c < BN; ++c)
-                                y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                                for (int c = 0; c < BN; ++c)
+                                    y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
+                            }
                         }
                     }
-                } else {
-                    for (int ch = 0; ch < cnt; ch += OC) {
-                        const int nk = min(OC, cnt - ch);
-                        named_barrier_sync(1, 128);
-                        for (int idx = et; idx < nk * BN; idx += 128) {
-                            const int k = idx / BN, c = idx - k * BN;
-                            const int r = brow0 + c;
-                            s_side[idx] =
-                                r < p.M ? __half2float(p.X16[(int64_t)r * p.K + p.col_idx[ch + k]]) : 0.f;
-                        }
-                        named_barrier_sync(1, 128);
-                        for (int k = 0; k < nk; ++k) {
-                            const float wv = j < p.N ? wtilde(p, j, p.col_idx[ch + k]) : 0.f;
+                    if (p.bias || p.act) {
+                        const float bv = (p.bias && j < p.N) ? __half2float(__ldg(p.bias + j)) : 0.f;
 #pragma unroll
-                            for (int c = 0; c < BN; ++c)
-                                y[c] = fmaf(wv, s_side[k * BN + c], y[c]);
-                        }
+                        for (int c = 0; c < BN; ++c)
+                            y[c] = bias_act(y[c], bv, p.act);
                     }
-                }
-                if (p.bias || p.act) {
-                    const float bv = (p.bias && j < p.N) ? __half2float(__ldg(p.bias + j)) : 0.f;
+                    if (j < p.N && p.out_f32) {
+                        float *Yc = reinterpret_cast<float *>(p.Y) + j;
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        y[c] = bias_act(y[c], bv, p.act);
-                }
-                if (j < p.N && p.out_f32) {
-                    float *Yc = reinterpret_cast<float *>(p.Y) + j;
+                        for (int c = 0; c < BN; ++c)
+                            if (brow0 + c < p.M)
+                                Yc[(int64_t)(brow0 + c) * p.N] = y[c];
+                    } else if (j < p.N) {
+                        __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (brow0 + c < p.M)
-                            Yc[(int64_t)(brow0 + c) * p.N] = y[c];
-                } else if (j < p.N) {
-                    __half *Yc = reinterpret_cast<__half *>(p.Y) + j;
-#pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (brow0 + c < p.M)
-                            Yc[(int64_t)(brow0 + c) * p.N] = __float2half_rn(y[c]);
+                        for (int c = 0; c < BN; ++c)
+                            if (brow0 + c < p.M)
+                                Yc[(int64_t)(brow0 + c) * p.N] = __float2half_rn(y[c]);
+                    }
                 }
             }
         }
-        } // not a parked part
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -1595,51 +1548,11 @@ cudaError_t run_pair(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stre
     p.sk_part = a.sk_part;
     p.sk_flag = a.sk_flag;
     if (stream_k) {
-        if (!a.sk_part || !a.sk_flag || pairs > kSkMaxPairs || tiles <= pairs)
+        if (!a.sk_part || !a.sk_flag || pairs > kSkMaxPairs || tiles <= pairs || KS != kStageSlices)
             return cudaErrorInvalidValue;
-        p.sk_tiles = tiles - (tiles / pairs - 1) * pairs;
+        p.sk_tiles = sk_tile_count(tiles, pairs);
     }
     return launch_dependent(kern, 2 * pairs, L::ALLOC, stream, ta, tb, ty, p);
-}
-
-// Tile width for CTA-pair tiles (256 x BN), and whether the last tiles run
-// stream-K: the plan that minimises the tile rounds times the time of one
-// tile. A tile's time is proportional to its width divided by the tensor
-// pipe's efficiency at that width (measured on B200: N = 224 runs at about
-// 95% of the per-column rate of N = 256). Stream-K (N = 256 tiles, when the
-// workspace has the slots and a tile has at least two K stages) spreads the
-// tiles' work evenly over the pairs; its fix-ups (a parked partial per pair,
-// stored once and read once) are charged as 2% of the total.
-struct PairPlan {
-    int bn;
-    bool stream_k;
-};
-
-PairPlan pick_pair_plan(int64_t M, int64_t N, int64_t K, int num_pairs, bool sk_slots)
-{
-    static const int cands[] = {256, 224, 192, 128};
-    static const int eff_permille[] = {1000, 946, 920, 950};
-    const int64_t m_blk = (M + 2 * BM - 1) / (2 * BM);
-    PairPlan best{256, false};
-    int64_t best_cost = INT64_MAX;
-    for (int i = 0; i < 4; ++i) {
-        const int bn = cands[i];
-        const int64_t tiles = m_blk * ((N + bn - 1) / bn);
-        const int64_t pairs = std::min<int64_t>(tiles, num_pairs);
-        const int64_t cost = ((tiles + pairs - 1) / pairs) * bn * 1000000 / eff_permille[i];
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = PairPlan{bn, false};
-        }
-    }
-    const int64_t tiles = m_blk * ((N + 255) / 256);
-    const int64_t stages = ((K + BK - 1) / BK + 1) / 2; // K stages of a tile (two 128-byte slices each)
-    if (sk_slots && num_pairs <= kSkMaxPairs && tiles > num_pairs && tiles % num_pairs != 0 && stages >= 2) {
-        const int64_t cost = tiles * 256 * 1020 / num_pairs;
-        if (cost < best_cost)
-            best = PairPlan{256, true};
-    }
-    return best;
 }
 
 // Tile width for the persistent prefill GEMM: the one that minimises the
@@ -1667,7 +1580,7 @@ template <bool RAW>
 cudaError_t run_prefill(const GemmArgs &a, const DeviceInfo &dev, cudaStream_t stream)
 {
     if (a.M >= 2 * BM && dev.num_sms >= 2) {
-        const PairPlan plan = pick_pair_plan(a.M, a.N, a.K, dev.num_sms / 2, a.sk_part && a.sk_flag);
+        const PairPlan plan = pick_pair_plan(a.M, a.N, a.K, dev.num_sms / 2, a.sk_part && a.sk_flag, kSkMaxPairs);
         switch (plan.bn) {
         case 224: return run_pair<224, 3, 2, RAW>(a, dev, stream, false);
         case 192: return run_pair<192, 3, 2, RAW>(a, dev, stream, false);
