@@ -487,7 +487,9 @@ def measure_secondary(L, dev, index):
     width, M = 1, 8, 32) in HBM GB/s of algorithmic bytes. Each is timed as a
     CUDA graph of back-to-back calls; the quantizer rotates over 8 inputs
     (256 MB, twice L2), the decode weights (205 MB) exceed L2 by themselves.
-    Every leg carries the SM clocks sampled while it ran."""
+    The 2048 x 16384 x 4096 prefill linear (TOPS) is timed the same way (its
+    output, 67 MB, and weight, 67 MB, together exceed L2). Every leg carries
+    the SM clocks sampled while it ran."""
     import torch
 
     peaks, _ = load_peaks()
@@ -521,6 +523,20 @@ def measure_secondary(L, dev, index):
         out[f"decode_M{M}"] = {"us": round(ms * 1e3, 2), "GBs": round(byts / (ms * 1e-3) / 1e9, 1),
                                "frac": round(byts / (ms * 1e-3) / 1e9 / hbm, 3), "clocks": clk.summary()}
         del layer, X, Y
+    torch.cuda.empty_cache()
+    # The 7B-class prefill linear (2048 x 16384 x 4096) through llmint8_matmul_mixed:
+    # quantizer, outlier gather and GEMM back to back, as in the zero-point leg below.
+    lin = synthetic.PREFILL_7B.linears[0]
+    X, W, _ = synthetic.torch_device_problem(lin, 0, dev)
+    layer = L.Int8MixedLinear.from_fp16(W, 6.0, keep_fp16_weights=True)
+    del W
+    Y = torch.empty((lin.M, lin.N), dtype=torch.float16, device=dev)
+    with ClockSampler(index) as clk:
+        ms = graph_time_ms([lambda: layer(X, Y)], reps=10)
+    out["prefill_2048x16384x4096"] = {"call_us": round(ms * 1e3, 1),
+                                      "call_tops": round(ops_of(lin) / (ms * 1e-3) / 1e12, 1),
+                                      "clocks": clk.summary()}
+    del layer, X, Y
     torch.cuda.empty_cache()
     out["zero_point"] = zero_point_times(L, dev, hbm, index)
     # Last: the per-linear GEMMs run the GPU at its power cap for seconds.
@@ -692,8 +708,9 @@ def run_reference(args, rank, world):
 
 def run_profile_case(args):
     """A minimal driver for ncu captures: set up the named BLOOM linear (or
-    'all' four), run one warm-up pass, then --steps passes inside an NVTX
-    range 'timed_steps'. Prints nothing; exits 0 on success."""
+    'all' four, or 'prefill' for the 2048 x 16384 x 4096 linear), run one
+    warm-up pass, then --steps passes inside an NVTX range 'timed_steps'.
+    Prints nothing; exits 0 on success."""
     import torch
 
     import int8_mixed_precision_rowwise_b200 as L
@@ -741,6 +758,8 @@ def run_profile_case(args):
         torch.cuda.nvtx.range_pop()
         return
     lins = [l for l in WORKLOAD.linears if args.profile_case in ("all", l.name)]
+    if args.profile_case == "prefill":
+        lins = list(synthetic.PREFILL_7B.linears)
     if not lins:
         raise SystemExit(f"unknown case {args.profile_case!r}")
     layers, xs, ys = [], [], []
@@ -769,7 +788,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--profile-case", default=None,
                     help="ncu driver: run only this BLOOM linear ('qkv', 'attn_out', 'fc1', 'fc2' or 'all'), "
-                         "the 4096 x 4096 'quantizer', 'decode_M1' / 'decode_M8' / 'decode_M32', or "
+                         "the 2048 x 16384 x 4096 'prefill' linear, the 4096 x 4096 'quantizer', "
+                         "'decode_M1' / 'decode_M8' / 'decode_M32', or "
                          "cuBLAS's int8 GEMM on a linear's shape ('cublas_int8_attn_out', ...)")
     args = ap.parse_args()
     if args.profile_case:
