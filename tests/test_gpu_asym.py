@@ -98,7 +98,9 @@ def test_code_row_sums_exact(lib, dev, oracle_mod):
 
 @pytest.mark.parametrize("M,N,K,nout,give_w16", [
     (333, 777, 1024, 5, True), (333, 777, 1024, 5, False), (100, 700, 1024, 8, False),
-    (16, 640, 1024, 6, True), (32, 300, 512, 3, False), (1024, 8192, 256, 6, True), (200, 384, 80, 2, True)])
+    (16, 640, 1024, 6, True), (32, 300, 512, 3, False), (1024, 8192, 256, 6, True), (200, 384, 80, 2, True),
+    # 150 tiles of 256 x 256 on 74 CTA pairs: the last tiles run stream-K
+    (300, 19000, 384, 5, True)])
 def test_matmul_asym_matches_oracle(lib, dev, oracle_mod, M, N, K, nout, give_w16):
     lin = Linear("a", M, N, K, nout, 60.0)
     X16, _ = make_activations(lin, seed=M + N)

@@ -534,7 +534,32 @@ def test_matmul_mixed_bias_activation(lib, dev, oracle_mod, M, N, K, act):
     assert not bad.any(), f"{bad.sum()} outside tolerance, worst {np.abs(y - r['Y']).max()}"
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 520, 1040), (4, 640, 1024), (64, 256, 4096)])
+@pytest.mark.parametrize("M,N,K,nout,act,give_w16", [(300, 19000, 384, 40, "gelu_tanh", True),
+                                                    (300, 19000, 384, 5, None, False)])
+def test_stream_k_epilogue_variants(lib, dev, oracle_mod, M, N, K, nout, act, give_w16):
+    """Stream-K (150 tiles on 74 pairs) under the other epilogue forms: more
+    than 32 outlier columns (two chunks, the partial sums kept in TMEM between
+    them) with a bias and GELU, and W's outlier columns recovered from CB with
+    a bias only; against the oracle with the bias/activation tolerance."""
+    if torch.cuda.get_device_properties(dev).multi_processor_count == 148:
+        assert _takes_stream_k(M, N, K, 148)
+    lin = Linear("ske", M, N, K, nout, 40.0)
+    X16, _ = make_activations(lin, seed=nout)
+    W16 = make_weight(lin, seed=nout)
+    bias = np.random.default_rng(nout).standard_normal(N).astype(np.float16)
+    X, W = to_dev(X16, dev), to_dev(W16, dev)
+    CB, SCB, _ = lib.quantize_rowwise(W, 0.0)
+    Y = lib.matmul_mixed(X, CB, SCB, W if give_w16 else None, 6.0, bias=to_dev(bias, dev), activation=act)
+    r = oracle_mod.matmul_mixed(X16, 6.0, W=W16, use_fp16_weight_cols=give_w16, bias=bias, activation=act)
+    assert r["O"].size == nout
+    y = Y.cpu().numpy().astype(np.float64)
+    pre = r["Y_lin"] + bias.astype(np.float64)[None, :]
+    tol = 1.13 * (1e-2 + 2e-3 * np.abs(pre)) + 5e-4 * np.abs(r["Y"])
+    bad = np.abs(y - r["Y"]) > tol
+    assert not bad.any(), f"{bad.sum()} outside tolerance, worst {np.abs(y - r['Y']).max()}"
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 520, 1040), (4, 640, 1024), (64, 256, 4096), (300, 19000, 384)])
 def test_fp16_weights_mode(lib, dev, oracle_mod, M, N, K):
     """llmint8_matmul_mixed_fp16w quantizes W on every call: its output is
     bit-identical to quantizing W once and calling matmul_mixed_ex, and its
