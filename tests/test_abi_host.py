@@ -57,6 +57,8 @@ def test_workspace_sizes(lib):
     grow = lib.workspace_size(M, 2 * N, K) - lib.workspace_size(M, N, K)
     assert 33 * 4 * N <= grow <= 33 * 4 * N + 1024
     assert lib.workspace_size(32, 2 * N, K) == lib.workspace_size(32, N, K)  # decode shapes have no such copies
+    # from M = 256 (CTA-pair GEMM) the stream-K slots: 80 pairs x 256 KB of int32 partials, and their flags
+    assert lib.workspace_size(256, N, K) - lib.workspace_size(255, N, K) >= 80 * 262144
     assert lib.quantize_workspace_size(M, K) < need
     assert lib.workspace_size(-1, N, K) == 0
 
