@@ -22,6 +22,10 @@
 //               run its main loop.
 // SWAP=true is the decode form (few tokens): W takes the MMA M side (128
 // output features per tile) and the tokens the N side (BN = 16 or 32).
+// From 256 rows of X the CTA-pair form runs instead (k_gemm_i8_pair: 256-row
+// tiles over two CTAs of a cluster, tcgen05.mma.cta_group::2); when its tiles
+// do not fill the last round, the last tiles are split over the pairs by K
+// stages (stream-K, work lists in sched.h) and the int32 parts summed exactly.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
