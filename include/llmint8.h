@@ -178,7 +178,9 @@ typedef struct llmint8_debug {
  * kernel: the outlier columns and codes of X are computed across all SMs
  * while the weight codes already stream in, W is split evenly over the SMs
  * and split tiles are summed exactly in int32. Larger M runs the quantizer
- * and then the persistent prefill GEMM (CTA pairs from M = 256).
+ * and then the persistent prefill GEMM (CTA pairs from M = 256; when the
+ * tiles do not fill the last round, the last ones are split over the pairs
+ * by K and their int32 parts summed exactly through the workspace).
  * Calls that share a workspace must be ordered (one stream, or events).
  */
 LLMINT8_API llmint8_status llmint8_matmul_mixed(const void *X_f16, int64_t M, int64_t K, const int8_t *CB,
